@@ -1,0 +1,83 @@
+// Device-side filler for the synthetic PLE table (input generation only).
+//
+// Fills table u8[2][R][D] (FP8-E4M3 codes, uniform over the 254 finite codes)
+// and scales f32[2][R] (uniform in [0.01, 0.1)) from the counter-based
+// splitmix64 generator (Steele, Lea and Flood, OOPSLA 2014). Element i of
+// stream `tag` is mix(base(seed, tag) + (i + 1) * GAMMA) with
+// base(seed, tag) = mix(seed ^ (tag << 32)). The host generator in
+// ple_inputs/__init__.py implements the same definition; tests compare the two
+// bit for bit on sampled rows. Nothing here computes any part of the layer.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace {
+
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+constexpr uint32_t kTagCodes = 1;
+constexpr uint32_t kTagScales = 2;
+
+__host__ __device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__host__ __device__ __forceinline__ uint64_t stream_base(uint64_t seed, uint32_t tag) {
+  return sm64_mix(seed ^ (static_cast<uint64_t>(tag) << 32));
+}
+
+// Uniform map onto the 254 finite E4M3 codes: i in [0,254), skip 0x7F.
+__device__ __forceinline__ uint32_t draw_code(uint64_t u) {
+  const uint32_t i = static_cast<uint32_t>(((u >> 32) * 254ull) >> 32);
+  return i + (i >= 127u ? 1u : 0u);
+}
+
+__global__ void fill_codes_kernel(uint8_t* __restrict__ table, uint64_t n16, uint64_t base) {
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t c = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < n16; c += stride) {
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint64_t i = c * 16 + q * 4 + b;
+        v |= draw_code(sm64_mix(base + (i + 1) * kGamma)) << (8 * b);
+      }
+      w[q] = v;
+    }
+    reinterpret_cast<uint4*>(table)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+__global__ void fill_scales_kernel(float* __restrict__ scales, uint64_t n, uint64_t base) {
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const uint64_t u = sm64_mix(base + (i + 1) * kGamma);
+    const double f = static_cast<double>(u >> 40) * 0x1p-24;          // exact
+    scales[i] = __double2float_rn(__dadd_rn(0.01, __dmul_rn(0.09, f)));  // no contraction
+  }
+}
+
+}  // namespace
+
+extern "C" uint64_t ple_synth_stream_base(uint64_t seed, uint32_t tag) {
+  return stream_base(seed, tag);
+}
+
+// Returns 0 on success, else the CUDA error code (or cudaErrorInvalidValue for bad sizes).
+extern "C" int ple_synth_fill_table(uint8_t* table, float* scales, int64_t rows_per_order,
+                                    int32_t row_dim, uint64_t seed, cudaStream_t stream) {
+  if (table == nullptr || scales == nullptr || rows_per_order <= 0 || row_dim <= 0 ||
+      (row_dim % 16) != 0 || (reinterpret_cast<uintptr_t>(table) % 16) != 0) {
+    return static_cast<int>(cudaErrorInvalidValue);
+  }
+  const uint64_t nbytes = 2ull * static_cast<uint64_t>(rows_per_order) * static_cast<uint64_t>(row_dim);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  fill_codes_kernel<<<sms * 8, 256, 0, stream>>>(table, nbytes / 16, stream_base(seed, kTagCodes));
+  fill_scales_kernel<<<sms * 2, 256, 0, stream>>>(scales, 2ull * static_cast<uint64_t>(rows_per_order),
+                                                  stream_base(seed, kTagScales));
+  return static_cast<int>(cudaGetLastError());
+}

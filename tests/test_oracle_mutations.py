@@ -1,0 +1,104 @@
+"""Plant plausible mistakes in the CPU oracle and check that a pin catches each.
+
+Every mutation is applied to the oracle on the CPU (monkeypatch) and removed
+after the test; the GPU path is not involved.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import oracle.ple_oracle as OP
+import tests.test_oracle_pins as pins
+
+
+def _fails(fn):
+    try:
+        fn()
+    except (AssertionError, ValueError, IndexError):
+        return True
+    return False
+
+
+def _patch(monkeypatch, name, fn):
+    monkeypatch.setattr(OP, name, fn)
+    monkeypatch.setattr(O, name, fn)
+
+
+def test_reversed_conv_taps_caught(monkeypatch):
+    def bad(u_hist, conv_w):
+        return OP.__dict__["_orig_short_conv"](u_hist, np.asarray(conv_w)[:, ::-1])
+    monkeypatch.setitem(OP.__dict__, "_orig_short_conv", OP.short_conv)
+    _patch(monkeypatch, "short_conv", bad)
+    assert _fails(pins.test_short_conv_matches_numpy_convolve)
+    assert _fails(pins.test_short_conv_delta_is_identity_and_impulse_response)
+
+
+def test_gate_sign_flip_caught(monkeypatch):
+    orig = OP.gate
+    _patch(monkeypatch, "gate", lambda h, w: orig(h, -np.asarray(w, np.float64)))
+    assert _fails(pins.test_gate_sign)
+    assert _fails(pins.test_zero_gate_returns_hidden)
+
+
+def test_dropped_trigram_term_caught(monkeypatch):
+    def bad(x0, x1, x2):
+        k2, _ = OP.__dict__["_orig_keys"](x0, x1, x2)
+        return k2, k2
+    monkeypatch.setitem(OP.__dict__, "_orig_keys", OP.ngram_keys)
+    _patch(monkeypatch, "ngram_keys", bad)
+    assert _fails(pins.test_ids_dependence_structure)
+
+
+def test_swapped_context_index_caught(monkeypatch):
+    orig = OP.ngram_contexts
+
+    def bad(tokens, offsets, hist=None):
+        x0, x1, x2 = orig(tokens, offsets, hist)
+        return x0, x2, x1
+    _patch(monkeypatch, "ngram_contexts", bad)
+    assert _fails(pins.test_ids_dependence_structure)
+
+
+def test_dropped_bigram_context_caught(monkeypatch):
+    def bad(x0, x1, x2):
+        return OP.__dict__["_orig_keys"](x0, 0, x2)
+    monkeypatch.setitem(OP.__dict__, "_orig_keys", OP.ngram_keys)
+    _patch(monkeypatch, "ngram_keys", bad)
+    assert _fails(pins.test_ids_dependence_structure)
+
+
+def test_swapped_history_slots_caught(monkeypatch):
+    orig = OP.ngram_contexts
+
+    def bad(tokens, offsets, hist=None):
+        h = None if hist is None else np.asarray(hist)[:, ::-1]
+        return orig(tokens, offsets, h)
+    _patch(monkeypatch, "ngram_contexts", bad)
+    assert _fails(pins.test_ids_carried_history_equals_whole_sequence)
+
+
+def test_transposed_projection_caught(monkeypatch):
+    _patch(monkeypatch, "project", lambda e, w: np.asarray(e, np.float64) @ np.asarray(w, np.float64).T)
+    assert _fails(pins.test_projection_one_hot_picks_weight_row)
+
+
+def test_missing_order_sum_caught(monkeypatch):
+    def bad(table, ids):
+        ids = np.asarray(ids, dtype=np.int64)
+        return OP.dequantise(table.codes(0, ids[:, 0]), table.scales(0, ids[:, 0]))
+    _patch(monkeypatch, "embed", bad)
+    assert _fails(pins.test_embed_sums_orders)
+
+
+def test_wrong_subnormal_decode_caught(monkeypatch):
+    table = O.E4M3_VALUES.copy()
+    table[1:8] *= 2.0            # subnormals scaled like normals (a classic slip)
+    monkeypatch.setattr(OP, "E4M3_VALUES", table)
+    monkeypatch.setattr(O, "E4M3_VALUES", table)
+    assert _fails(pins.test_e4m3_all_codes_match_torch_float8)
+
+
+@pytest.mark.parametrize("shift", [31, 33])
+def test_wrong_fold_shift_caught_by_brute_force(monkeypatch, shift):
+    _patch(monkeypatch, "fold", lambda k: k ^ (k >> shift))
+    assert _fails(pins.test_layer_matches_brute_force_tiny)
