@@ -1,0 +1,487 @@
+// The C ABI of libple: handle life cycle, host-side argument checks, launch
+// planning and per-stage timing. Every step of the layer runs in the kernels
+// of ple_kernels.cu and ple_gemm.cu; nothing here computes on the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "ple.h"
+#include "ple_device.cuh"
+#include "ple_internal.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kTileM = 128;       // channels per projection tile
+constexpr int kTileK = 64;        // K per pipeline stage
+constexpr int kFusedRows = 256;   // token rows of a fused tile
+constexpr int kHalo = 3;          // conv taps before the current token
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+struct Plan {
+  bool fused;
+  int n_tok, tok_stride, tok_origin, halo, n_tiles, k_splits;
+};
+
+}  // namespace
+
+struct ple_handle {
+  ple_config cfg{};
+  ple_weights w{};
+  int device = 0;
+  int num_sms = 148;
+  __half* w16 = nullptr;
+  __half* e = nullptr;
+  int32_t* ids = nullptr;
+  ple::TokMeta* meta = nullptr;
+  float* partial = nullptr;
+  int64_t partial_elems = 0;
+  float* conv0 = nullptr;
+  int32_t* hist_new = nullptr;
+  int32_t* status = nullptr;
+  EncodeTiledFn encode = nullptr;
+  CUtensorMap tmap_w{};
+  int32_t forward_path = 0;
+  bool profiling = false;
+  struct Rec { int stage; cudaEvent_t a, b; };
+  std::vector<Rec> pending;
+  std::vector<cudaEvent_t> free_events;
+  double stage_ms[PLE_NUM_STAGES] = {0, 0, 0, 0};
+  int64_t stage_launches[PLE_NUM_STAGES] = {0, 0, 0, 0};
+  int64_t launches = 0;
+};
+
+namespace {
+
+Plan plan_projection(const ple_handle* h, int T, int path, int64_t partial_cap) {
+  const int m_tiles = h->cfg.hidden / kTileM;
+  const int num_kb = h->cfg.row_dim / kTileK;
+  const int fused_tiles_n = ceil_div(T, kFusedRows - kHalo);
+  bool fused = (path == 1) || (path == 0 && static_cast<int64_t>(m_tiles) * fused_tiles_n >= h->num_sms);
+  if (!fused) {
+    const int n_tok = std::min(256, ceil_div(T, 16) * 16);
+    const int n_tiles = ceil_div(T, n_tok);
+    const int tiles = m_tiles * n_tiles;
+    int ks = std::max(1, std::min(h->num_sms / std::max(tiles, 1), std::min(num_kb, 16)));
+    while (ks > 1 && static_cast<int64_t>(ks) * T * h->cfg.hidden > partial_cap) --ks;
+    if (static_cast<int64_t>(T) * h->cfg.hidden <= partial_cap)
+      return Plan{false, n_tok, n_tok, 0, 0, n_tiles, ks};
+    fused = true;   // no room for partials: fall back to the fused path
+  }
+  return Plan{true, kFusedRows, kFusedRows - kHalo, -kHalo, kHalo, fused_tiles_n, 1};
+}
+
+cudaEvent_t take_event(ple_handle* h) {
+  if (!h->free_events.empty()) {
+    cudaEvent_t e = h->free_events.back();
+    h->free_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+template <class F>
+ple_status run_stage(ple_handle* h, int stage, cudaStream_t s, F&& launch) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (h->profiling) {
+    a = take_event(h);
+    b = take_event(h);
+    cudaEventRecord(a, s);
+  }
+  const cudaError_t err = launch();
+  if (err != cudaSuccess) return PLE_ERR_CUDA;
+  ++h->launches;
+  if (h->profiling) {
+    cudaEventRecord(b, s);
+    h->pending.push_back({stage, a, b});
+  }
+  return PLE_OK;
+}
+
+bool encode_2d(ple_handle* h, CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = h->encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+void free_all(ple_handle* h) {
+  cudaFree(h->w16);
+  cudaFree(h->e);
+  cudaFree(h->ids);
+  cudaFree(h->meta);
+  cudaFree(h->partial);
+  cudaFree(h->conv0);
+  cudaFree(h->hist_new);
+  cudaFree(h->status);
+  for (auto& r : h->pending) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : h->free_events) cudaEventDestroy(e);
+}
+
+// Runs prepare + gather + projection (+ combine) for a packed batch.
+ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
+                     int32_t uniform_q, const void* hidden, void* out, ple_out_dtype dtype,
+                     const ple_state* state, int32_t* dec_hist, float* dec_conv, const int32_t* n_commit,
+                     cudaStream_t stream) {
+  const ple_config& c = h->cfg;
+  const bool decode = uniform_q > 0;
+  const Plan pl = plan_projection(h, T, decode ? 2 : h->forward_path, h->partial_elems);
+
+  ple::PrepareArgs pa{};
+  pa.tokens = tokens;
+  pa.T = T;
+  pa.offsets = offsets;
+  pa.S = S;
+  pa.uniform_q = uniform_q;
+  pa.hist = decode ? dec_hist : (state ? state->hist : nullptr);
+  pa.vocab = c.vocab;
+  pa.rows0 = c.rows[0];
+  pa.rows1 = c.rows[1];
+  pa.ids = h->ids;
+  pa.hidden = static_cast<const __nv_bfloat16*>(hidden);
+  pa.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
+  pa.H = c.hidden;
+  pa.meta = h->meta;
+  if (!decode && state != nullptr) {
+    pa.conv_in = state->conv;
+    pa.conv_copy = h->conv0;
+    pa.hist_new = h->hist_new;
+  }
+  pa.status = h->status;
+  ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_prepare(pa, stream); });
+  if (st != PLE_OK) return st;
+
+  st = run_stage(h, PLE_STAGE_GATHER, stream, [&] {
+    return ple::launch_gather(h->ids, T, h->w.table, h->w.scales, c.rows[0], c.rows[1], c.row_dim, h->e, false,
+                              stream);
+  });
+  if (st != PLE_OK) return st;
+
+  CUtensorMap tmap_e{}, tmap_h{}, tmap_o{}, tmap_o_head{};
+  if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->e, c.row_dim, T, static_cast<uint64_t>(c.row_dim) * 2,
+                 kTileK, pl.n_tok, CU_TENSOR_MAP_SWIZZLE_128B))
+    return PLE_ERR_CUDA;
+  if (!encode_2d(h, &tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, c.hidden, T,
+                 static_cast<uint64_t>(c.hidden) * 2, kTileM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return PLE_ERR_CUDA;
+
+  if (pl.fused && dtype == PLE_OUT_BF16) {
+    if (!encode_2d(h, &tmap_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, c.hidden, T,
+                   static_cast<uint64_t>(c.hidden) * 2, kTileM, 32, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_2d(h, &tmap_o_head, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, c.hidden, T,
+                   static_cast<uint64_t>(c.hidden) * 2, kTileM, 32 - kHalo, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return PLE_ERR_CUDA;
+  }
+
+  ple::GemmParams gp{};
+  gp.T = T;
+  gp.H = c.hidden;
+  gp.D = c.row_dim;
+  gp.n_tok = pl.n_tok;
+  gp.tok_stride = pl.tok_stride;
+  gp.tok_origin = pl.tok_origin;
+  gp.halo = pl.halo;
+  gp.m_tiles = c.hidden / kTileM;
+  gp.n_tiles = pl.n_tiles;
+  gp.k_splits = pl.k_splits;
+  gp.num_kb = c.row_dim / kTileK;
+  gp.fused = pl.fused ? 1 : 0;
+  gp.meta = h->meta;
+  gp.conv_w = h->w.conv_w;
+  gp.conv0 = (!decode && state) ? h->conv0 : nullptr;
+  gp.conv_state = (!decode && state) ? state->conv : nullptr;
+  gp.hist_state = (!decode && state) ? state->hist : nullptr;
+  gp.hist_new = h->hist_new;
+  gp.out = out;
+  gp.out_f32 = dtype == PLE_OUT_F32 ? 1 : 0;
+  gp.partial = h->partial;
+  gp.status = h->status;
+  const int total = gp.m_tiles * gp.n_tiles * gp.k_splits;
+  const int grid = std::min(total, h->num_sms);
+  st = run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_gemm(h->tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, gp, grid, stream);
+  });
+  if (st != PLE_OK || pl.fused) return st;
+
+  if (decode) {
+    ple::DecodeCombineArgs da{};
+    da.B = S;
+    da.q = uniform_q;
+    da.H = c.hidden;
+    da.k_splits = pl.k_splits;
+    da.partial = h->partial;
+    da.meta = h->meta;
+    da.hidden = static_cast<const __nv_bfloat16*>(hidden);
+    da.conv_w = h->w.conv_w;
+    da.tokens = tokens;
+    da.hist = dec_hist;
+    da.conv_state = dec_conv;
+    da.n_commit = n_commit;
+    da.out = out;
+    da.out_f32 = gp.out_f32;
+    da.status = h->status;
+    return run_stage(h, PLE_STAGE_COMBINE, stream, [&] { return ple::launch_combine_decode(da, stream); });
+  }
+  ple::CombineArgs ca{};
+  ca.T = T;
+  ca.H = c.hidden;
+  ca.k_splits = pl.k_splits;
+  ca.partial = h->partial;
+  ca.meta = h->meta;
+  ca.hidden = static_cast<const __nv_bfloat16*>(hidden);
+  ca.conv_w = h->w.conv_w;
+  ca.conv0 = gp.conv0;
+  ca.conv_state = gp.conv_state;
+  ca.hist_state = gp.hist_state;
+  ca.hist_new = h->hist_new;
+  ca.out = out;
+  ca.out_f32 = gp.out_f32;
+  return run_stage(h, PLE_STAGE_COMBINE, stream, [&] { return ple::launch_combine_forward(ca, stream); });
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ple_status_string(ple_status s) {
+  switch (s) {
+    case PLE_OK: return "ok";
+    case PLE_ERR_INVALID_ARG: return "invalid argument";
+    case PLE_ERR_SHAPE: return "size outside the handle's configuration";
+    case PLE_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case PLE_ERR_RANGE: return "token outside [0, vocab) or inconsistent offsets / n_commit";
+    case PLE_ERR_OOM: return "device allocation failed";
+    case PLE_ERR_CUDA: return "CUDA runtime error";
+    case PLE_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case PLE_ERR_UNSUPPORTED: return "unsupported configuration";
+  }
+  return "unknown status";
+}
+
+ple_status ple_create(const ple_config* config, const ple_weights* weights, cudaStream_t stream, ple_handle** out) {
+  if (config == nullptr || weights == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const ple_config& c = *config;
+  if (c.reserved != 0 || c.vocab <= 0 || c.hidden <= 0 || c.row_dim <= 0 || c.max_tokens <= 0 || c.max_seqs <= 0)
+    return PLE_ERR_INVALID_ARG;
+  if (c.hidden % 128 != 0 || c.row_dim % 64 != 0) return PLE_ERR_UNSUPPORTED;
+  for (int n = 0; n < 2; ++n)
+    if (c.rows[n] <= 0 || c.rows[n] >= (int64_t(1) << 31)) return PLE_ERR_INVALID_ARG;
+  if (weights->table == nullptr || weights->scales == nullptr || weights->w_proj == nullptr ||
+      weights->w_gate == nullptr || weights->conv_w == nullptr)
+    return PLE_ERR_INVALID_ARG;
+  if (!aligned(weights->table, 16) || !aligned(weights->w_proj, 16) || !aligned(weights->w_gate, 16) ||
+      !aligned(weights->conv_w, 16) || !aligned(weights->scales, 4))
+    return PLE_ERR_ALIGN;
+
+  ple_handle* h = new (std::nothrow) ple_handle();
+  if (h == nullptr) return PLE_ERR_OOM;
+  h->cfg = c;
+  h->w = *weights;
+  cudaGetDevice(&h->device);
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    delete h;
+    return PLE_ERR_CUDA;
+  }
+  h->encode = reinterpret_cast<EncodeTiledFn>(fn);
+
+  // partial-sum capacity: whatever the automatic plan needs up to max_tokens, and
+  // at least one split of min(max_tokens, 4096) tokens (forced split-K path)
+  int64_t cap = static_cast<int64_t>(std::min(c.max_tokens, 4096)) * c.hidden;
+  for (int T = 1; T <= c.max_tokens; ++T) {
+    const Plan p = plan_projection(h, T, 0, INT64_MAX);
+    if (p.fused) continue;
+    cap = std::max(cap, static_cast<int64_t>(p.k_splits) * T * c.hidden);
+  }
+  h->partial_elems = cap;
+
+  const int64_t e_rows = std::max<int64_t>(c.max_tokens, 256);
+  bool ok = cudaMalloc(&h->w16, static_cast<size_t>(c.row_dim) * c.hidden * 2) == cudaSuccess &&
+            cudaMalloc(&h->e, static_cast<size_t>(e_rows) * c.row_dim * 2) == cudaSuccess &&
+            cudaMalloc(&h->ids, static_cast<size_t>(c.max_tokens) * 2 * 4) == cudaSuccess &&
+            cudaMalloc(&h->meta, static_cast<size_t>(c.max_tokens) * sizeof(ple::TokMeta)) == cudaSuccess &&
+            cudaMalloc(&h->partial, static_cast<size_t>(cap) * 4) == cudaSuccess &&
+            cudaMalloc(&h->conv0, static_cast<size_t>(c.max_seqs) * 3 * c.hidden * 4) == cudaSuccess &&
+            cudaMalloc(&h->hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess &&
+            cudaMalloc(&h->status, 4) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_all(h);
+    delete h;
+    return PLE_ERR_OOM;
+  }
+  cudaMemsetAsync(h->status, 0, 4, stream);
+  if (ple::launch_convert_w(static_cast<const __nv_bfloat16*>(weights->w_proj), c.row_dim, c.hidden, h->w16,
+                            h->status, stream) != cudaSuccess) {
+    free_all(h);
+    delete h;
+    return PLE_ERR_CUDA;
+  }
+  int32_t bad = 0;
+  if (cudaMemcpyAsync(&bad, h->status, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess) {
+    free_all(h);
+    delete h;
+    return PLE_ERR_CUDA;
+  }
+  if (bad != 0) {
+    free_all(h);
+    delete h;
+    return PLE_ERR_UNSUPPORTED;
+  }
+  if (cudaMemsetAsync(h->status, 0, 4, stream) != cudaSuccess ||
+      !encode_2d(h, &h->tmap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->w16, c.row_dim, c.hidden,
+                 static_cast<uint64_t>(c.row_dim) * 2, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      cudaStreamSynchronize(stream) != cudaSuccess) {
+    free_all(h);
+    delete h;
+    return PLE_ERR_CUDA;
+  }
+  *out = h;
+  return PLE_OK;
+}
+
+ple_status ple_destroy(ple_handle* h) {
+  if (h == nullptr) return PLE_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  free_all(h);
+  delete h;
+  return PLE_OK;
+}
+
+ple_status ple_ngram_ids(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
+                         const int32_t* hist, int32_t* ids, cudaStream_t stream) {
+  if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
+  if (T == 0) return PLE_OK;
+  if (tokens == nullptr || offsets == nullptr || ids == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(tokens, 4) || !aligned(offsets, 4) || !aligned(ids, 8) || (hist && !aligned(hist, 4)))
+    return PLE_ERR_ALIGN;
+  ple::PrepareArgs pa{};
+  pa.tokens = tokens;
+  pa.T = T;
+  pa.offsets = offsets;
+  pa.S = S;
+  pa.hist = hist;
+  pa.vocab = h->cfg.vocab;
+  pa.rows0 = h->cfg.rows[0];
+  pa.rows1 = h->cfg.rows[1];
+  pa.ids = ids;
+  pa.H = h->cfg.hidden;
+  pa.status = h->status;
+  return run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_prepare(pa, stream); });
+}
+
+ple_status ple_gather_rows(ple_handle* h, const int32_t* ids, int32_t T, void* e_out, cudaStream_t stream) {
+  if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (T == 0) return PLE_OK;
+  if (ids == nullptr || e_out == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(ids, 8) || !aligned(e_out, 16)) return PLE_ERR_ALIGN;
+  const ple_config& c = h->cfg;
+  return run_stage(h, PLE_STAGE_GATHER, stream, [&] {
+    return ple::launch_gather(ids, T, h->w.table, h->w.scales, c.rows[0], c.rows[1], c.row_dim,
+                              static_cast<__half*>(e_out), true, stream);
+  });
+}
+
+ple_status ple_forward(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
+                       const void* hidden, void* out, ple_out_dtype out_dtype, const ple_state* state,
+                       cudaStream_t stream) {
+  if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
+  if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
+  if (T == 0) return PLE_OK;
+  if (tokens == nullptr || offsets == nullptr || hidden == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
+  if (out == hidden && out_dtype != PLE_OUT_BF16) return PLE_ERR_INVALID_ARG;
+  if (state != nullptr && (state->hist == nullptr || state->conv == nullptr)) return PLE_ERR_INVALID_ARG;
+  if (!aligned(tokens, 4) || !aligned(offsets, 4) || !aligned(hidden, 16) || !aligned(out, 16) ||
+      (state && (!aligned(state->hist, 4) || !aligned(state->conv, 16))))
+    return PLE_ERR_ALIGN;
+  return run_layer(h, tokens, T, offsets, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, stream);
+}
+
+ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const void* hidden, void* out,
+                           ple_out_dtype out_dtype, int32_t* hist, float* conv_state, const int32_t* n_commit,
+                           cudaStream_t stream) {
+  if (h == nullptr) return PLE_ERR_INVALID_ARG;
+  if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
+  if (B < 1 || q < 1 || B > h->cfg.max_seqs || static_cast<int64_t>(B) * q > h->cfg.max_tokens) return PLE_ERR_SHAPE;
+  if (tokens == nullptr || hidden == nullptr || out == nullptr || hist == nullptr || conv_state == nullptr)
+    return PLE_ERR_INVALID_ARG;
+  if (out == hidden && out_dtype != PLE_OUT_BF16) return PLE_ERR_INVALID_ARG;
+  if (!aligned(tokens, 4) || !aligned(hidden, 16) || !aligned(out, 16) || !aligned(hist, 4) ||
+      !aligned(conv_state, 16) || (n_commit && !aligned(n_commit, 4)))
+    return PLE_ERR_ALIGN;
+  return run_layer(h, tokens, B * q, nullptr, B, q, hidden, out, out_dtype, nullptr, hist, conv_state, n_commit,
+                   stream);
+}
+
+ple_status ple_get_error(ple_handle* h) {
+  if (h == nullptr) return PLE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PLE_ERR_CUDA;
+  int32_t s = 0;
+  if (cudaMemcpy(&s, h->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return PLE_ERR_CUDA;
+  if (cudaMemset(h->status, 0, 4) != cudaSuccess) return PLE_ERR_CUDA;
+  return static_cast<ple_status>(s);
+}
+
+ple_status ple_set_profiling(ple_handle* h, int32_t enable) {
+  if (h == nullptr) return PLE_ERR_INVALID_ARG;
+  h->profiling = enable != 0;
+  return PLE_OK;
+}
+
+ple_status ple_get_stage_times(ple_handle* h, float* ms, int64_t* launches) {
+  if (h == nullptr || ms == nullptr || launches == nullptr) return PLE_ERR_INVALID_ARG;
+  double acc[PLE_NUM_STAGES] = {0, 0, 0, 0};
+  int64_t cnt[PLE_NUM_STAGES] = {0, 0, 0, 0};
+  ple_status st = PLE_OK;
+  for (auto& r : h->pending) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) st = PLE_ERR_CUDA;
+    acc[r.stage] += t;
+    cnt[r.stage] += 1;
+    h->free_events.push_back(r.a);
+    h->free_events.push_back(r.b);
+  }
+  h->pending.clear();
+  for (int i = 0; i < PLE_NUM_STAGES; ++i) {
+    ms[i] = static_cast<float>(acc[i]);
+    launches[i] = cnt[i];
+  }
+  return st;
+}
+
+ple_status ple_set_forward_path(ple_handle* h, int32_t path) {
+  if (h == nullptr || path < 0 || path > 2) return PLE_ERR_INVALID_ARG;
+  h->forward_path = path;
+  return PLE_OK;
+}
+
+int64_t ple_launch_count(const ple_handle* h) { return h ? h->launches : -1; }
+
+}  // extern "C"

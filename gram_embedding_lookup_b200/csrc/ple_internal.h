@@ -1,0 +1,107 @@
+// Host-side declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ple.h"
+
+namespace ple {
+
+struct TokMeta;
+
+// Prepare stage: sequence map, n-gram row IDs, gate, state snapshot.
+struct PrepareArgs {
+  const int32_t* tokens;
+  int32_t T;
+  const int32_t* offsets;      // [S+1]; unused when uniform_q > 0
+  int32_t S;
+  int32_t uniform_q;           // > 0: sequence s covers tokens [s*q, (s+1)*q)
+  const int32_t* hist;         // [S][2] or null
+  int32_t vocab;
+  int64_t rows0, rows1;
+  int32_t* ids;                // [T][2]
+  const __nv_bfloat16* hidden; // [T][H] (null: ids only)
+  const __nv_bfloat16* w_gate; // [H]
+  int32_t H;
+  TokMeta* meta;               // [T] (null: ids only)
+  const float* conv_in;        // [S][3][H] user state (null: none)
+  float* conv_copy;            // [S][3][H] scratch snapshot of conv_in
+  int32_t* hist_new;           // [S][2] state after each sequence (null: none)
+  int32_t* status;
+};
+cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
+
+// Gather stage: e[t] = deq(row of order 0) + deq(row of order 1), fp16.
+cudaError_t launch_gather(const int32_t* ids, int32_t T, const uint8_t* table, const float* scales,
+                          int64_t rows0, int64_t rows1, int32_t D, __half* e, bool reduce_ids,
+                          cudaStream_t stream);
+
+// W_proj bf16 [D][H] -> fp16 [H][D]; *bad set to 1 when a value is outside the fp16 range.
+cudaError_t launch_convert_w(const __nv_bfloat16* w, int32_t D, int32_t H, __half* w16, int32_t* bad,
+                             cudaStream_t stream);
+
+// Projection kernel (tcgen05).
+struct GemmParams {
+  int32_t T, H, D;
+  int32_t n_tok;         // tokens per tile (MMA N): multiple of 16, <= 256
+  int32_t tok_stride;    // token step between consecutive token tiles
+  int32_t tok_origin;    // first token of tile 0 (negative: halo before token 0)
+  int32_t halo;          // leading rows of a tile that are not output (fused mode)
+  int32_t m_tiles, n_tiles, k_splits, num_kb;
+  int32_t fused;         // 1: gate+conv+residual epilogue, 0: write fp32 partials
+  const TokMeta* meta;
+  const float* conv_w;
+  const float* conv0;    // state snapshot [S][3][H] or null (fresh)
+  float* conv_state;     // [S][3][H] written at each sequence's last token, or null
+  int32_t* hist_state;   // [S][2] or null
+  const int32_t* hist_new;
+  void* out;
+  int32_t out_f32;
+  float* partial;        // [k_splits][T][H]
+  int32_t* status;
+};
+constexpr int kGemmSmemBytes = 4 * 16384 + 4 * 32768 + 3 * 8192 + 256 * 16 + 64 + 256 + 1024;
+// tmap_o / tmap_o_head: bf16 output tiles of 32 and of 29 tokens (the first
+// chunk of a fused tile without its halo rows).
+cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_e, const CUtensorMap& tmap_h,
+                        const CUtensorMap& tmap_o, const CUtensorMap& tmap_o_head, const GemmParams& p, int grid,
+                        cudaStream_t stream);
+
+// Combine split-K partials + gate + conv + residual (+ state) for a packed batch.
+struct CombineArgs {
+  int32_t T, H, k_splits;
+  const float* partial;
+  const TokMeta* meta;
+  const __nv_bfloat16* hidden;
+  const float* conv_w;
+  const float* conv0;      // snapshot or null
+  float* conv_state;       // null: no state
+  int32_t* hist_state;
+  const int32_t* hist_new;
+  void* out;
+  int32_t out_f32;
+};
+cudaError_t launch_combine_forward(const CombineArgs& a, cudaStream_t stream);
+
+// Decode-step combine: B sequences of q tokens, commit the first n_commit[b].
+struct DecodeCombineArgs {
+  int32_t B, q, H, k_splits;
+  const float* partial;
+  const TokMeta* meta;
+  const __nv_bfloat16* hidden;
+  const float* conv_w;
+  const int32_t* tokens;   // [B][q]
+  int32_t* hist;           // [B][2] in/out
+  float* conv_state;       // [B][3][H] in/out
+  const int32_t* n_commit; // [B] or null
+  void* out;
+  int32_t out_f32;
+  int32_t* status;
+};
+cudaError_t launch_combine_decode(const DecodeCombineArgs& a, cudaStream_t stream);
+
+}  // namespace ple

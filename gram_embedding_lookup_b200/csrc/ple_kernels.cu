@@ -1,0 +1,359 @@
+// libple kernels other than the projection: the prepare stage (sequence map,
+// n-gram row IDs, sigmoid gate), the row gather with E4M3 dequantisation, the
+// one-time W_proj conversion, and the combine kernels used after a split-K
+// projection (small batches and decode steps).
+//
+// The n-gram definition follows the DGX Spark deployment report
+// ("【Qwen3.8-Flash-Next 端侧部署】01-模型架构与整体方案", section
+// "n-gram embedding 是一条附加的条件记忆路径": IDs from token IDs, positions and
+// sequence boundaries only) and the RTX 3090 llama.cpp report (section
+// "n-gram表格": the last few tokens are hashed into bigram and trigram rows).
+// The concrete hash is the one stated in include/ple.h.
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "ple_device.cuh"
+#include "ple_internal.h"
+
+namespace ple {
+namespace {
+
+constexpr uint64_t kP0 = 0x9E3779B97F4A7C15ull;
+constexpr uint64_t kP1 = 0xC2B2AE3D27D4EB4Full;
+constexpr uint64_t kP2 = 0x165667B19E3779F9ull;
+
+__device__ __forceinline__ uint64_t context_of(int32_t tok) {
+  return static_cast<uint64_t>(static_cast<uint32_t>(tok)) + 1ull;
+}
+
+__device__ __forceinline__ uint64_t fold64(uint64_t k) { return k ^ (k >> 32); }
+
+// ------------------------------------------------------------------ prepare
+constexpr int kPrepWarps = 8;   // one warp per token, 8 tokens per block
+
+__global__ void __launch_bounds__(256) prepare_kernel(const PrepareArgs a, int token_blocks) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (static_cast<int>(blockIdx.x) >= token_blocks) {
+    // ---- state and offsets blocks
+    const int sb = blockIdx.x - token_blocks;
+    const int nsb = gridDim.x - token_blocks;
+    if (sb == 0 && a.uniform_q == 0) {
+      // offsets must start at 0, end at T and be non-decreasing
+      if (threadIdx.x == 0 && (a.offsets[0] != 0 || a.offsets[a.S] != a.T)) set_status(a.status, PLE_ERR_RANGE);
+      for (int s = threadIdx.x; s < a.S; s += blockDim.x)
+        if (a.offsets[s] > a.offsets[s + 1]) set_status(a.status, PLE_ERR_RANGE);
+    }
+    if (a.conv_in != nullptr) {
+      const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
+      const float4* src = reinterpret_cast<const float4*>(a.conv_in);
+      float4* dst = reinterpret_cast<float4*>(a.conv_copy);
+      for (int64_t i = static_cast<int64_t>(sb) * blockDim.x + threadIdx.x; i < n4;
+           i += static_cast<int64_t>(nsb) * blockDim.x)
+        dst[i] = src[i];
+    }
+    if (a.hist_new != nullptr && sb == 0) {
+      for (int s = threadIdx.x; s < a.S; s += blockDim.x) {
+        int32_t begin, end;
+        if (a.uniform_q > 0) { begin = s * a.uniform_q; end = begin + a.uniform_q; }
+        else { begin = a.offsets[s]; end = a.offsets[s + 1]; }
+        end = min(max(end, 0), a.T);
+        begin = min(max(begin, 0), end);
+        const int32_t len = end - begin;
+        const int32_t h0 = a.hist ? a.hist[2 * s] : -1;
+        const int32_t h1 = a.hist ? a.hist[2 * s + 1] : -1;
+        int32_t n0, n1;
+        if (len >= 2) { n0 = a.tokens[end - 2]; n1 = a.tokens[end - 1]; }
+        else if (len == 1) { n0 = h1; n1 = a.tokens[end - 1]; }
+        else { n0 = h0; n1 = h1; }
+        a.hist_new[2 * s] = n0;
+        a.hist_new[2 * s + 1] = n1;
+      }
+    }
+    return;
+  }
+
+  const int t = blockIdx.x * kPrepWarps + warp;
+  if (t >= a.T) return;
+
+  // ---- sequence and position (every lane computes the same values)
+  int32_t s, pos, last;
+  if (a.uniform_q > 0) {
+    s = t / a.uniform_q;
+    pos = t - s * a.uniform_q;
+    last = (pos == a.uniform_q - 1);
+  } else {
+    int lo = 0, hi = a.S - 1;
+    while (lo < hi) {                         // largest s with offsets[s] <= t
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.offsets[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    s = lo;
+    const int32_t begin = a.offsets[s];
+    const int32_t end = a.offsets[s + 1];
+    pos = t - begin;
+    if (pos < 0 || t >= end) {                // inconsistent offsets: keep every access in bounds
+      if (lane == 0) set_status(a.status, PLE_ERR_RANGE);
+      pos = max(0, min(pos, t));
+    }
+    last = (t == end - 1);
+  }
+
+  // ---- n-gram contexts, keys and rows
+  const int32_t tok = a.tokens[t];
+  if (lane == 0 && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
+  const uint64_t x0 = context_of(tok);
+  auto carried = [&](int k) -> uint64_t {     // the token k places before the sequence start
+    if (a.hist == nullptr) return 0ull;
+    const int32_t h = a.hist[2 * s + (2 - k)];
+    return h < 0 ? 0ull : context_of(h);
+  };
+  const uint64_t x1 = pos >= 1 ? context_of(a.tokens[t - 1]) : carried(1);
+  const uint64_t x2 = pos >= 2 ? context_of(a.tokens[t - 2]) : (pos == 1 ? carried(1) : carried(2));
+  const uint64_t k2 = (x0 * kP0) ^ (x1 * kP1);
+  const uint64_t k3 = k2 ^ (x2 * kP2);
+  if (lane == 0) {
+    const int32_t r0 = static_cast<int32_t>(fold64(k2) % static_cast<uint64_t>(a.rows0));
+    const int32_t r1 = static_cast<int32_t>(fold64(k3) % static_cast<uint64_t>(a.rows1));
+    reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
+  }
+  if (a.meta == nullptr) return;
+
+  // ---- gate: g = sigmoid(w_gate . h_t), fp32 accumulation, warp reduction
+  const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+  const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+  float acc = 0.f;
+  for (int j = lane; j < a.H / 8; j += 32) {
+    const uint4 hv = hrow[j];
+    const uint4 wv = __ldg(wg + j);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hv);
+    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 hf = __bfloat1622float2(h2[q]);
+      const float2 wf = __bfloat1622float2(w2[q]);
+      acc = fmaf(hf.x, wf.x, acc);
+      acc = fmaf(hf.y, wf.y, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    TokMeta m;
+    m.g = 1.0f / (1.0f + expf(-acc));
+    m.seq = s;
+    m.pos = pos;
+    m.flags = last ? kFlagLast : 0;
+    a.meta[t] = m;
+  }
+}
+
+// ------------------------------------------------------------------ gather
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu),
+                                                     __NV_E4M3);
+  __half2 h;
+  h = *reinterpret_cast<const __half2*>(&hr);
+  return __half22float2(h);
+}
+
+// e = a*s0 + b*s1 for 4 codes per word, 16 codes per thread -> 16 fp16.
+__device__ __forceinline__ uint32_t combine_pair(uint32_t wa, uint32_t wb, int shift, float s0, float s1) {
+  const float2 a = e4m3x2_to_float2(wa >> shift);
+  const float2 b = e4m3x2_to_float2(wb >> shift);
+  const __half2 r = __floats2half2_rn(fmaf(a.x, s0, b.x * s1), fmaf(a.y, s0, b.y * s1));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ ids, int32_t T,
+                                                     const uint8_t* __restrict__ table,
+                                                     const float* __restrict__ scales, int64_t rows0,
+                                                     int64_t rows1, int32_t D, __half* __restrict__ e,
+                                                     int reduce_ids) {
+  const int chunks = D >> 4;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= static_cast<int64_t>(T) * chunks) return;
+  const int32_t t = static_cast<int32_t>(g / chunks);
+  const int32_t c = static_cast<int32_t>(g - static_cast<int64_t>(t) * chunks);
+  int2 id = ids[t];
+  if (reduce_ids) {
+    id.x = static_cast<int32_t>(static_cast<uint32_t>(id.x) % static_cast<uint32_t>(rows0));
+    id.y = static_cast<int32_t>(static_cast<uint32_t>(id.y) % static_cast<uint32_t>(rows1));
+  }
+  const int64_t row0 = id.x;
+  const int64_t row1 = rows0 + id.y;
+  const uint4 a = ld_stream_v4(table + row0 * D + c * 16);
+  const uint4 b = ld_stream_v4(table + row1 * D + c * 16);
+  const float s0 = __ldg(scales + row0);
+  const float s1 = __ldg(scales + row1);
+  uint4 o0, o1;
+  o0.x = combine_pair(a.x, b.x, 0, s0, s1);
+  o0.y = combine_pair(a.x, b.x, 16, s0, s1);
+  o0.z = combine_pair(a.y, b.y, 0, s0, s1);
+  o0.w = combine_pair(a.y, b.y, 16, s0, s1);
+  o1.x = combine_pair(a.z, b.z, 0, s0, s1);
+  o1.y = combine_pair(a.z, b.z, 16, s0, s1);
+  o1.z = combine_pair(a.w, b.w, 0, s0, s1);
+  o1.w = combine_pair(a.w, b.w, 16, s0, s1);
+  uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D + c * 16);
+  dst[0] = o0;
+  dst[1] = o1;
+}
+
+// ------------------------------------------------------------------ W_proj conversion
+__global__ void convert_w_kernel(const __nv_bfloat16* __restrict__ w, int32_t D, int32_t H,
+                                 __half* __restrict__ w16, int32_t* bad) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int k = k0 + i, j = j0 + threadIdx.x;
+    float v = 0.f;
+    if (k < D && j < H) v = __bfloat162float(w[static_cast<int64_t>(k) * H + j]);
+    if (!(fabsf(v) <= 65504.f)) atomicExch(bad, 1);   // also catches NaN
+    tile[i][threadIdx.x] = v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int j = j0 + i, k = k0 + threadIdx.x;
+    if (k < D && j < H) w16[static_cast<int64_t>(j) * D + k] = __float2half_rn(tile[threadIdx.x][i]);
+  }
+}
+
+// ------------------------------------------------------------------ combine (packed batch)
+__device__ __forceinline__ void store_out(void* out, int32_t out_f32, int64_t idx, float v) {
+  if (out_f32) reinterpret_cast<float*>(out)[idx] = v;
+  else reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
+}
+
+__global__ void __launch_bounds__(128) combine_forward_kernel(const CombineArgs a) {
+  const int32_t t = blockIdx.y;
+  const int32_t j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= a.H || t >= a.T) return;
+  const TokMeta mt = a.meta[t];
+  float u[4];                          // u[k] = u_{t-3+k}
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int lag = 3 - k;
+    if (mt.pos - lag >= 0) {
+      const int32_t tk = t - lag;
+      float v = 0.f;
+      for (int sp = 0; sp < a.k_splits; ++sp)
+        v += a.partial[(static_cast<int64_t>(sp) * a.T + tk) * a.H + j];
+      u[k] = a.meta[tk].g * v;
+    } else {
+      u[k] = a.conv0 ? a.conv0[(static_cast<int64_t>(mt.seq) * 3 + (3 + mt.pos - lag)) * a.H + j] : 0.f;
+    }
+  }
+  const float4 cw = reinterpret_cast<const float4*>(a.conv_w)[j];
+  const float y = cw.x * u[0] + cw.y * u[1] + cw.z * u[2] + cw.w * u[3];
+  const int64_t idx = static_cast<int64_t>(t) * a.H + j;
+  store_out(a.out, a.out_f32, idx, __bfloat162float(a.hidden[idx]) + y);
+  if (a.conv_state != nullptr && (mt.flags & kFlagLast)) {
+    float* cs = a.conv_state + static_cast<int64_t>(mt.seq) * 3 * a.H + j;
+    cs[0] = u[1];
+    cs[a.H] = u[2];
+    cs[2 * a.H] = u[3];
+    if (j == 0) {
+      a.hist_state[2 * mt.seq] = a.hist_new[2 * mt.seq];
+      a.hist_state[2 * mt.seq + 1] = a.hist_new[2 * mt.seq + 1];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ combine (decode step)
+__global__ void __launch_bounds__(128) combine_decode_kernel(const DecodeCombineArgs a) {
+  const int32_t b = blockIdx.y;
+  const int32_t j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= a.H || b >= a.B) return;
+  int32_t nc = a.n_commit ? a.n_commit[b] : a.q;
+  if (nc < 1 || nc > a.q) {
+    if (j == 0) set_status(a.status, PLE_ERR_RANGE);
+    nc = max(1, min(nc, a.q));
+  }
+  float* cs = a.conv_state + static_cast<int64_t>(b) * 3 * a.H + j;
+  float w0 = cs[0], w1 = cs[a.H], w2 = cs[2 * a.H];
+  float c0 = w0, c1 = w1, c2 = w2;
+  const float4 cw = reinterpret_cast<const float4*>(a.conv_w)[j];
+  for (int i = 0; i < a.q; ++i) {
+    const int32_t t = b * a.q + i;
+    const int32_t T = a.B * a.q;
+    float v = 0.f;
+    for (int sp = 0; sp < a.k_splits; ++sp) v += a.partial[(static_cast<int64_t>(sp) * T + t) * a.H + j];
+    const float u = a.meta[t].g * v;
+    const float y = cw.x * w0 + cw.y * w1 + cw.z * w2 + cw.w * u;
+    w0 = w1; w1 = w2; w2 = u;
+    const int64_t idx = static_cast<int64_t>(t) * a.H + j;
+    store_out(a.out, a.out_f32, idx, __bfloat162float(a.hidden[idx]) + y);
+    if (i == nc - 1) { c0 = w0; c1 = w1; c2 = w2; }
+  }
+  cs[0] = c0;
+  cs[a.H] = c1;
+  cs[2 * a.H] = c2;
+  if (j == 0) {
+    // last two committed tokens, taking carried ones when fewer than two were committed
+    const int32_t* tk = a.tokens + static_cast<int64_t>(b) * a.q;
+    const int32_t h0 = a.hist[2 * b], h1 = a.hist[2 * b + 1];
+    const int32_t n1 = tk[nc - 1];
+    const int32_t n0 = nc >= 2 ? tk[nc - 2] : h1;
+    (void)h0;
+    a.hist[2 * b] = n0;
+    a.hist[2 * b + 1] = n1;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
+  const int token_blocks = (a.T + kPrepWarps - 1) / kPrepWarps;
+  int state_blocks = 1;
+  if (a.conv_in != nullptr) {
+    const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
+    const int64_t want = (n4 + 255) / 256;
+    state_blocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
+  }
+  prepare_kernel<<<token_blocks + state_blocks, 256, 0, stream>>>(a, token_blocks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const int32_t* ids, int32_t T, const uint8_t* table, const float* scales,
+                          int64_t rows0, int64_t rows1, int32_t D, __half* e, bool reduce_ids,
+                          cudaStream_t stream) {
+  const int64_t threads = static_cast<int64_t>(T) * (D / 16);
+  const int blocks = static_cast<int>((threads + 255) / 256);
+  gather_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const int2*>(ids), T, table, scales, rows0,
+                                            rows1, D, e, reduce_ids ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert_w(const __nv_bfloat16* w, int32_t D, int32_t H, __half* w16, int32_t* bad,
+                             cudaStream_t stream) {
+  dim3 grid((H + 31) / 32, (D + 31) / 32), block(32, 8);
+  convert_w_kernel<<<grid, block, 0, stream>>>(w, D, H, w16, bad);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_forward(const CombineArgs& a, cudaStream_t stream) {
+  dim3 grid((a.H + 127) / 128, a.T);
+  combine_forward_kernel<<<grid, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_decode(const DecodeCombineArgs& a, cudaStream_t stream) {
+  dim3 grid((a.H + 127) / 128, a.B);
+  combine_decode_kernel<<<grid, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ple

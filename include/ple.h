@@ -1,0 +1,182 @@
+/*
+ * libple — the n-gram embedding ("PLE") layer of Qwen3.8 Flash-Next on one B200.
+ *
+ * What the layer computes is described in the DGX Spark deployment report
+ * ("【Qwen3.8-Flash-Next 端侧部署】01-模型架构与整体方案", section
+ * "n-gram embedding 是一条附加的条件记忆路径"): from raw token IDs,
+ * positions and sequence boundaries the engine derives n-gram IDs, reads the
+ * matching rows of a large FP8 table, and the rows go through
+ * dequantisation, projection, gating and a short convolution before they are
+ * merged into the hidden states. The RTX 3090 llama.cpp report (section
+ * "n-gram表格") adds that rows are keyed by hashing the last few tokens,
+ * bigram and trigram entries, and depend only on the text.
+ *
+ * The pages leave the hash, the scale layout and the gate open; this library
+ * fixes them as follows (all arithmetic is integer or IEEE fp32 unless noted):
+ *   context  x = (uint64)(uint32)token + 1; 0 for a position before the
+ *            sequence start with no carried history (a carried entry < 0 is
+ *            absent). Every token gets one bigram row and one trigram row.
+ *   keys     k2 = x_t*0x9E3779B97F4A7C15 ^ x_{t-1}*0xC2B2AE3D27D4EB4F,
+ *            k3 = k2 ^ x_{t-2}*0x165667B19E3779F9   (wrap-around mod 2^64)
+ *   rows     row_n = (k_n ^ (k_n >> 32)) mod rows[n]  (unsigned 64-bit)
+ *   embed    e_t[k] = E4M3(table[0][row_2][k])*scales[0][row_2]
+ *                   + E4M3(table[1][row_3][k])*scales[1][row_3]
+ *   project  v_t = e_t W_proj            (W_proj bf16 [row_dim][hidden])
+ *   gate     g_t = sigmoid(w_gate . h_t) (one scalar per token)
+ *   conv     y_t[j] = sum_{k=0..3} conv_w[j][k] * u_{t-3+k}[j],  u = g v,
+ *            u before a fresh sequence = 0, else the carried state
+ *   residual out_t = h_t + y_t
+ *
+ * Precision: the GPU rounds e_t to fp16 (computed in fp32) and multiplies it
+ * with an fp16 copy of W_proj on the tensor cores with fp32 accumulation;
+ * everything after the projection is fp32. Against a float64 evaluation the
+ * fp32 output stays within max |err| 2e-2 and relative L2 error 1e-3 on the
+ * workloads the tests cover.
+ *
+ * Conventions for every call below:
+ *   - pointers are DEVICE pointers unless stated otherwise; all calls are
+ *     asynchronous and ordered on the given stream (cudaStream_t, 0 = legacy);
+ *   - argument errors are detected on the host before anything is launched,
+ *     and the call returns the error without side effects;
+ *   - errors that only the device can see (token outside [0, vocab),
+ *     inconsistent offsets, an internal wait that ran out) set a sticky status
+ *     word in the handle, read and cleared by ple_get_error();
+ *   - a handle is used by one stream at a time.
+ */
+#ifndef PLE_H_
+#define PLE_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PLE_OK = 0,
+  PLE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum, forbidden aliasing */
+  PLE_ERR_SHAPE = 2,         /* a size is outside what the handle was created for */
+  PLE_ERR_ALIGN = 3,         /* a pointer is not 16-byte aligned */
+  PLE_ERR_RANGE = 4,         /* (device) token outside [0, vocab) or inconsistent offsets */
+  PLE_ERR_OOM = 5,           /* device allocation failed in ple_create */
+  PLE_ERR_CUDA = 6,          /* a CUDA runtime call failed */
+  PLE_ERR_TIMEOUT = 7,       /* (device) a bounded internal wait ran out; outputs invalid */
+  PLE_ERR_UNSUPPORTED = 8    /* configuration the kernels do not support (e.g. |W_proj| > 65504) */
+} ple_status;
+
+typedef enum { PLE_OUT_BF16 = 0, PLE_OUT_F32 = 1 } ple_out_dtype;
+
+/* Sizes fixed at creation. hidden % 128 == 0, row_dim % 64 == 0,
+ * 0 < rows[n] < 2^31. max_tokens bounds T of every call (and B*q of a decode
+ * step); max_seqs bounds S (and B). */
+typedef struct {
+  int32_t vocab;
+  int32_t hidden;
+  int32_t row_dim;
+  int32_t max_tokens;
+  int32_t max_seqs;
+  int32_t reserved;          /* must be 0 */
+  int64_t rows[2];           /* rows of the bigram (0) and trigram (1) sub-tables */
+} ple_config;
+
+/* Parameters. All are BORROWED: they must stay valid and unchanged for the
+ * handle's lifetime, except w_proj, which is read once by ple_create. */
+typedef struct {
+  const uint8_t* table;      /* FP8-E4M3 codes; sub-table n, row r at byte offset
+                                (n*rows[0] + r)*row_dim  (so [2][rows][row_dim]
+                                when rows[0] == rows[1]); 16-byte aligned */
+  const float* scales;       /* fp32 per-row scales; sub-table n, row r at n*rows[0] + r */
+  const void* w_proj;        /* bf16 [row_dim][hidden], row-major */
+  const void* w_gate;        /* bf16 [hidden] */
+  const float* conv_w;       /* fp32 [hidden][4]; tap 3 multiplies the current token */
+} ple_weights;
+
+/* Per-sequence carried state (caller-owned, device memory). */
+typedef struct {
+  int32_t* hist;             /* [S][2]: token t-2, token t-1 before the sequence; < 0 = absent */
+  float* conv;               /* [S][3][hidden]: u_{t-3}, u_{t-2}, u_{t-1} */
+} ple_state;
+
+typedef struct ple_handle ple_handle;
+
+/* Creates a handle on the current device. Allocates the handle's own device
+ * memory (an fp16 K-major copy of W_proj and scratch sized by max_tokens and
+ * max_seqs) and converts W_proj on `stream`; synchronises `stream`.
+ * Returns PLE_ERR_UNSUPPORTED if some |W_proj| exceeds the fp16 range. */
+ple_status ple_create(const ple_config* config, const ple_weights* weights,
+                      cudaStream_t stream, ple_handle** out);
+
+/* Frees the handle and its device memory (synchronises the device first). */
+ple_status ple_destroy(ple_handle* handle);
+
+/* N-gram row IDs only. tokens int32 [T]; offsets int32 [S+1] with
+ * offsets[0] = 0, offsets[S] = T, non-decreasing (sequence s covers
+ * [offsets[s], offsets[s+1])); hist int32 [S][2] or NULL (all absent);
+ * ids int32 [T][2] receives (bigram row, trigram row), each in [0, rows[n]). */
+ple_status ple_ngram_ids(ple_handle* handle, const int32_t* tokens, int32_t T,
+                         const int32_t* offsets, int32_t S, const int32_t* hist,
+                         int32_t* ids, cudaStream_t stream);
+
+/* The gather stage alone: e_out fp16 [T][row_dim] receives e_t (see top of
+ * file) for the given row IDs int32 [T][2]. IDs must be in range (the call
+ * reduces them mod rows[n] so that no access leaves the table). */
+ple_status ple_gather_rows(ple_handle* handle, const int32_t* ids, int32_t T,
+                           void* e_out, cudaStream_t stream);
+
+/* The layer on a packed batch (prefill or one chunk of a chunked prefill).
+ * hidden bf16 [T][hidden]; out [T][hidden] of `out_dtype`, may equal hidden
+ * only with PLE_OUT_BF16 (in-place residual add). state == NULL: every
+ * sequence starts fresh and no state is written. Otherwise state->hist and
+ * state->conv ([S] entries) are read as the state before each sequence and
+ * overwritten with the state after it (unchanged for an empty sequence).
+ * T == 0 is allowed and does nothing. */
+ple_status ple_forward(ple_handle* handle, const int32_t* tokens, int32_t T,
+                       const int32_t* offsets, int32_t S, const void* hidden, void* out,
+                       ple_out_dtype out_dtype, const ple_state* state, cudaStream_t stream);
+
+/* One decode / speculative-verify step: B sequences with q new tokens each.
+ * tokens int32 [B][q]; hidden bf16 [B*q][hidden]; out [B*q][hidden];
+ * hist int32 [B][2] and conv_state fp32 [B][3][hidden] are read and updated.
+ * Outputs are computed for all q tokens; the state advances by the first
+ * n_commit[b] tokens of sequence b (1 <= n_commit[b] <= q; NULL means q),
+ * i.e. accepted draft tokens are committed and rejected ones rolled back. */
+ple_status ple_decode_step(ple_handle* handle, const int32_t* tokens, int32_t B, int32_t q,
+                           const void* hidden, void* out, ple_out_dtype out_dtype,
+                           int32_t* hist, float* conv_state, const int32_t* n_commit,
+                           cudaStream_t stream);
+
+/* Synchronises the device, returns the sticky device status and clears it. */
+ple_status ple_get_error(ple_handle* handle);
+
+/* Static description of a status code. */
+const char* ple_status_string(ple_status status);
+
+/* ---- measurement and test controls -------------------------------------- */
+
+/* Kernel stages of the library, in launch order within a call. */
+enum { PLE_STAGE_PREPARE = 0, PLE_STAGE_GATHER = 1, PLE_STAGE_GEMM = 2, PLE_STAGE_COMBINE = 3,
+       PLE_NUM_STAGES = 4 };
+
+/* enable != 0: record CUDA events around every kernel the handle launches
+ * (on the call's stream) so that ple_get_stage_times can report them. */
+ple_status ple_set_profiling(ple_handle* handle, int32_t enable);
+
+/* Synchronises the recorded events and writes, per stage, the summed kernel
+ * time in milliseconds (ms[PLE_NUM_STAGES]) and the number of launches
+ * (launches[PLE_NUM_STAGES]) since the last call; then resets the counters. */
+ple_status ple_get_stage_times(ple_handle* handle, float* ms, int64_t* launches);
+
+/* Path selection for ple_forward: 0 = automatic, 1 = fused epilogue
+ * (gate, conv and residual inside the projection kernel, conv halo
+ * recomputed per tile), 2 = split-K projection followed by a combine kernel. */
+ple_status ple_set_forward_path(ple_handle* handle, int32_t path);
+
+/* Total number of kernels the handle has launched since creation. */
+int64_t ple_launch_count(const ple_handle* handle);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PLE_H_ */

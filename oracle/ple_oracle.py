@@ -260,7 +260,7 @@ def ple_forward(tokens, offsets, hidden_bits, w_proj_bits, w_gate_bits, conv_w, 
     rows those outputs depend on are gathered and projected.
 
     Returns a dict: ``ids`` [T][2]; ``out`` float64 [len(sample) or T][H];
-    ``hist_out`` [S][2] and ``conv_out`` [S][3][H] (the end state, full runs only).
+    ``hist_out`` [S][2] and ``conv_out`` [S][3][H] (the state after each sequence).
     """
     tokens = np.asarray(tokens).reshape(-1)
     offsets = np.asarray(offsets, dtype=np.int64)
@@ -272,12 +272,16 @@ def ple_forward(tokens, offsets, hidden_bits, w_proj_bits, w_gate_bits, conv_w, 
     conv0 = np.zeros((S, 3, H)) if conv_state is None else np.asarray(conv_state, np.float64)
 
     want = np.arange(T) if sample is None else np.asarray(sample, dtype=np.int64)
-    # tokens whose u is needed: each wanted token and up to 3 predecessors in its sequence
+    # tokens whose u is needed: each wanted token and up to 3 predecessors in its
+    # sequence, and the last 3 tokens of every sequence (for the end state)
     need = set()
     for t in want:
         for k in range(4):
             if pos[t] - k >= 0:
                 need.add(int(t) - k)
+    for s in range(S):
+        for t in range(max(int(offsets[s]), int(offsets[s + 1]) - 3), int(offsets[s + 1])):
+            need.add(t)
     need = np.array(sorted(need), dtype=np.int64)
     idx_of = {int(t): i for i, t in enumerate(need)}
 
@@ -300,9 +304,10 @@ def ple_forward(tokens, offsets, hidden_bits, w_proj_bits, w_gate_bits, conv_w, 
         y = short_conv(window, conv_w)[0]
         out[i] = bf16_bits_to_f64(np.asarray(hidden_bits)[t]) + y
 
+    u_full = np.zeros((T, H))
+    u_full[need] = u
     res = dict(ids=ids, out=out)
-    if sample is None:
-        res["hist_out"], res["conv_out"] = end_state(tokens, offsets, u, hist, conv0)
+    res["hist_out"], res["conv_out"] = end_state(tokens, offsets, u_full, hist, conv0)
     return res
 
 

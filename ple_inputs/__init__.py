@@ -281,8 +281,9 @@ def mtp_session(w: Workload, steps=None, B=None, q=None, prefix=None):
 
     Returns a dict with the prompts (int32 [B][prefix]), and per step the tokens
     int32 [B][q], hidden bf16 bits [B*q][H] and n_commit int32 [B].
-    The first ``shared`` sequences share one Zipf prompt and identical
-    continuations (duplicated greedy requests); the rest are independent Zipf.
+    The first ``shared`` sequences share one Zipf prompt, identical
+    continuations and identical hidden states (duplicated greedy requests);
+    the rest are independent Zipf.
     n_commit = 1 + Bern(0.70) * (1 + Bern(0.45)) per sequence and step, from the
     per-position draft acceptance measured on the kipfel.ltd page (section 6).
     """
@@ -295,7 +296,9 @@ def mtp_session(w: Workload, steps=None, B=None, q=None, prefix=None):
     rng = np.random.default_rng([w.seed, 17])
     prompts = tokens_zipf(rng, B * prefix, w.vocab).reshape(B, prefix)
     prompts[:shared] = prompts[0]
-    prompt_hidden = hidden_bf16(rng, B * prefix, w.hidden)
+    prompt_hidden = hidden_bf16(rng, B * prefix, w.hidden).reshape(B, prefix, w.hidden)
+    prompt_hidden[:shared] = prompt_hidden[0]
+    prompt_hidden = prompt_hidden.reshape(B * prefix, w.hidden)
     out_steps = []
     for _ in range(steps):
         toks = tokens_zipf(rng, B * q, w.vocab).reshape(B, q)
@@ -305,8 +308,9 @@ def mtp_session(w: Workload, steps=None, B=None, q=None, prefix=None):
         n_commit = (1 + acc1 * (1 + acc2)).astype(np.int32)
         n_commit[:shared] = n_commit[0]
         n_commit = np.minimum(n_commit, q)
-        hid = hidden_bf16(rng, B * q, w.hidden)
-        out_steps.append((toks, hid, n_commit))
+        hid = hidden_bf16(rng, B * q, w.hidden).reshape(B, q, w.hidden)
+        hid[:shared] = hid[0]                 # duplicated requests see identical hidden states
+        out_steps.append((toks, hid.reshape(B * q, w.hidden), n_commit))
     return dict(prompts=prompts, prompt_hidden=prompt_hidden, steps=out_steps)
 
 

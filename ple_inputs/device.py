@@ -1,0 +1,61 @@
+"""Device-resident synthetic inputs for the GPU tests and the benchmark.
+
+Allocates the synthetic table, scales and weights of a workload in device
+memory (torch is used only to allocate and to copy), fills the table with the
+device generator, and creates a libple handle over them. Nothing here computes
+any part of the layer.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import gram_embedding_lookup_b200 as ple
+from . import Workload, fill_table_device
+
+
+def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """bf16 bit patterns (uint16 ndarray) -> torch.bfloat16 tensor on `device`."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device) if device is not None else t
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+class DeviceLayer:
+    """A workload's table and weights on the current device, plus a libple handle."""
+
+    def __init__(self, w: Workload, max_tokens: int, max_seqs: int, weights=None, stream=None):
+        self.w = w
+        R, D, H = w.rows_per_order, w.row_dim, w.hidden
+        self.table = torch.empty(2 * R * D, dtype=torch.uint8, device="cuda")
+        self.scales = torch.empty(2 * R, dtype=torch.float32, device="cuda")
+        s = torch.cuda.current_stream() if stream is None else stream
+        fill_table_device(self.table.data_ptr(), self.scales.data_ptr(), R, D, w.table_seed, s.cuda_stream)
+        self.host_weights = weights if weights is not None else w.weights()
+        self.w_proj = bf16_tensor(self.host_weights.w_proj)
+        self.w_gate = bf16_tensor(self.host_weights.w_gate)
+        self.conv_w = torch.from_numpy(np.ascontiguousarray(self.host_weights.conv_w, np.float32)).cuda()
+        cfg = ple.PleConfig()
+        cfg.vocab, cfg.hidden, cfg.row_dim = w.vocab, H, D
+        cfg.max_tokens, cfg.max_seqs, cfg.reserved = max_tokens, max_seqs, 0
+        cfg.rows[0] = R
+        cfg.rows[1] = R
+        self.config = cfg
+        pw = ple.PleWeights(self.table.data_ptr(), self.scales.data_ptr(), self.w_proj.data_ptr(),
+                            self.w_gate.data_ptr(), self.conv_w.data_ptr())
+        self.weights = pw
+        self.handle = ple.ple_create(cfg, pw, s.cuda_stream)
+
+    def close(self):
+        if self.handle:
+            ple.ple_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
