@@ -16,13 +16,15 @@ __all__ = [
     "PleError", "PleConfig", "PleWeights", "PleState", "lib", "ple_create", "ple_destroy",
     "ple_ngram_ids", "ple_gather_rows", "ple_forward", "ple_decode_step", "ple_get_error",
     "ple_status_string", "ple_set_profiling", "ple_get_stage_times", "ple_set_forward_path",
-    "ple_launch_count", "PLE_OUT_BF16", "PLE_OUT_F32", "STATUS", "STAGES", "LIB_PATH",
+    "ple_launch_count", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32", "STATUS",
+    "STAGES", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libple.so")
 
 PLE_OUT_BF16 = 0
 PLE_OUT_F32 = 1
+PLE_STATIC_MAX_TOKENS = 16384   # the fixed row-ID array of ple_embed_static
 STATUS = {0: "PLE_OK", 1: "PLE_ERR_INVALID_ARG", 2: "PLE_ERR_SHAPE", 3: "PLE_ERR_ALIGN", 4: "PLE_ERR_RANGE",
           5: "PLE_ERR_OOM", 6: "PLE_ERR_CUDA", 7: "PLE_ERR_TIMEOUT", 8: "PLE_ERR_UNSUPPORTED"}
 STAGES = ("prepare", "gather", "gemm", "combine")
@@ -75,6 +77,8 @@ def lib() -> ctypes.CDLL:
             "ple_get_stage_times": ([_VP, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int64)], _I32),
             "ple_set_forward_path": ([_VP, _I32], _I32),
             "ple_launch_count": ([_VP], ctypes.c_int64),
+            "ple_embed_static": ([_VP, _I32, _VP, _I32, _VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, _I32, _I32,
+                                  _VP, _VP, _VP], _I32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -174,3 +178,16 @@ def ple_set_forward_path(handle, path: int) -> None:
 
 def ple_launch_count(handle) -> int:
     return int(lib().ple_launch_count(handle))
+
+
+def ple_embed_static(tokens, T, offsets, S, hist, table, scales, rows0, rows1, row_dim, vocab, e_out,
+                     status_out=None, stream=None) -> None:
+    """N-gram row IDs and row gather into e_out (fp16 [T][row_dim]) without any
+    device allocation, for callers that cannot allocate: the row IDs go to a
+    fixed array in the library (at most PLE_STATIC_MAX_TOKENS tokens per call,
+    one call at a time per device; see include/ple.h)."""
+    if T > PLE_STATIC_MAX_TOKENS:
+        raise ValueError(f"ple_embed_static takes at most {PLE_STATIC_MAX_TOKENS} tokens per call, got {T}")
+    _check(lib().ple_embed_static(_ptr(tokens), T, _ptr(offsets), S, _ptr(hist), _ptr(table), _ptr(scales),
+                                  rows0, rows1, row_dim, vocab, _ptr(e_out), _ptr(status_out), _stream(stream)),
+           "ple_embed_static")

@@ -146,6 +146,37 @@ ple_status ple_decode_step(ple_handle* handle, const int32_t* tokens, int32_t B,
                            int32_t* hist, float* conv_state, const int32_t* n_commit,
                            cudaStream_t stream);
 
+/* ---- lookup without allocation ------------------------------------------
+ * The pages have no counterpart of this entry point; it exists for callers of
+ * this library that cannot allocate device memory where they run the layer:
+ * serving engines whose caching allocator reserves the whole device budget at
+ * start-up (a later cudaMalloc fails or fragments that pool), and runtimes
+ * that forbid device allocation after initialisation. Such callers cannot
+ * create a handle either, since ple_create allocates.
+ *
+ * ple_embed_static computes the n-gram row IDs of a packed batch (as
+ * ple_ngram_ids) and gathers and dequantises the rows into e_out fp16
+ * [T][row_dim] (as ple_gather_rows). It allocates nothing: the row IDs live in
+ * a fixed array inside the library image, PLE_STATIC_MAX_TOKENS x 2 int32
+ * (128 KiB), which every GPU that loads the library holds until the process
+ * exits. The caller passes all inputs and the output; table and scales are
+ * laid out as in ple_weights, with rows0 / rows1 rows in the two sub-tables.
+ *   - T > PLE_STATIC_MAX_TOKENS returns PLE_ERR_SHAPE; nothing is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents. Calls that overlap on the GPU (other streams, other threads)
+ *     race on it: order them on one stream.
+ *   - status_out (device int32, may be NULL) receives the call's device status:
+ *     PLE_ERR_RANGE for a token outside [0, vocab) or inconsistent offsets,
+ *     else PLE_OK. The status word is cleared at the start of every call. */
+#define PLE_STATIC_MAX_TOKENS 16384
+ple_status ple_embed_static(const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
+                            const int32_t* hist, const uint8_t* table, const float* scales,
+                            int64_t rows0, int64_t rows1, int32_t row_dim, int32_t vocab, void* e_out,
+                            int32_t* status_out, cudaStream_t stream);
+
 /* Synchronises the device, returns the sticky device status and clears it. */
 ple_status ple_get_error(ple_handle* handle);
 
