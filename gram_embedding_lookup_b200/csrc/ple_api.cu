@@ -30,6 +30,7 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 struct Plan {
   bool fused;
   int n_tok, tok_stride, tok_origin, halo, n_tiles, k_splits;
+  int ctas;   // 2: SM-pair tiles of 256 channels; 1: single-SM tiles of 128
 };
 
 }  // namespace
@@ -66,7 +67,7 @@ Plan plan_projection(const ple_handle* h, int T, int path, int64_t partial_cap) 
   const int m_tiles = h->cfg.hidden / kTileM;
   const int num_kb = h->cfg.row_dim / kTileK;
   const int fused_tiles_n = ceil_div(T, kFusedRows - kHalo);
-  bool fused = (path == 1) || (path == 0 && static_cast<int64_t>(m_tiles) * fused_tiles_n >= h->num_sms);
+  bool fused = (path == 1 || path == 3) || (path == 0 && static_cast<int64_t>(m_tiles) * fused_tiles_n >= h->num_sms);
   if (!fused) {
     const int n_tok = std::min(256, ceil_div(T, 16) * 16);
     const int n_tiles = ceil_div(T, n_tok);
@@ -74,10 +75,11 @@ Plan plan_projection(const ple_handle* h, int T, int path, int64_t partial_cap) 
     int ks = std::max(1, std::min(h->num_sms / std::max(tiles, 1), std::min(num_kb, 16)));
     while (ks > 1 && static_cast<int64_t>(ks) * T * h->cfg.hidden > partial_cap) --ks;
     if (static_cast<int64_t>(T) * h->cfg.hidden <= partial_cap)
-      return Plan{false, n_tok, n_tok, 0, 0, n_tiles, ks};
+      return Plan{false, n_tok, n_tok, 0, 0, n_tiles, ks, 1};
     fused = true;   // no room for partials: fall back to the fused path
   }
-  return Plan{true, kFusedRows, kFusedRows - kHalo, -kHalo, kHalo, fused_tiles_n, 1};
+  const int ctas = (path != 3 && h->cfg.hidden % (2 * kTileM) == 0 && h->num_sms >= 2) ? 2 : 1;
+  return Plan{true, kFusedRows, kFusedRows - kHalo, -kHalo, kHalo, fused_tiles_n, 1, ctas};
 }
 
 cudaEvent_t take_event(ple_handle* h) {
@@ -179,7 +181,7 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
 
   CUtensorMap tmap_e{}, tmap_h{}, tmap_o{}, tmap_o_head{};
   if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->e, c.row_dim, T, static_cast<uint64_t>(c.row_dim) * 2,
-                 kTileK, pl.n_tok, CU_TENSOR_MAP_SWIZZLE_128B))
+                 kTileK, pl.n_tok / pl.ctas, CU_TENSOR_MAP_SWIZZLE_128B))
     return PLE_ERR_CUDA;
   if (!encode_2d(h, &tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, c.hidden, T,
                  static_cast<uint64_t>(c.hidden) * 2, kTileM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -201,7 +203,7 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   gp.tok_stride = pl.tok_stride;
   gp.tok_origin = pl.tok_origin;
   gp.halo = pl.halo;
-  gp.m_tiles = c.hidden / kTileM;
+  gp.m_tiles = c.hidden / (kTileM * pl.ctas);
   gp.n_tiles = pl.n_tiles;
   gp.k_splits = pl.k_splits;
   gp.num_kb = c.row_dim / kTileK;
@@ -217,8 +219,8 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   gp.partial = h->partial;
   gp.status = h->status;
   const int total = gp.m_tiles * gp.n_tiles * gp.k_splits;
-  const int grid = std::min(total, h->num_sms);
-  st = run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_gemm(h->tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, gp, grid, stream);
+  const int grid = pl.ctas == 2 ? 2 * std::min(total, h->num_sms / 2) : std::min(total, h->num_sms);
+  st = run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_gemm(h->tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, gp, grid, pl.ctas, stream);
   });
   if (st != PLE_OK || pl.fused) return st;
 
@@ -477,7 +479,7 @@ ple_status ple_get_stage_times(ple_handle* h, float* ms, int64_t* launches) {
 }
 
 ple_status ple_set_forward_path(ple_handle* h, int32_t path) {
-  if (h == nullptr || path < 0 || path > 2) return PLE_ERR_INVALID_ARG;
+  if (h == nullptr || path < 0 || path > 3) return PLE_ERR_INVALID_ARG;
   h->forward_path = path;
   return PLE_OK;
 }

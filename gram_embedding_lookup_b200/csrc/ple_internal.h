@@ -64,12 +64,14 @@ struct GemmParams {
   float* partial;        // [k_splits][T][H]
   int32_t* status;
 };
-constexpr int kGemmSmemBytes = 4 * 16384 + 4 * 32768 + 3 * 8192 + 256 * 16 + 64 + 256 + 1024;
+constexpr int kGemmSmemBytes = 227 * 1024;   // the sm_100 per-block maximum
 // tmap_o / tmap_o_head: bf16 output tiles of 32 and of 29 tokens (the first
 // chunk of a fused tile without its halo rows).
+// ctas = 2: SM-pair tiles (clusters of two CTAs, 256 channels per tile, grid even,
+// m_tiles = hidden / 256, tmap_e boxes of n_tok / 2 rows); ctas = 1: single-SM tiles.
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_e, const CUtensorMap& tmap_h,
                         const CUtensorMap& tmap_o, const CUtensorMap& tmap_o_head, const GemmParams& p, int grid,
-                        cudaStream_t stream);
+                        int ctas, cudaStream_t stream);
 
 // Combine split-K partials + gate + conv + residual (+ state) for a packed batch.
 struct CombineArgs {

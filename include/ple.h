@@ -200,7 +200,9 @@ ple_status ple_get_stage_times(ple_handle* handle, float* ms, int64_t* launches)
 
 /* Path selection for ple_forward: 0 = automatic, 1 = fused epilogue
  * (gate, conv and residual inside the projection kernel, conv halo
- * recomputed per tile), 2 = split-K projection followed by a combine kernel. */
+ * recomputed per tile; SM-pair tiles of 256 channels when hidden % 256 == 0),
+ * 2 = split-K projection followed by a combine kernel, 3 = fused epilogue with
+ * single-SM tiles of 128 channels. */
 ple_status ple_set_forward_path(ple_handle* handle, int32_t path);
 
 /* Total number of kernels the handle has launched since creation. */

@@ -67,3 +67,18 @@ def full_layer():
     L.host_table = w.table()
     yield L
     L.close()
+
+
+MID = pi.Workload("mid", 5000, 8192, 128, 256, table_seed=7, seed=7)
+
+
+@pytest.fixture(scope="session")
+def mid_layer():
+    """hidden 256: the fused path runs on SM-pair tiles (path 1) or single-SM tiles (path 3)."""
+    import torch  # noqa: F401
+    from ple_inputs.device import DeviceLayer
+    L = DeviceLayer(MID, max_tokens=4096, max_seqs=64)
+    codes, scales = MID.table().full()
+    L.host_table = O.ArrayTable(codes, scales)
+    yield L
+    L.close()

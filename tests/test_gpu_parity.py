@@ -13,7 +13,7 @@ import pytest
 import oracle as O
 import ple_inputs as pi
 from tests.gpu_common import (MAX_ABS, REL_L2, assert_bf16_close, assert_close, full_layer,  # noqa: F401
-                              tiny_layer)
+                              mid_layer, tiny_layer)
 
 torch = pytest.importorskip("torch")
 ple = pytest.importorskip("gram_embedding_lookup_b200")
@@ -554,3 +554,57 @@ def test_stage_timing_and_launch_count(tiny_layer):
     assert ple.ple_launch_count(h) - n0 == 7
     assert st["prepare"][1] == 2 and st["gather"][1] == 2 and st["gemm"][1] == 2 and st["combine"][1] == 1
     assert all(v[0] > 0 for k, v in st.items())
+
+
+# ----------------------------------------------------------------------------- SM-pair tiles (hidden 256)
+def _mid_batch(lengths, seed):
+    from tests.gpu_common import MID
+    rng = np.random.default_rng(seed)
+    T = sum(lengths)
+    toks = rng.integers(0, MID.vocab, T).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    hid = pi.hidden_bf16(rng, T, MID.hidden)
+    return toks, offs, hid
+
+
+@pytest.mark.parametrize("path", [1, 3, 2])
+@pytest.mark.parametrize("lengths", [[1000], [1, 2, 3, 600, 0, 400], [253], [254, 253, 1], [4096]])
+def test_forward_mid_paths(mid_layer, path, lengths):
+    toks, offs, hid = _mid_batch(lengths, sum(lengths) + len(lengths))
+    ref = oracle_forward(mid_layer, toks, offs, hid)
+    out, _ = gpu_forward(mid_layer, toks, offs, hid, 1, path=path)
+    assert_close(out, ref["out"], f"mid {lengths} path {path}")
+    out16, _ = gpu_forward(mid_layer, toks, offs, hid, 0, path=path)
+    assert np.array_equal(out16, O.to_bf16_bits(out))
+    assert_bf16_close(out16, ref["out"])
+
+
+@pytest.mark.parametrize("path", [1, 3])
+def test_forward_mid_state(mid_layer, path):
+    toks, _, hid = _mid_batch([900], 5)
+    rng = np.random.default_rng(6)
+    offs = np.array([0, 300, 301, 301, 900], np.int32)
+    hist0 = rng.integers(-1, 5000, (4, 2)).astype(np.int32)
+    conv0 = rng.standard_normal((4, 3, 256)).astype(np.float32)
+    ref = oracle_forward(mid_layer, toks, offs, hid, hist=hist0, conv=conv0)
+    out, st = gpu_forward(mid_layer, toks, offs, hid, 1, state=(hist0, conv0), path=path)
+    assert_close(out, ref["out"], "mid state")
+    check_state(st, ref)
+
+
+def test_forward_mid_pair_equals_single(mid_layer):
+    toks, offs, hid = _mid_batch([700, 300], 9)
+    a, _ = gpu_forward(mid_layer, toks, offs, hid, 1, path=1)
+    b, _ = gpu_forward(mid_layer, toks, offs, hid, 1, path=3)
+    assert np.abs(a - b).max() < 1e-4
+
+
+def test_forward_mid_in_place(mid_layer):
+    toks, offs, hid = _mid_batch([2000, 96], 10)
+    ref16, _ = gpu_forward(mid_layer, toks, offs, hid, 0, path=1)
+    h = dev_bf16(hid)
+    ple.ple_set_forward_path(mid_layer.handle, 1)
+    ple.ple_forward(mid_layer.handle, dev_i32(toks), len(toks), dev_i32(offs), 2, h, h, 0)
+    torch.cuda.synchronize()
+    ple.ple_set_forward_path(mid_layer.handle, 0)
+    assert np.array_equal(to_bits(h), ref16)
