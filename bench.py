@@ -39,8 +39,8 @@ GATHER_SOURCES = ["gram_embedding_lookup_b200/csrc/ple_kernels.cu"]
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ple", "reference"], default="ple")
     ap.add_argument("--table-rows", type=int, default=0,
                     help="rows per sub-table (default: the full 10,000,048); smaller only for profiling captures")
@@ -82,25 +82,52 @@ def load_traffic(kernel: str, workload: str, src_hash: str):
     return None
 
 
-class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+_SAMPLER = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+bus, idx, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+dev = None
+if bus != "-":
+    try:
+        dev = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+    except Exception:
+        dev = None
+if dev is None:
+    dev = pynvml.nvmlDeviceGetHandleByIndex(idx)
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(dev, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    try:
+        print(pynvml.nvmlDeviceGetClockInfo(dev, pynvml.NVML_CLOCK_SM),
+              pynvml.nvmlDeviceGetCurrentClocksEventReasons(dev), flush=True)
+    except Exception:
+        pass
+    time.sleep(period)
+"""
 
-    def __init__(self, index: int):
+
+class ClockSampler:
+    """SM clock and throttle reasons, sampled through NVML every few milliseconds by a
+    separate process while running (reads only; no setting is changed)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, index: int, period_s: float = 0.005, pci_bus_id: str | None = None):
         self.index = index
+        self.period = period_s
+        self.pci_bus_id = pci_bus_id
         self.proc = None
-        self.path = os.environ.get("PLE_CLOCKS_CSV") or os.path.join(
-            tempfile.gettempdir(), f"ple_clocks_{os.getpid()}_{index}.csv")
 
     def start(self):
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        """Starts the sampler and returns once it is producing samples."""
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER, self.pci_bus_id or "-", str(self.index),
+                                          str(self.period)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            first = self.proc.stdout.readline().split()
+            self.max_mhz = float(first[1]) if len(first) == 2 and first[0] == "max" else float("nan")
+            self.proc.stdout.readline()             # one sample taken: the sampler is live
+        except Exception:  # pragma: no cover - no NVML on this host
             self.proc = None
 
     def stop(self):
@@ -108,29 +135,26 @@ class ClockSampler:
             return None
         self.proc.terminate()
         try:
-            self.proc.wait(timeout=5)
+            out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        self.f.close()
-        sms, maxs, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                c = [x.strip() for x in line.split(",")]
-                if len(c) < 9:
-                    continue
-                try:
-                    sms.append(float(c[1]))
-                    maxs.append(float(c[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, c[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        if not sms:
+            out, _ = self.proc.communicate()
+        mhz, reasons = [], set()
+        for line in out.splitlines():
+            parts = line.split()
+            if len(parts) != 2:
+                continue
+            try:
+                m, r = float(parts[0]), int(parts[1])
+            except ValueError:
+                continue
+            mhz.append(m)
+            reasons |= {n for n, bit in self.REASONS.items() if r & bit}
+        if not mhz:
             return None
-        return {"sm_mhz": float(np.median(sms)), "sm_max_mhz": float(max(maxs)), "reasons": sorted(reasons),
-                "samples": len(sms)}
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "sm_min_mhz": float(min(mhz)),
+                "reasons": sorted(reasons), "samples": len(mhz),
+                "source": "NVML in a separate process, sampled inside the timed region"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs
@@ -238,13 +262,15 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
+    ctx = dict(torch=torch, ple=ple, pi=pi, bf16_tensor=bf16_tensor, barrier=barrier,
+               max_over_ranks=max_over_ranks, world=world, args=args)
     stream = torch.cuda.current_stream()
     w0 = pi.workload("prefill")
     w = w0 if args.table_rows <= 0 else pi.Workload("prefill", w0.vocab, args.table_rows, w0.row_dim, w0.hidden,
                                                       w0.table_seed, w0.seed, w0.extra)
     layer = DeviceLayer(w, max_tokens=16384, max_seqs=64)
     h = layer.handle
-    H = w.hidden
+    H, D = w.hidden, w.row_dim
 
     sets = []
     for v in range(args.sets):
@@ -265,11 +291,15 @@ def main():
     if ple.ple_get_error(h) != 0:
         raise SystemExit("device status error during warm-up")
 
+    # ------------------------------------------------------------------ timed region
     ple.ple_set_profiling(h, True)
     ple.ple_get_stage_times(h)
-    clocks = ClockSampler(local) if not args.no_extras else None
-    if clocks:
-        clocks.start()
+    props = torch.cuda.get_device_properties(local)
+    bus = None
+    if hasattr(props, "pci_bus_id"):
+        bus = f"{getattr(props, 'pci_domain_id', 0):08x}:{props.pci_bus_id:02x}:{getattr(props, 'pci_device_id', 0):02x}.0"
+    clocks = ClockSampler(local, pci_bus_id=bus)
+    clocks.start()
     launches0 = ple.ple_launch_count(h)
     barrier()
     torch.cuda.synchronize()
@@ -279,9 +309,9 @@ def main():
         step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
+    clk = clocks.stop()     # stops at the end of the timed region (it started just before it)
     barrier()
     launches = ple.ple_launch_count(h) - launches0
-    clk = clocks.stop() if clocks else None
     stage = ple.ple_get_stage_times(h)
     ple.ple_set_profiling(h, False)
     status = ple.ple_get_error(h)
@@ -291,42 +321,49 @@ def main():
     value = T * world * args.steps / (ms / 1e3)
 
     peaks, peak_kind = load_peaks()
-    D = w.row_dim
     gemm_ms, gemm_n = stage["gemm"]
     gemm_s = gemm_ms / 1e3 / max(gemm_n, 1)
     flops = 2.0 * D * H * T
     achieved_tf = flops / gemm_s / 1e12
-    peak_tf = peaks["bf16_tflops"]   # fp16 and bf16 share the nominal dense rate (ratio 1)
-    gemm_traffic = load_traffic("gemm", "prefill", source_hash(GEMM_SOURCES))
-    roofline = {"kernel": "ple gemm (tcgen05 projection + fused gate/conv/residual)", "bound": "tensor",
+    # the GEMM runs back to back in a loop long enough to reach the power cap: compare it with
+    # the sustained bf16 figure (fp16 and bf16 share the nominal dense rate, ratio 1)
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    roofline = {"kernel": "gemm_kernel (tcgen05 projection + fused gate/conv/residual)", "bound": "tensor",
                 "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
-                "peak_source": f"{peak_kind} bf16_tflops (burst); fp16 nominal ratio 1.0",
-                "traffic": gemm_traffic, "algorithmic_flops_per_launch": flops, "launch_ms": gemm_s * 1e3}
-
-    g_ms, g_n = stage["gather"]
-    g_s = g_ms / 1e3 / max(g_n, 1)
-    gather_bytes = T * (2 * D + 8 + 8 + 2 * D)   # rows + scales + ids in, fp16 e out
-    gather = {"bound": "hbm", "achieved": gather_bytes / g_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-              "frac": gather_bytes / g_s / 1e9 / peaks["hbm_gbs"],
-              "gathered_row_gbs": T * 2 * D / g_s / 1e9, "launch_ms": g_s * 1e3,
-              "traffic": load_traffic("gather", "prefill", source_hash(GATHER_SOURCES)),
-              "algorithmic_bytes_per_launch": gather_bytes}
-    stages_ms = {k: (v[0] / max(v[1], 1)) for k, v in stage.items()}
+                "peak_source": f"{peak_kind} bf16_tflops_sustained (loop of {args.steps} steps under the power "
+                               f"cap); fp16 nominal ratio 1.0",
+                "frac_of_burst_peak": achieved_tf / peaks["bf16_tflops"],
+                "traffic": load_traffic("gemm", "prefill", source_hash(GEMM_SOURCES)),
+                "algorithmic_flops_per_launch": flops, "launch_ms": gemm_s * 1e3}
+    e_ms, e_n = stage["prepare"]
+    e_s = e_ms / 1e3 / max(e_n, 1)
+    embed_bytes = T * (2 * H + 2 * D + 8 + 2 * D + 8 + 16 + 4)   # h, rows, scales in; e, ids, meta out; tokens
+    embed = {"kernel": "embed_kernel (ids + gate + row gather/dequant)", "bound": "hbm",
+             "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"], "launch_ms": e_s * 1e3,
+             "algorithmic_bytes_per_launch": embed_bytes,
+             "traffic": load_traffic("embed", "prefill", source_hash(GATHER_SOURCES))}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": prefill_config(args, w, world),
-        "roofline": roofline, "gather_roofline": gather, "stage_ms_per_launch": stages_ms,
+        "roofline": roofline, "embed_roofline": embed,
+        "stage_ms_per_launch": {k: (v[0] / max(v[1], 1)) for k, v in stage.items() if v[1]},
         "gpu_launches": int(launches) * world, "device_status": int(status),
         "gathered_row_gbs_end_to_end": T * 2 * D * args.steps / (ms / 1e3) / 1e9,
+        "timing_note": "device time of the K-step loop (CUDA events on the launching stream); library stage "
+                       "events recorded inside the same loop",
     }
     if clk:
         line["clocks"] = clk
+    line["gather_roofline"] = gather_bench(ctx, layer, sets, stream, peaks)
 
     if not args.no_extras:
         line["e2e"] = e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier)
-        line["decode"] = decode_bench(args, ple, pi, layer, stream, max_over_ranks, barrier, world)
+        line["decode"] = decode_bench(ctx, layer, stream)
+        line["mtp"] = mtp_bench(ctx, layer, stream)
+        line["long_context"] = long_bench(ctx, layer, stream)
 
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         tokens, offsets, hidden = sets[0]["host"]
@@ -350,6 +387,52 @@ def main():
         dist.destroy_process_group()
 
 
+def timed(ctx, stream, fn, n):
+    """Device time (ms) of n calls of fn on `stream`, max over ranks."""
+    torch = ctx["torch"]
+    ctx["barrier"]()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ctx["barrier"]()
+    return ctx["max_over_ranks"](e0.elapsed_time(e1))
+
+
+def gather_bench(ctx, layer, sets, stream, peaks):
+    """The gather stage alone (ple_gather_rows) over the prefill batches' row IDs:
+    algorithmic bytes per launch = T x (2 rows x D codes + 2 scales + 2 ids + D fp16 written)."""
+    torch, ple = ctx["torch"], ctx["ple"]
+    h = layer.handle
+    D = layer.w.row_dim
+    ids, es = [], []
+    for s in sets:
+        t = torch.empty(s["T"], 2, dtype=torch.int32, device="cuda")
+        ple.ple_ngram_ids(h, s["tokens"], s["T"], s["offsets"], s["S"], None, t, stream)
+        ids.append(t)
+        es.append(torch.empty(s["T"], D, dtype=torch.float16, device="cuda"))
+    T = sets[0]["T"]
+
+    def fn(i):
+        k = i % len(sets)
+        ple.ple_gather_rows(h, ids[k], T, es[k], stream)
+
+    for i in range(5):
+        fn(i)
+    n = 200
+    ms = timed(ctx, stream, fn, n)
+    per = ms / 1e3 / n
+    nbytes = T * (2 * D + 8 + 8 + 2 * D)
+    return {"kernel": "gather_kernel (ple_gather_rows, standalone)", "bound": "hbm",
+            "achieved": nbytes / per / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": nbytes / per / 1e9 / peaks["hbm_gbs"], "gathered_row_gbs": T * 2 * D / per / 1e9,
+            "launch_ms": per * 1e3, "launches": n, "algorithmic_bytes_per_launch": nbytes,
+            "traffic": load_traffic("gather", "prefill", source_hash(GATHER_SOURCES))}
+
+
 def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
     """Same metric through the C ABI with host buffers: H2D of the step's inputs from
     pinned memory, the layer, D2H of the output, all inside the timed region."""
@@ -370,13 +453,13 @@ def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
                         None, stream)
         hs["out"].copy_(s["out"], non_blocking=True)
 
-    for i in range(args.warmup):
+    for i in range(max(args.warmup, 3)):
         step(i)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    steps = max(3, min(args.steps, 20))
+    steps = 20
     for i in range(steps):
         step(i)
     e1.record(stream)
@@ -390,10 +473,10 @@ def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps}
 
 
-def decode_bench(args, ple, pi, layer, stream, max_over_ranks, barrier, world):
-    """Full-scale decode: 8 sequences x 1 new token per step, carried history and conv state."""
-    import torch
-    from ple_inputs.device import bf16_tensor
+def decode_bench(ctx, layer, stream):
+    """Full-scale decode: 8 sequences x 1 new token per step with carried history and
+    conv state; timed eagerly and as a replayed CUDA graph of one ple_decode_step."""
+    torch, ple, pi, bf16_tensor = ctx["torch"], ctx["ple"], ctx["pi"], ctx["bf16_tensor"]
     wd = pi.workload("decode")
     tokens, hidden, hist, conv = pi.decode_batch(wd)
     B, q = tokens.shape
@@ -404,30 +487,106 @@ def decode_bench(args, ple, pi, layer, stream, max_over_ranks, barrier, world):
     out = torch.empty(B * q, wd.hidden, dtype=torch.bfloat16, device="cuda")
     h = layer.handle
 
-    def step():
-        ple.ple_decode_step(h, tk, B, q, hd, out, ple.PLE_OUT_BF16, hs, cs, None, stream)
+    def eager(i, st=stream):
+        ple.ple_decode_step(h, tk, B, q, hd, out, ple.PLE_OUT_BF16, hs, cs, None, st)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    barrier()
-    n = 200
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(5):
+        eager(i)
+    n = 500
+    ms_eager = timed(ctx, stream, eager, n)
     ple.ple_set_profiling(h, True)
     ple.ple_get_stage_times(h)
-    e0.record(stream)
-    for _ in range(n):
-        step()
-    e1.record(stream)
+    for i in range(50):
+        eager(i)
     torch.cuda.synchronize()
     stage = ple.ple_get_stage_times(h)
     ple.ple_set_profiling(h, False)
-    barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for i in range(3):
+            eager(i, side)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        eager(0, torch.cuda.current_stream())
+    ms_graph = timed(ctx, stream, lambda i: graph.replay(), n)
+    world = ctx["world"]
     return {"workload": "full-scale decode: 8 sequences x 1 token, 2-token history + 3x2560 conv state",
-            "value": B * q * world * n / (ms / 1e3), "unit": "tokens/s", "us_per_step": 1e3 * ms / n,
-            "stage_us_per_launch": {k: 1e3 * v[0] / max(v[1], 1) for k, v in stage.items()},
-            "note": "consecutive steps reuse one batch; W_proj (13 MB) stays L2-resident, as in a real decode loop"}
+            "value": B * q * world * n / (ms_eager / 1e3), "unit": "tokens/s", "us_per_step": 1e3 * ms_eager / n,
+            "graph_value": B * q * world * n / (ms_graph / 1e3), "graph_us_per_step": 1e3 * ms_graph / n,
+            "stage_us_per_launch": {k: 1e3 * v[0] / max(v[1], 1) for k, v in stage.items() if v[1]},
+            "note": "one batch reused; the graph replays one captured ple_decode_step on static buffers"}
+
+
+def mtp_bench(ctx, layer, stream):
+    """MTP-style decode: 64 sequences x 3 tokens per step (1 accepted + 2 drafts) for 100
+    steps after a 512-token prompt per sequence (19 sequences share prompt and continuation);
+    the state advances by each step's n_commit."""
+    torch, ple, pi, bf16_tensor = ctx["torch"], ctx["ple"], ctx["pi"], ctx["bf16_tensor"]
+    w = pi.workload("mtp")
+    sess = pi.mtp_session(w)
+    B, P = sess["prompts"].shape
+    q = w.extra["q"]
+    h = layer.handle
+    hist = torch.full((B, 2), -1, dtype=torch.int32, device="cuda")
+    conv = torch.zeros(B, 3, w.hidden, dtype=torch.float32, device="cuda")
+    half = B // 2
+    for b0 in (0, half):                       # prompts in two packed batches of 16,384 tokens
+        toks = torch.from_numpy(np.ascontiguousarray(sess["prompts"][b0:b0 + half].reshape(-1))).cuda()
+        offs = torch.from_numpy((np.arange(half + 1) * P).astype(np.int32)).cuda()
+        hid = bf16_tensor(sess["prompt_hidden"][b0 * P:(b0 + half) * P])
+        out = torch.empty_like(hid)
+        ple.ple_forward(h, toks, half * P, offs, half, hid, out, ple.PLE_OUT_BF16,
+                        (hist[b0:b0 + half], conv[b0:b0 + half]), stream)
+    steps = [(torch.from_numpy(t).cuda(), bf16_tensor(hd), torch.from_numpy(nc).cuda())
+             for t, hd, nc in sess["steps"]]
+    out = torch.empty(B * q, w.hidden, dtype=torch.bfloat16, device="cuda")
+
+    def step(i):
+        tk, hd, nc = steps[i % len(steps)]
+        ple.ple_decode_step(h, tk, B, q, hd, out, ple.PLE_OUT_BF16, hist, conv, nc, stream)
+
+    for i in range(3):
+        step(i)
+    n = len(steps)
+    ms = timed(ctx, stream, step, n)
+    committed = int(sum(int(nc.sum()) for _, _, nc in sess["steps"]))
+    world = ctx["world"]
+    return {"workload": "MTP decode: 64 sequences x 3 tokens/step, 100 steps, 30% shared prefix",
+            "value": B * q * world * n / (ms / 1e3), "unit": "tokens/s (processed)",
+            "committed_tokens_per_s": committed * world / (ms / 1e3), "us_per_step": 1e3 * ms / n}
+
+
+def long_bench(ctx, layer, stream):
+    """Long-context chunked prefill: one 262,144-token sequence of uniform tokens in 16
+    chunks of 16,384, conv state and the last two tokens carried across chunks."""
+    torch, ple, pi, bf16_tensor = ctx["torch"], ctx["ple"], ctx["pi"], ctx["bf16_tensor"]
+    w = pi.workload("long")
+    chunk = w.extra["chunk"]
+    n_chunks = w.extra["total"] // chunk
+    rng = np.random.default_rng([w.seed, 13])
+    toks = [torch.from_numpy(pi.tokens_uniform(rng, chunk, w.vocab)).cuda() for _ in range(n_chunks)]
+    hids = [bf16_tensor(pi.hidden_bf16(rng, chunk, w.hidden)) for _ in range(4)]   # hidden values reused
+    offs = torch.tensor([0, chunk], dtype=torch.int32, device="cuda")
+    out = torch.empty(chunk, w.hidden, dtype=torch.bfloat16, device="cuda")
+    hist = torch.full((1, 2), -1, dtype=torch.int32, device="cuda")
+    conv = torch.zeros(1, 3, w.hidden, dtype=torch.float32, device="cuda")
+    h = layer.handle
+
+    def fn(i):
+        ple.ple_forward(h, toks[i % n_chunks], chunk, offs, 1, hids[i % 4], out, ple.PLE_OUT_BF16, (hist, conv),
+                        stream)
+
+    fn(0)
+    hist.fill_(-1)
+    conv.zero_()
+    ms = timed(ctx, stream, fn, n_chunks)
+    world = ctx["world"]
+    return {"workload": "long context: 262,144 uniform tokens, 16 chunks of 16,384 with carried state",
+            "value": chunk * n_chunks * world / (ms / 1e3), "unit": "tokens/s", "ms_total": ms}
 
 
 if __name__ == "__main__":

@@ -170,12 +170,9 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
     pa.hist_new = h->hist_new;
   }
   pa.status = h->status;
-  ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_prepare(pa, stream); });
-  if (st != PLE_OK) return st;
-
-  st = run_stage(h, PLE_STAGE_GATHER, stream, [&] {
-    return ple::launch_gather(h->ids, T, h->w.table, h->w.scales, c.rows[0], c.rows[1], c.row_dim, h->e, false,
-                              stream);
+  // row IDs, gate and the gathered, dequantised rows in one kernel
+  ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
+    return ple::launch_embed(pa, h->w.table, h->w.scales, c.row_dim, h->e, stream);
   });
   if (st != PLE_OK) return st;
 

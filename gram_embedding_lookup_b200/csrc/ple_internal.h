@@ -35,6 +35,11 @@ struct PrepareArgs {
 };
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
 
+// Prepare and gather fused (one warp per token, one pass over HBM): ids,
+// metadata with the gate, and e[t] for the batch.
+cudaError_t launch_embed(const PrepareArgs& a, const uint8_t* table, const float* scales, int32_t D, __half* e,
+                         cudaStream_t stream);
+
 // Gather stage: e[t] = deq(row of order 0) + deq(row of order 1), fp16.
 cudaError_t launch_gather(const int32_t* ids, int32_t T, const uint8_t* table, const float* scales,
                           int64_t rows0, int64_t rows1, int32_t D, __half* e, bool reduce_ids,

@@ -31,57 +31,10 @@ __device__ __forceinline__ uint64_t context_of(int32_t tok) {
 
 __device__ __forceinline__ uint64_t fold64(uint64_t k) { return k ^ (k >> 32); }
 
-// ------------------------------------------------------------------ prepare
-constexpr int kPrepWarps = 8;   // one warp per token, 8 tokens per block
-
-__global__ void __launch_bounds__(256) prepare_kernel(const PrepareArgs a, int token_blocks) {
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (static_cast<int>(blockIdx.x) >= token_blocks) {
-    // ---- state and offsets blocks
-    const int sb = blockIdx.x - token_blocks;
-    const int nsb = gridDim.x - token_blocks;
-    if (sb == 0 && a.uniform_q == 0) {
-      // offsets must start at 0, end at T and be non-decreasing
-      if (threadIdx.x == 0 && (a.offsets[0] != 0 || a.offsets[a.S] != a.T)) set_status(a.status, PLE_ERR_RANGE);
-      for (int s = threadIdx.x; s < a.S; s += blockDim.x)
-        if (a.offsets[s] > a.offsets[s + 1]) set_status(a.status, PLE_ERR_RANGE);
-    }
-    if (a.conv_in != nullptr) {
-      const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
-      const float4* src = reinterpret_cast<const float4*>(a.conv_in);
-      float4* dst = reinterpret_cast<float4*>(a.conv_copy);
-      for (int64_t i = static_cast<int64_t>(sb) * blockDim.x + threadIdx.x; i < n4;
-           i += static_cast<int64_t>(nsb) * blockDim.x)
-        dst[i] = src[i];
-    }
-    if (a.hist_new != nullptr && sb == 0) {
-      for (int s = threadIdx.x; s < a.S; s += blockDim.x) {
-        int32_t begin, end;
-        if (a.uniform_q > 0) { begin = s * a.uniform_q; end = begin + a.uniform_q; }
-        else { begin = a.offsets[s]; end = a.offsets[s + 1]; }
-        end = min(max(end, 0), a.T);
-        begin = min(max(begin, 0), end);
-        const int32_t len = end - begin;
-        const int32_t h0 = a.hist ? a.hist[2 * s] : -1;
-        const int32_t h1 = a.hist ? a.hist[2 * s + 1] : -1;
-        int32_t n0, n1;
-        if (len >= 2) { n0 = a.tokens[end - 2]; n1 = a.tokens[end - 1]; }
-        else if (len == 1) { n0 = h1; n1 = a.tokens[end - 1]; }
-        else { n0 = h0; n1 = h1; }
-        a.hist_new[2 * s] = n0;
-        a.hist_new[2 * s + 1] = n1;
-      }
-    }
-    return;
-  }
-
-  const int t = blockIdx.x * kPrepWarps + warp;
-  if (t >= a.T) return;
-
-  // ---- sequence and position (every lane computes the same values)
-  int32_t s, pos, last;
+// Sequence, position, last-token flag and the two row IDs of token t (every
+// lane of the calling warp computes the same values; lane 0 reports errors).
+__device__ __forceinline__ void sequence_and_rows(const PrepareArgs& a, int t, int lane, int32_t& s, int32_t& pos,
+                                                  int32_t& last, int32_t& r0, int32_t& r1) {
   if (a.uniform_q > 0) {
     s = t / a.uniform_q;
     pos = t - s * a.uniform_q;
@@ -102,8 +55,6 @@ __global__ void __launch_bounds__(256) prepare_kernel(const PrepareArgs a, int t
     }
     last = (t == end - 1);
   }
-
-  // ---- n-gram contexts, keys and rows
   const int32_t tok = a.tokens[t];
   if (lane == 0 && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
   const uint64_t x0 = context_of(tok);
@@ -116,11 +67,63 @@ __global__ void __launch_bounds__(256) prepare_kernel(const PrepareArgs a, int t
   const uint64_t x2 = pos >= 2 ? context_of(a.tokens[t - 2]) : (pos == 1 ? carried(1) : carried(2));
   const uint64_t k2 = (x0 * kP0) ^ (x1 * kP1);
   const uint64_t k3 = k2 ^ (x2 * kP2);
-  if (lane == 0) {
-    const int32_t r0 = static_cast<int32_t>(fold64(k2) % static_cast<uint64_t>(a.rows0));
-    const int32_t r1 = static_cast<int32_t>(fold64(k3) % static_cast<uint64_t>(a.rows1));
-    reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
+  r0 = static_cast<int32_t>(fold64(k2) % static_cast<uint64_t>(a.rows0));
+  r1 = static_cast<int32_t>(fold64(k3) % static_cast<uint64_t>(a.rows1));
+}
+
+// The state and offsets blocks of the prepare / embed kernels.
+__device__ __forceinline__ void state_blocks(const PrepareArgs& a, int sb, int nsb) {
+  if (sb == 0 && a.uniform_q == 0) {
+    // offsets must start at 0, end at T and be non-decreasing
+    if (threadIdx.x == 0 && (a.offsets[0] != 0 || a.offsets[a.S] != a.T)) set_status(a.status, PLE_ERR_RANGE);
+    for (int s = threadIdx.x; s < a.S; s += blockDim.x)
+      if (a.offsets[s] > a.offsets[s + 1]) set_status(a.status, PLE_ERR_RANGE);
   }
+  if (a.conv_in != nullptr) {
+    const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
+    const float4* src = reinterpret_cast<const float4*>(a.conv_in);
+    float4* dst = reinterpret_cast<float4*>(a.conv_copy);
+    for (int64_t i = static_cast<int64_t>(sb) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(nsb) * blockDim.x)
+      dst[i] = src[i];
+  }
+  if (a.hist_new != nullptr && sb == 0) {
+    for (int s = threadIdx.x; s < a.S; s += blockDim.x) {
+      int32_t begin, end;
+      if (a.uniform_q > 0) { begin = s * a.uniform_q; end = begin + a.uniform_q; }
+      else { begin = a.offsets[s]; end = a.offsets[s + 1]; }
+      end = min(max(end, 0), a.T);
+      begin = min(max(begin, 0), end);
+      const int32_t len = end - begin;
+      const int32_t h0 = a.hist ? a.hist[2 * s] : -1;
+      const int32_t h1 = a.hist ? a.hist[2 * s + 1] : -1;
+      int32_t n0, n1;
+      if (len >= 2) { n0 = a.tokens[end - 2]; n1 = a.tokens[end - 1]; }
+      else if (len == 1) { n0 = h1; n1 = a.tokens[end - 1]; }
+      else { n0 = h0; n1 = h1; }
+      a.hist_new[2 * s] = n0;
+      a.hist_new[2 * s + 1] = n1;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ prepare
+constexpr int kPrepWarps = 8;   // one warp per token, 8 tokens per block
+
+__global__ void __launch_bounds__(256) prepare_kernel(const PrepareArgs a, int token_blocks) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (static_cast<int>(blockIdx.x) >= token_blocks) {
+    state_blocks(a, blockIdx.x - token_blocks, gridDim.x - token_blocks);
+    return;
+  }
+
+  const int t = blockIdx.x * kPrepWarps + warp;
+  if (t >= a.T) return;
+  int32_t s, pos, last, r0, r1;
+  sequence_and_rows(a, t, lane, s, pos, last, r0, r1);
+  if (lane == 0) reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
   if (a.meta == nullptr) return;
 
   // ---- gate: g = sigmoid(w_gate . h_t), fp32 accumulation, warp reduction
@@ -210,6 +213,110 @@ __global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ id
   uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D + c * 16);
   dst[0] = o0;
   dst[1] = o1;
+}
+
+// ------------------------------------------------------------------ embed (prepare + gather)
+// One warp per token does, in one pass over HBM: the sequence map and row IDs,
+// the gate dot product over h_t, and the row gather with E4M3 dequantisation
+// into fp16 e_t. The h loads are issued first so that they overlap the hash,
+// and both rows' loads are issued before any arithmetic on them. Rows up to
+// 2560 codes and hidden sizes up to 2560 stay in registers; larger sizes take
+// a tail loop.
+constexpr int kEmbedH4 = 10;    // uint4 of h per lane held in registers
+constexpr int kEmbedD16 = 5;    // 16-code chunks per lane and row held in registers
+
+__global__ void __launch_bounds__(256) embed_kernel(const PrepareArgs a, int token_blocks,
+                                                    const uint8_t* __restrict__ table,
+                                                    const float* __restrict__ scales, int32_t D,
+                                                    __half* __restrict__ e) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (static_cast<int>(blockIdx.x) >= token_blocks) {
+    state_blocks(a, blockIdx.x - token_blocks, gridDim.x - token_blocks);
+    return;
+  }
+  const int t = blockIdx.x * kPrepWarps + warp;
+  if (t >= a.T) return;
+
+  const int H8 = a.H / 8;
+  const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+  uint4 hv[kEmbedH4];
+#pragma unroll
+  for (int r = 0; r < kEmbedH4; ++r) {
+    const int j = lane + 32 * r;
+    hv[r] = j < H8 ? ld_stream_v4(hrow + j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  int32_t s, pos, last, r0, r1;
+  sequence_and_rows(a, t, lane, s, pos, last, r0, r1);
+  const int D16 = D / 16;
+  const uint8_t* ra = table + static_cast<int64_t>(r0) * D;
+  const uint8_t* rb = table + (a.rows0 + r1) * D;
+  uint4 ca[kEmbedD16], cb[kEmbedD16];
+#pragma unroll
+  for (int r = 0; r < kEmbedD16; ++r) {
+    const int j = lane + 32 * r;
+    if (j < D16) {
+      ca[r] = ld_stream_v4(ra + 16 * j);
+      cb[r] = ld_stream_v4(rb + 16 * j);
+    }
+  }
+  const float s0 = __ldg(scales + r0);
+  const float s1 = __ldg(scales + a.rows0 + r1);
+  if (lane == 0) reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
+
+  // gate: g = sigmoid(w_gate . h_t), fp32, the same summation order as prepare_kernel
+  const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+  float acc = 0.f;
+  auto dot8 = [&](const uint4& hq, const uint4& wq) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
+    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 hf = __bfloat1622float2(h2[q]);
+      const float2 wf = __bfloat1622float2(w2[q]);
+      acc = fmaf(hf.x, wf.x, acc);
+      acc = fmaf(hf.y, wf.y, acc);
+    }
+  };
+#pragma unroll
+  for (int r = 0; r < kEmbedH4; ++r) {
+    const int j = lane + 32 * r;
+    if (j < H8) dot8(hv[r], __ldg(wg + j));
+  }
+  for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) dot8(ld_stream_v4(hrow + j), __ldg(wg + j));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    TokMeta m;
+    m.g = 1.0f / (1.0f + expf(-acc));
+    m.seq = s;
+    m.pos = pos;
+    m.flags = last ? kFlagLast : 0;
+    a.meta[t] = m;
+  }
+
+  // e_t = deq(bigram row) + deq(trigram row), fp16
+  uint4* erow = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D);
+  auto emit = [&](int j, const uint4& x, const uint4& y) {
+    uint4 o0, o1;
+    o0.x = combine_pair(x.x, y.x, 0, s0, s1);
+    o0.y = combine_pair(x.x, y.x, 16, s0, s1);
+    o0.z = combine_pair(x.y, y.y, 0, s0, s1);
+    o0.w = combine_pair(x.y, y.y, 16, s0, s1);
+    o1.x = combine_pair(x.z, y.z, 0, s0, s1);
+    o1.y = combine_pair(x.z, y.z, 16, s0, s1);
+    o1.z = combine_pair(x.w, y.w, 0, s0, s1);
+    o1.w = combine_pair(x.w, y.w, 16, s0, s1);
+    erow[2 * j] = o0;
+    erow[2 * j + 1] = o1;
+  };
+#pragma unroll
+  for (int r = 0; r < kEmbedD16; ++r) {
+    const int j = lane + 32 * r;
+    if (j < D16) emit(j, ca[r], cb[r]);
+  }
+  for (int j = lane + 32 * kEmbedD16; j < D16; j += 32) emit(j, ld_stream_v4(ra + 16 * j), ld_stream_v4(rb + 16 * j));
 }
 
 // ------------------------------------------------------------------ W_proj conversion
@@ -324,6 +431,19 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
     state_blocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
   }
   prepare_kernel<<<token_blocks + state_blocks, 256, 0, stream>>>(a, token_blocks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_embed(const PrepareArgs& a, const uint8_t* table, const float* scales, int32_t D, __half* e,
+                         cudaStream_t stream) {
+  const int token_blocks = (a.T + kPrepWarps - 1) / kPrepWarps;
+  int state_blocks = 1;
+  if (a.conv_in != nullptr) {
+    const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
+    const int64_t want = (n4 + 255) / 256;
+    state_blocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
+  }
+  embed_kernel<<<token_blocks + state_blocks, 256, 0, stream>>>(a, token_blocks, table, scales, D, e);
   return cudaGetLastError();
 }
 

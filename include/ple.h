@@ -185,7 +185,9 @@ const char* ple_status_string(ple_status status);
 
 /* ---- measurement and test controls -------------------------------------- */
 
-/* Kernel stages of the library, in launch order within a call. */
+/* Kernel stages of the library, in launch order within a call. In
+ * ple_forward and ple_decode_step the PREPARE stage also gathers and
+ * dequantises the rows (one fused kernel); GATHER counts ple_gather_rows. */
 enum { PLE_STAGE_PREPARE = 0, PLE_STAGE_GATHER = 1, PLE_STAGE_GEMM = 2, PLE_STAGE_COMBINE = 3,
        PLE_NUM_STAGES = 4 };
 
