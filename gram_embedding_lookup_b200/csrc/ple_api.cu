@@ -48,9 +48,14 @@ struct ple_handle {
   int64_t partial_elems = 0;
   float* conv0 = nullptr;
   int32_t* hist_new = nullptr;
-  int32_t* status = nullptr;
+  int32_t* status = nullptr;     // [0]: sticky status; [1]: tiles completed by the decode kernel
+  bool decode_small = false;     // the single-kernel decode step fits this shape and device
+  ple::DecodePlan decode_plan{};
+  float* decode_partial = nullptr;
+  int32_t* tile_count = nullptr;
   EncodeTiledFn encode = nullptr;
   CUtensorMap tmap_w{};
+  CUtensorMap tmap_wd{};         // fp16 W_proj, 64 x 16 boxes for the decode kernel
   int32_t forward_path = 0;
   bool profiling = false;
   struct Rec { int stage; cudaEvent_t a, b; };
@@ -133,6 +138,8 @@ void free_all(ple_handle* h) {
   cudaFree(h->conv0);
   cudaFree(h->hist_new);
   cudaFree(h->status);
+  cudaFree(h->decode_partial);
+  cudaFree(h->tile_count);
   for (auto& r : h->pending) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
@@ -326,14 +333,21 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
             cudaMalloc(&h->partial, static_cast<size_t>(cap) * 4) == cudaSuccess &&
             cudaMalloc(&h->conv0, static_cast<size_t>(c.max_seqs) * 3 * c.hidden * 4) == cudaSuccess &&
             cudaMalloc(&h->hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess &&
-            cudaMalloc(&h->status, 4) == cudaSuccess;
+            cudaMalloc(&h->status, 8) == cudaSuccess;
+  h->decode_small = ok && ple::decode_small_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
+  if (h->decode_small) {
+    ok = cudaMalloc(&h->decode_partial,
+                    static_cast<size_t>(ple::decode_small_partial_elems(h->decode_plan, c.hidden)) * 4) == cudaSuccess &&
+         cudaMalloc(&h->tile_count, static_cast<size_t>(c.hidden / 16) * 4) == cudaSuccess &&
+         cudaMemsetAsync(h->tile_count, 0, static_cast<size_t>(c.hidden / 16) * 4, stream) == cudaSuccess;
+  }
   if (!ok) {
     cudaGetLastError();
     free_all(h);
     delete h;
     return PLE_ERR_OOM;
   }
-  cudaMemsetAsync(h->status, 0, 4, stream);
+  cudaMemsetAsync(h->status, 0, 8, stream);
   if (ple::launch_convert_w(static_cast<const __nv_bfloat16*>(weights->w_proj), c.row_dim, c.hidden, h->w16,
                             h->status, stream) != cudaSuccess) {
     free_all(h);
@@ -355,6 +369,9 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   if (cudaMemsetAsync(h->status, 0, 4, stream) != cudaSuccess ||
       !encode_2d(h, &h->tmap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->w16, c.row_dim, c.hidden,
                  static_cast<uint64_t>(c.row_dim) * 2, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      (h->decode_small &&
+       !encode_2d(h, &h->tmap_wd, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->w16, c.row_dim, c.hidden,
+                  static_cast<uint64_t>(c.row_dim) * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) ||
       cudaStreamSynchronize(stream) != cudaSuccess) {
     free_all(h);
     delete h;
@@ -435,6 +452,38 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
   if (!aligned(tokens, 4) || !aligned(hidden, 16) || !aligned(out, 16) || !aligned(hist, 4) ||
       !aligned(conv_state, 16) || (n_commit && !aligned(n_commit, 4)))
     return PLE_ERR_ALIGN;
+  const ple_config& c = h->cfg;
+  if (h->forward_path != 2 && h->decode_small && out != hidden && ple::decode_small_supported(B, q)) {
+    ple::DecodeSmallArgs a{};
+    a.tokens = tokens;
+    a.B = B;
+    a.q = q;
+    a.hist = hist;
+    a.conv_state = conv_state;
+    a.n_commit = n_commit;
+    a.vocab = c.vocab;
+    a.rows0 = c.rows[0];
+    a.rows1 = c.rows[1];
+    a.magic0 = ple::barrett_magic(c.rows[0]);
+    a.magic1 = ple::barrett_magic(c.rows[1]);
+    a.table = h->w.table;
+    a.scales = h->w.scales;
+    a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
+    a.conv_w = h->w.conv_w;
+    a.hidden = static_cast<const __nv_bfloat16*>(hidden);
+    a.out = out;
+    a.out_f32 = out_dtype == PLE_OUT_F32 ? 1 : 0;
+    a.H = c.hidden;
+    a.D = c.row_dim;
+    a.units_max = h->decode_plan.units_max;
+    a.slots = h->decode_plan.slots;
+    a.partial = h->decode_partial;
+    a.tile_count = h->tile_count;
+    a.tiles_done = h->status + 1;
+    a.status = h->status;
+    return run_stage(h, PLE_STAGE_GEMM, stream,
+                     [&] { return ple::launch_decode_small(h->tmap_wd, a, h->decode_plan.grid, stream); });
+  }
   return run_layer(h, tokens, B * q, nullptr, B, q, hidden, out, out_dtype, nullptr, hist, conv_state, n_commit,
                    stream);
 }

@@ -290,4 +290,34 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------------------------------ E4M3 dequantisation
+// e = fp16(a * s0 + b * s1) for 16 codes of two table rows (a, b): each code is
+// decoded exactly (E4M3 -> fp16 -> fp32 conversions; NaN codes stay NaN), the
+// sum is fmaf(a, s0, b * s1) in fp32, rounded to nearest even. Every kernel of
+// the library dequantises through this function.
+__device__ __forceinline__ float2 e4m3x2_cvt(uint32_t two_codes) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu),
+                                                     __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&hr));
+}
+
+__device__ __forceinline__ uint32_t deq2(uint32_t wa, uint32_t wb, int shift, float s0, float s1) {
+  const float2 a = e4m3x2_cvt(wa >> shift);
+  const float2 b = e4m3x2_cvt(wb >> shift);
+  const __half2 r = __floats2half2_rn(fmaf(a.x, s0, b.x * s1), fmaf(a.y, s0, b.y * s1));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// o0 = outputs of codes 0..7 (words a.x, a.y), o1 = codes 8..15.
+__device__ __forceinline__ void deq16(const uint4& a, const uint4& b, float s0, float s1, uint4& o0, uint4& o1) {
+  o0.x = deq2(a.x, b.x, 0, s0, s1);
+  o0.y = deq2(a.x, b.x, 16, s0, s1);
+  o0.z = deq2(a.y, b.y, 0, s0, s1);
+  o0.w = deq2(a.y, b.y, 16, s0, s1);
+  o1.x = deq2(a.z, b.z, 0, s0, s1);
+  o1.y = deq2(a.z, b.z, 16, s0, s1);
+  o1.z = deq2(a.w, b.w, 0, s0, s1);
+  o1.w = deq2(a.w, b.w, 16, s0, s1);
+}
+
 }  // namespace ple

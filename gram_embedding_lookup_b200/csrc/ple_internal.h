@@ -111,4 +111,44 @@ struct DecodeCombineArgs {
 };
 cudaError_t launch_combine_decode(const DecodeCombineArgs& a, cudaStream_t stream);
 
+// A whole decode step in one kernel for B * q <= 16 tokens, one CTA per SM.
+struct DecodeSmallArgs {
+  const int32_t* tokens;   // [B][q]
+  int32_t B, q;
+  int32_t* hist;           // [B][2] in/out
+  float* conv_state;       // [B][3][H] in/out
+  const int32_t* n_commit; // [B] or null
+  int32_t vocab;
+  int64_t rows0, rows1;
+  uint64_t magic0, magic1; // barrett_magic(rows0), barrett_magic(rows1)
+  const uint8_t* table;
+  const float* scales;
+  const __nv_bfloat16* w_gate;
+  const float* conv_w;
+  const __nv_bfloat16* hidden;
+  void* out;
+  int32_t out_f32;
+  int32_t H, D;
+  int32_t units_max;       // DecodePlan::units_max
+  int32_t slots;           // DecodePlan::slots
+  float* partial;          // [H / 16][slots][16 * 16] per-CTA tile sums
+  int32_t* tile_count;     // [H / 16], zero between launches
+  int32_t* tiles_done;     // zero between launches
+  int32_t* status;
+};
+// Work split of the single-kernel decode step for a layer shape and SM count.
+struct DecodePlan {
+  int32_t grid;            // CTAs (one per SM)
+  int32_t units_max;       // most 16 x 64 W_proj units one CTA owns
+  int32_t slots;           // most CTAs that share one 16-channel tile
+};
+// False when the shape does not fit the kernel (the step then runs split-K).
+bool decode_small_plan(int32_t H, int32_t D, int32_t num_sms, DecodePlan* plan);
+bool decode_small_supported(int32_t B, int32_t q);
+int64_t decode_small_partial_elems(const DecodePlan& plan, int32_t H);
+uint64_t barrett_magic(int64_t m);
+// tmap_w: fp16 W_proj [H][D], box 64 x 16, 128-byte swizzle.
+cudaError_t launch_decode_small(const CUtensorMap& tmap_w, const DecodeSmallArgs& a, int32_t grid,
+                                cudaStream_t stream);
+
 }  // namespace ple

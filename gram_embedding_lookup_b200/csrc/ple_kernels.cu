@@ -164,22 +164,6 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
-  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu),
-                                                     __NV_E4M3);
-  __half2 h;
-  h = *reinterpret_cast<const __half2*>(&hr);
-  return __half22float2(h);
-}
-
-// e = a*s0 + b*s1 for 4 codes per word, 16 codes per thread -> 16 fp16.
-__device__ __forceinline__ uint32_t combine_pair(uint32_t wa, uint32_t wb, int shift, float s0, float s1) {
-  const float2 a = e4m3x2_to_float2(wa >> shift);
-  const float2 b = e4m3x2_to_float2(wb >> shift);
-  const __half2 r = __floats2half2_rn(fmaf(a.x, s0, b.x * s1), fmaf(a.y, s0, b.y * s1));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-
 __global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ ids, int32_t T,
                                                      const uint8_t* __restrict__ table,
                                                      const float* __restrict__ scales, int64_t rows0,
@@ -202,14 +186,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ id
   const float s0 = __ldg(scales + row0);
   const float s1 = __ldg(scales + row1);
   uint4 o0, o1;
-  o0.x = combine_pair(a.x, b.x, 0, s0, s1);
-  o0.y = combine_pair(a.x, b.x, 16, s0, s1);
-  o0.z = combine_pair(a.y, b.y, 0, s0, s1);
-  o0.w = combine_pair(a.y, b.y, 16, s0, s1);
-  o1.x = combine_pair(a.z, b.z, 0, s0, s1);
-  o1.y = combine_pair(a.z, b.z, 16, s0, s1);
-  o1.z = combine_pair(a.w, b.w, 0, s0, s1);
-  o1.w = combine_pair(a.w, b.w, 16, s0, s1);
+  deq16(a, b, s0, s1, o0, o1);
   uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D + c * 16);
   dst[0] = o0;
   dst[1] = o1;
@@ -300,14 +277,7 @@ __global__ void __launch_bounds__(256) embed_kernel(const PrepareArgs a, int tok
   uint4* erow = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D);
   auto emit = [&](int j, const uint4& x, const uint4& y) {
     uint4 o0, o1;
-    o0.x = combine_pair(x.x, y.x, 0, s0, s1);
-    o0.y = combine_pair(x.x, y.x, 16, s0, s1);
-    o0.z = combine_pair(x.y, y.y, 0, s0, s1);
-    o0.w = combine_pair(x.y, y.y, 16, s0, s1);
-    o1.x = combine_pair(x.z, y.z, 0, s0, s1);
-    o1.y = combine_pair(x.z, y.z, 16, s0, s1);
-    o1.z = combine_pair(x.w, y.w, 0, s0, s1);
-    o1.w = combine_pair(x.w, y.w, 16, s0, s1);
+    deq16(x, y, s0, s1, o0, o1);
     erow[2 * j] = o0;
     erow[2 * j + 1] = o1;
   };

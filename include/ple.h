@@ -138,6 +138,7 @@ ple_status ple_forward(ple_handle* handle, const int32_t* tokens, int32_t T,
 /* One decode / speculative-verify step: B sequences with q new tokens each.
  * tokens int32 [B][q]; hidden bf16 [B*q][hidden]; out [B*q][hidden];
  * hist int32 [B][2] and conv_state fp32 [B][3][hidden] are read and updated.
+ * out may equal hidden only with PLE_OUT_BF16 (in-place residual add).
  * Outputs are computed for all q tokens; the state advances by the first
  * n_commit[b] tokens of sequence b (1 <= n_commit[b] <= q; NULL means q),
  * i.e. accepted draft tokens are committed and rejected ones rolled back. */
@@ -200,11 +201,13 @@ ple_status ple_set_profiling(ple_handle* handle, int32_t enable);
  * (launches[PLE_NUM_STAGES]) since the last call; then resets the counters. */
 ple_status ple_get_stage_times(ple_handle* handle, float* ms, int64_t* launches);
 
-/* Path selection for ple_forward: 0 = automatic, 1 = fused epilogue
+/* Path selection. For ple_forward: 0 = automatic, 1 = fused epilogue
  * (gate, conv and residual inside the projection kernel, conv halo
  * recomputed per tile; SM-pair tiles of 256 channels when hidden % 256 == 0),
  * 2 = split-K projection followed by a combine kernel, 3 = fused epilogue with
- * single-SM tiles of 128 channels. */
+ * single-SM tiles of 128 channels. For ple_decode_step: steps of B * q <= 16
+ * tokens with out != hidden run as one kernel unless path is 2, which forces
+ * the split-K path. */
 ple_status ple_set_forward_path(ple_handle* handle, int32_t path);
 
 /* Total number of kernels the handle has launched since creation. */

@@ -164,6 +164,45 @@ def test_gather_tiny_all_rows(tiny_layer):
     _check_fp16_rounding(_gather(tiny_layer, ids), O.embed(tiny_layer.host_table, ids))
 
 
+def test_gather_every_code_and_scale_kind(tiny_layer):
+    """Every E4M3 code (NaN codes 0x7F / 0xFF included) against every scale kind
+    the dequantisation distinguishes: ordinary, >= 2^7, subnormal, -0, NaN. The
+    first 256 rows of each order are overwritten and restored afterwards."""
+    L = tiny_layer
+    R, D = L.w.rows_per_order, L.w.row_dim
+    n = 256
+    k = np.arange(D)
+    codes = np.empty((2, n, D), np.uint8)
+    for i in range(n):
+        codes[0, i] = (i * D + k) % 256
+        codes[1, i] = (i * D + 5 * k + 17) % 256
+    kinds = np.array([0.0123, -3.5, 200.0, 127.9, 128.0, 1e-40, -0.0, np.nan, 2.0 ** -20, 65504 / 448,
+                      -1e-3, 7.25], np.float32)
+    scales = np.stack([kinds[np.arange(n) % len(kinds)], kinds[(np.arange(n) * 5 + 3) % len(kinds)]])
+    tab = L.table.view(2, R, D)
+    sc = L.scales.view(2, R)
+    saved = (tab[:, :n].clone(), sc[:, :n].clone())
+    try:
+        tab[:, :n] = torch.from_numpy(codes).cuda()
+        sc[:, :n] = torch.from_numpy(scales).cuda()
+        t = np.arange(2048)
+        ids = np.stack([t % n, (t * 37 + t // n) % n], axis=1)
+        got = _gather(L, ids)
+    finally:
+        tab[:, :n] = saved[0]
+        sc[:, :n] = saved[1]
+        torch.cuda.synchronize()
+    with np.errstate(invalid="ignore", over="ignore"):
+        ref = O.embed(O.ArrayTable(codes, scales), ids).astype(np.float16)
+    nan = np.isnan(ref)
+    assert nan.any() and np.array_equal(np.isnan(got), nan)
+    a = got[~nan].view(np.uint16).astype(np.int32)
+    b = ref[~nan].view(np.uint16).astype(np.int32)
+    ka = np.where(a & 0x8000, -(a & 0x7FFF), a & 0x7FFF)
+    kb = np.where(b & 0x8000, -(b & 0x7FFF), b & 0x7FFF)
+    assert np.abs(ka - kb).max() <= 1
+
+
 def test_gather_full_sample(full_layer):
     rng = np.random.default_rng(2)
     R = full_layer.w.rows_per_order
@@ -609,3 +648,83 @@ def test_forward_mid_in_place(mid_layer):
     torch.cuda.synchronize()
     ple.ple_set_forward_path(mid_layer.handle, 0)
     assert np.array_equal(to_bits(h), ref16)
+
+
+def test_decode_mid_in_place(mid_layer):
+    """out == hidden: every CTA of the single-kernel step reads whole hidden rows
+    for the gates, so an in-place step runs the split-K kernels; it must equal
+    the out-of-place split-K step bit for bit and stay within tolerance of the
+    single-kernel one."""
+    from tests.gpu_common import MID
+    B, q = 8, 1
+    rng = np.random.default_rng(77)
+    toks = rng.integers(0, MID.vocab, (B, q)).astype(np.int32)
+    hid = pi.hidden_bf16(rng, B * q, MID.hidden)
+    hist = rng.integers(-1, MID.vocab, (B, 2)).astype(np.int32)
+    conv = rng.standard_normal((B, 3, MID.hidden)).astype(np.float32)
+    single, h_s, c_s = gpu_decode(mid_layer, toks, hid, hist, conv, out_dtype=0)      # bf16 bits
+    ple.ple_set_forward_path(mid_layer.handle, 2)
+    split, _, _ = gpu_decode(mid_layer, toks, hid, hist, conv, out_dtype=0)
+    ple.ple_set_forward_path(mid_layer.handle, 0)
+    h = dev_bf16(hid)
+    hs = dev_i32(hist)
+    cs = torch.from_numpy(np.ascontiguousarray(conv, np.float32)).cuda()
+    ple.ple_decode_step(mid_layer.handle, dev_i32(toks), B, q, h, h, 0, hs, cs)
+    torch.cuda.synchronize()
+    assert ple.ple_get_error(mid_layer.handle) == 0
+    assert np.array_equal(to_bits(h), split)
+    assert np.array_equal(hs.cpu().numpy(), h_s)
+    assert_close(cs.cpu().numpy(), c_s, "in-place decode state")
+    W = mid_layer.host_weights
+    ref = O.ple_decode_step(toks, hid, W.w_proj, W.w_gate, W.conv_w, mid_layer.host_table, MID.rows_per_order,
+                            hist, conv)
+    assert_bf16_close(to_bits(h), ref["out"])
+    assert_bf16_close(single, ref["out"])
+
+
+# ----------------------------------------------------------------------------- decode: single-kernel path
+@pytest.mark.parametrize("shape", [(1, 1), (8, 1), (5, 3), (16, 1), (2, 8), (6, 3), (3, 7)])
+def test_decode_paths_tiny(tiny_layer, shape):
+    """B * q <= 16 runs the single-kernel step, larger steps the split-K path; both
+    match the oracle and each other (path 2 forces split-K)."""
+    w = tiny_layer.w
+    B, q = shape
+    rng = np.random.default_rng(B * 100 + q)
+    toks = rng.integers(0, w.vocab, (B, q)).astype(np.int32)
+    hid = pi.hidden_bf16(rng, B * q, w.hidden)
+    hist = rng.integers(-1, w.vocab, (B, 2)).astype(np.int32)
+    conv = rng.standard_normal((B, 3, w.hidden)).astype(np.float32)
+    nc = rng.integers(1, q + 1, B).astype(np.int32)
+    W = w.weights()
+    ref = O.ple_decode_step(toks, hid, W.w_proj, W.w_gate, W.conv_w, tiny_layer.host_table, w.rows_per_order,
+                            hist, conv, n_commit=nc)
+    outs = []
+    for path in (0, 2):
+        ple.ple_set_forward_path(tiny_layer.handle, path)
+        out, h2, c2 = gpu_decode(tiny_layer, toks, hid, hist, conv, nc)
+        ple.ple_set_forward_path(tiny_layer.handle, 0)
+        assert_close(out, ref["out"], f"decode {shape} path {path}")
+        assert np.array_equal(h2, ref["hist_out"])
+        assert_close(c2, ref["conv_out"], f"decode state {shape} path {path}")
+        outs.append(out)
+    assert np.abs(outs[0] - outs[1]).max() < 1e-4
+
+
+@pytest.mark.parametrize("shape", [(8, 1), (4, 3), (16, 1)])
+def test_decode_single_kernel_mid(mid_layer, shape):
+    from tests.gpu_common import MID
+    B, q = shape
+    rng = np.random.default_rng(B * 7 + q)
+    toks = rng.integers(0, MID.vocab, (B, q)).astype(np.int32)
+    hid = pi.hidden_bf16(rng, B * q, MID.hidden)
+    hist = rng.integers(-1, MID.vocab, (B, 2)).astype(np.int32)
+    conv = rng.standard_normal((B, 3, MID.hidden)).astype(np.float32)
+    W = mid_layer.host_weights
+    ref = O.ple_decode_step(toks, hid, W.w_proj, W.w_gate, W.conv_w, mid_layer.host_table, MID.rows_per_order,
+                            hist, conv)
+    out, h2, c2 = gpu_decode(mid_layer, toks, hid, hist, conv)
+    assert_close(out, ref["out"], f"mid decode {shape}")
+    assert np.array_equal(h2, ref["hist_out"])
+    assert_close(c2, ref["conv_out"], "mid decode state")
+    out16, _, _ = gpu_decode(mid_layer, toks, hid, hist, conv, out_dtype=0)
+    assert np.array_equal(out16, O.to_bf16_bits(out))
