@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "PLE layer tokens/s (prefill & decode) and gathered-row HBM GB/s vs peak, 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 GEMM_SOURCES = ["gram_embedding_lookup_b200/csrc/ple_gemm.cu", "gram_embedding_lookup_b200/csrc/ple_device.cuh"]
-GATHER_SOURCES = ["gram_embedding_lookup_b200/csrc/ple_kernels.cu"]
+GATHER_SOURCES = ["gram_embedding_lookup_b200/csrc/ple_kernels.cu", "gram_embedding_lookup_b200/csrc/ple_device.cuh"]
 
 
 def parse_args():

@@ -179,7 +179,7 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   pa.status = h->status;
   // row IDs, gate and the gathered, dequantised rows in one kernel
   ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
-    return ple::launch_embed(pa, h->w.table, h->w.scales, c.row_dim, h->e, stream);
+    return ple::launch_embed(pa, h->w.table, h->w.scales, c.row_dim, h->e, h->num_sms, stream);
   });
   if (st != PLE_OK) return st;
 

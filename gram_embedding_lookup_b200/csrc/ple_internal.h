@@ -23,6 +23,7 @@ struct PrepareArgs {
   const int32_t* hist;         // [S][2] or null
   int32_t vocab;
   int64_t rows0, rows1;
+  uint64_t magic0, magic1;     // floor((2^64 - 1) / rows): set by the launchers
   int32_t* ids;                // [T][2]
   const __nv_bfloat16* hidden; // [T][H] (null: ids only)
   const __nv_bfloat16* w_gate; // [H]
@@ -35,10 +36,10 @@ struct PrepareArgs {
 };
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
 
-// Prepare and gather fused (one warp per token, one pass over HBM): ids,
-// metadata with the gate, and e[t] for the batch.
+// Prepare and gather fused (one pass over HBM): ids, metadata with the gate,
+// and e[t] for the batch. num_sms sizes the persistent grid.
 cudaError_t launch_embed(const PrepareArgs& a, const uint8_t* table, const float* scales, int32_t D, __half* e,
-                         cudaStream_t stream);
+                         int32_t num_sms, cudaStream_t stream);
 
 // Gather stage: e[t] = deq(row of order 0) + deq(row of order 1), fp16.
 cudaError_t launch_gather(const int32_t* ids, int32_t T, const uint8_t* table, const float* scales,

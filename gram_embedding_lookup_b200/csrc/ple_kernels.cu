@@ -15,6 +15,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "ple_device.cuh"
 #include "ple_internal.h"
 
@@ -30,6 +32,22 @@ __device__ __forceinline__ uint64_t context_of(int32_t tok) {
 }
 
 __device__ __forceinline__ uint64_t fold64(uint64_t k) { return k ^ (k >> 32); }
+
+// x mod m for m < 2^31 by Barrett reduction with magic = floor((2^64 - 1) / m):
+// the quotient estimate umulhi(x, magic) is at most 2 below floor(x / m).
+__device__ __forceinline__ uint64_t mod_barrett(uint64_t x, uint64_t m, uint64_t magic) {
+  uint64_t r = x - __umul64hi(x, magic) * m;
+  if (r >= m) r -= m;
+  if (r >= m) r -= m;
+  return r;
+}
+
+PrepareArgs with_magic(const PrepareArgs& in) {
+  PrepareArgs a = in;
+  a.magic0 = ~0ull / static_cast<uint64_t>(a.rows0);
+  a.magic1 = ~0ull / static_cast<uint64_t>(a.rows1);
+  return a;
+}
 
 // Sequence, position, last-token flag and the two row IDs of token t (every
 // lane of the calling warp computes the same values; lane 0 reports errors).
@@ -67,28 +85,29 @@ __device__ __forceinline__ void sequence_and_rows(const PrepareArgs& a, int t, i
   const uint64_t x2 = pos >= 2 ? context_of(a.tokens[t - 2]) : (pos == 1 ? carried(1) : carried(2));
   const uint64_t k2 = (x0 * kP0) ^ (x1 * kP1);
   const uint64_t k3 = k2 ^ (x2 * kP2);
-  r0 = static_cast<int32_t>(fold64(k2) % static_cast<uint64_t>(a.rows0));
-  r1 = static_cast<int32_t>(fold64(k3) % static_cast<uint64_t>(a.rows1));
+  r0 = static_cast<int32_t>(mod_barrett(fold64(k2), static_cast<uint64_t>(a.rows0), a.magic0));
+  r1 = static_cast<int32_t>(mod_barrett(fold64(k3), static_cast<uint64_t>(a.rows1), a.magic1));
 }
 
-// The state and offsets blocks of the prepare / embed kernels.
-__device__ __forceinline__ void state_blocks(const PrepareArgs& a, int sb, int nsb) {
+// The state and offsets work of the prepare / embed kernels, by threads
+// [0, nthr) of blocks sb of nsb (tid: the calling thread's index among them).
+__device__ __forceinline__ void state_blocks(const PrepareArgs& a, int sb, int nsb, int tid, int nthr) {
   if (sb == 0 && a.uniform_q == 0) {
     // offsets must start at 0, end at T and be non-decreasing
-    if (threadIdx.x == 0 && (a.offsets[0] != 0 || a.offsets[a.S] != a.T)) set_status(a.status, PLE_ERR_RANGE);
-    for (int s = threadIdx.x; s < a.S; s += blockDim.x)
+    if (tid == 0 && (a.offsets[0] != 0 || a.offsets[a.S] != a.T)) set_status(a.status, PLE_ERR_RANGE);
+    for (int s = tid; s < a.S; s += nthr)
       if (a.offsets[s] > a.offsets[s + 1]) set_status(a.status, PLE_ERR_RANGE);
   }
   if (a.conv_in != nullptr) {
     const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
     const float4* src = reinterpret_cast<const float4*>(a.conv_in);
     float4* dst = reinterpret_cast<float4*>(a.conv_copy);
-    for (int64_t i = static_cast<int64_t>(sb) * blockDim.x + threadIdx.x; i < n4;
-         i += static_cast<int64_t>(nsb) * blockDim.x)
+    for (int64_t i = static_cast<int64_t>(sb) * nthr + tid; i < n4;
+         i += static_cast<int64_t>(nsb) * nthr)
       dst[i] = src[i];
   }
   if (a.hist_new != nullptr && sb == 0) {
-    for (int s = threadIdx.x; s < a.S; s += blockDim.x) {
+    for (int s = tid; s < a.S; s += nthr) {
       int32_t begin, end;
       if (a.uniform_q > 0) { begin = s * a.uniform_q; end = begin + a.uniform_q; }
       else { begin = a.offsets[s]; end = a.offsets[s + 1]; }
@@ -115,7 +134,7 @@ __global__ void __launch_bounds__(256) prepare_kernel(const PrepareArgs a, int t
   const int lane = threadIdx.x & 31;
 
   if (static_cast<int>(blockIdx.x) >= token_blocks) {
-    state_blocks(a, blockIdx.x - token_blocks, gridDim.x - token_blocks);
+    state_blocks(a, blockIdx.x - token_blocks, gridDim.x - token_blocks, threadIdx.x, blockDim.x);
     return;
   }
 
@@ -193,100 +212,182 @@ __global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ id
 }
 
 // ------------------------------------------------------------------ embed (prepare + gather)
-// One warp per token does, in one pass over HBM: the sequence map and row IDs,
-// the gate dot product over h_t, and the row gather with E4M3 dequantisation
-// into fp16 e_t. The h loads are issued first so that they overlap the hash,
-// and both rows' loads are issued before any arithmetic on them. Rows up to
-// 2560 codes and hidden sizes up to 2560 stay in registers; larger sizes take
-// a tail loop.
-constexpr int kEmbedH4 = 10;    // uint4 of h per lane held in registers
-constexpr int kEmbedD16 = 5;    // 16-code chunks per lane and row held in registers
+constexpr int kEmbedH4 = 10;    // uint4 of h per lane held in registers (hidden <= 2560)
+constexpr int kEmbedD16 = 5;    // 16-code chunks per lane and row held in registers (rows <= 2560 codes)
 
-__global__ void __launch_bounds__(256) embed_kernel(const PrepareArgs a, int token_blocks,
-                                                    const uint8_t* __restrict__ table,
-                                                    const float* __restrict__ scales, int32_t D,
-                                                    __half* __restrict__ e) {
+// ------------------------------------------------------------------ embed, pipelined
+// n-gram row IDs, the gate dot product over h_t, and the row gather with E4M3
+// dequantisation into fp16 e_t, in one pass over HBM. One persistent CTA per
+// SM takes a contiguous range of tokens. Its
+// producer warp computes the row IDs of 30 tokens at a time (a lane per token)
+// into a ring of kPipeBatches batches in shared memory. Each of the 15
+// consumer warps takes two tokens of every batch and issues all of a token's
+// loads at once: its hidden row and its two table rows (plain 16-byte loads,
+// which keep more bytes in flight per SM than bulk copies of single rows do).
+// Then come the gate dot product (fp32, lane-strided, then a warp reduction),
+// the dequantisation into fp16 e_t and the metadata. Batches go through the
+// ring in order, so every parity wait is for the phase after the one last
+// released.
+constexpr int kPipeConsumers = 15;                   // 16 warps in all: 128 registers per thread
+constexpr int kPipeThreads = 32 * (1 + kPipeConsumers);
+constexpr int kPipeBatch = 2 * kPipeConsumers;       // tokens per batch: 2 per consumer warp
+static_assert(kPipeBatch <= 32, "a producer lane per token of a batch");
+constexpr int kPipeBatches = 4;                      // batches in the ring
+
+struct PipeTok {                                     // per token, written by the producer
+  int32_t r0, r1, seq, pos, flags, pad0, pad1, pad2;
+};
+
+struct PipeSmem {
+  PipeTok tok[kPipeBatches][kPipeBatch];
+  uint64_t full[kPipeBatches];                       // producer -> consumers (count 1)
+  uint64_t empty[kPipeBatches];                      // consumers -> producer (count kPipeConsumers)
+};
+
+__global__ void __launch_bounds__(kPipeThreads, 1)
+    embed_pipe_kernel(const PrepareArgs a, const uint8_t* __restrict__ table, const float* __restrict__ scales,
+                      int32_t D, __half* __restrict__ e) {
+  __shared__ PipeSmem sm;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (static_cast<int>(blockIdx.x) >= token_blocks) {
-    state_blocks(a, blockIdx.x - token_blocks, gridDim.x - token_blocks);
-    return;
-  }
-  const int t = blockIdx.x * kPrepWarps + warp;
-  if (t >= a.T) return;
-
-  const int H8 = a.H / 8;
-  const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
-  uint4 hv[kEmbedH4];
-#pragma unroll
-  for (int r = 0; r < kEmbedH4; ++r) {
-    const int j = lane + 32 * r;
-    hv[r] = j < H8 ? ld_stream_v4(hrow + j) : make_uint4(0u, 0u, 0u, 0u);
-  }
-
-  int32_t s, pos, last, r0, r1;
-  sequence_and_rows(a, t, lane, s, pos, last, r0, r1);
-  const int D16 = D / 16;
-  const uint8_t* ra = table + static_cast<int64_t>(r0) * D;
-  const uint8_t* rb = table + (a.rows0 + r1) * D;
-  uint4 ca[kEmbedD16], cb[kEmbedD16];
-#pragma unroll
-  for (int r = 0; r < kEmbedD16; ++r) {
-    const int j = lane + 32 * r;
-    if (j < D16) {
-      ca[r] = ld_stream_v4(ra + 16 * j);
-      cb[r] = ld_stream_v4(rb + 16 * j);
+  const int t0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * a.T / gridDim.x);
+  const int t1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * a.T / gridDim.x);
+  const int n = t1 - t0;
+  const int nb = (n + kPipeBatch - 1) / kPipeBatch;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPipeBatches; ++i) {
+      mbar_init(smem_u32(&sm.full[i]), 1);
+      mbar_init(smem_u32(&sm.empty[i]), kPipeConsumers);
     }
+    fence_barrier_init();
   }
-  const float s0 = __ldg(scales + r0);
-  const float s1 = __ldg(scales + a.rows0 + r1);
-  if (lane == 0) reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
+  __syncthreads();
 
-  // gate: g = sigmoid(w_gate . h_t), fp32, the same summation order as prepare_kernel
-  const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
-  float acc = 0.f;
-  auto dot8 = [&](const uint4& hq, const uint4& wq) {
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
-    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 hf = __bfloat1622float2(h2[q]);
-      const float2 wf = __bfloat1622float2(w2[q]);
-      acc = fmaf(hf.x, wf.x, acc);
-      acc = fmaf(hf.y, wf.y, acc);
+  if (warp == 0) {
+    // ---- producer: row IDs, a lane per token
+    for (int b = 0; b < nb; ++b) {
+      const int slot = b % kPipeBatches, round = b / kPipeBatches;
+      if (round > 0 && !mbar_wait(smem_u32(&sm.empty[slot]), (round - 1) & 1)) {
+        if (lane == 0) set_status(a.status, PLE_ERR_TIMEOUT);
+        break;
+      }
+      const int k = b * kPipeBatch + lane;
+      if (lane < kPipeBatch && k < n) {
+        int32_t s, pos, last, r0, r1;
+        sequence_and_rows(a, t0 + k, 0, s, pos, last, r0, r1);
+        reinterpret_cast<int2*>(a.ids)[t0 + k] = make_int2(r0, r1);
+        PipeTok& pt = sm.tok[slot][lane];
+        pt.r0 = r0;
+        pt.r1 = r1;
+        pt.seq = s;
+        pt.pos = pos;
+        pt.flags = last ? kFlagLast : 0;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.full[slot]));
     }
-  };
+  } else {
+    // ---- consumers: two tokens of every batch, lane-parallel within the warp.
+    //      A token's hidden row does not depend on its row IDs, so the loads of
+    //      the first one are issued before the wait for the batch (the first
+    //      time, the conv-state snapshot, the new token history and the offsets
+    //      check run meanwhile). Every warp waits for every batch, so that its
+    //      release of a slot always counts in the slot's current round.
+    const int cw = warp - 1;
+    const int H8 = a.H / 8;
+    const int D16 = D / 16;
+    const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+    bool state_done = false;
+    for (int b = 0; b < nb; ++b) {
+      const int slot = b % kPipeBatches, round = b / kPipeBatches;
+      uint4 hv[kEmbedH4], ca[kEmbedD16], cb[kEmbedD16];
+      auto load_hidden = [&](int t) {
+        const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
 #pragma unroll
-  for (int r = 0; r < kEmbedH4; ++r) {
-    const int j = lane + 32 * r;
-    if (j < H8) dot8(hv[r], __ldg(wg + j));
-  }
-  for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) dot8(ld_stream_v4(hrow + j), __ldg(wg + j));
+        for (int r = 0; r < kEmbedH4; ++r) {
+          const int j = lane + 32 * r;
+          if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+        }
+      };
+      if (b * kPipeBatch + cw < n) load_hidden(t0 + b * kPipeBatch + cw);
+      if (!state_done) {
+        state_blocks(a, blockIdx.x, gridDim.x, threadIdx.x - 32, blockDim.x - 32);
+        state_done = true;
+      }
+      if (!mbar_wait(smem_u32(&sm.full[slot]), round & 1)) {
+        if (lane == 0) set_status(a.status, PLE_ERR_TIMEOUT);
+        break;
+      }
+#pragma unroll 1
+      for (int half = 0; half < kPipeBatch / kPipeConsumers; ++half) {
+        const int i = cw + kPipeConsumers * half;
+        const int k = b * kPipeBatch + i;
+        if (k >= n) break;                                   // warp-uniform
+        const int t = t0 + k;
+        const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+        if (half > 0) load_hidden(t);
+        const PipeTok pt = sm.tok[slot][i];
+        const uint8_t* ra = table + static_cast<int64_t>(pt.r0) * D;
+        const uint8_t* rb = table + (a.rows0 + pt.r1) * D;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) {
-    TokMeta m;
-    m.g = 1.0f / (1.0f + expf(-acc));
-    m.seq = s;
-    m.pos = pos;
-    m.flags = last ? kFlagLast : 0;
-    a.meta[t] = m;
-  }
-
-  // e_t = deq(bigram row) + deq(trigram row), fp16
-  uint4* erow = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D);
-  auto emit = [&](int j, const uint4& x, const uint4& y) {
-    uint4 o0, o1;
-    deq16(x, y, s0, s1, o0, o1);
-    erow[2 * j] = o0;
-    erow[2 * j + 1] = o1;
-  };
+        for (int r = 0; r < kEmbedD16; ++r) {
+          const int j = lane + 32 * r;
+          if (j < D16) {
+            ca[r] = ld_stream_v4(ra + 16 * j);
+            cb[r] = ld_stream_v4(rb + 16 * j);
+          }
+        }
+        const float s0 = __ldg(scales + pt.r0);
+        const float s1 = __ldg(scales + a.rows0 + pt.r1);
+        // gate: g = sigmoid(w_gate . h_t), fp32
+        float acc = 0.f;
+        auto dot8 = [&](const uint4& hq, const uint4& wq) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
+          const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
 #pragma unroll
-  for (int r = 0; r < kEmbedD16; ++r) {
-    const int j = lane + 32 * r;
-    if (j < D16) emit(j, ca[r], cb[r]);
+          for (int q = 0; q < 4; ++q) {
+            const float2 hf = __bfloat1622float2(h2[q]);
+            const float2 wf = __bfloat1622float2(w2[q]);
+            acc = fmaf(hf.x, wf.x, acc);
+            acc = fmaf(hf.y, wf.y, acc);
+          }
+        };
+#pragma unroll
+        for (int r = 0; r < kEmbedH4; ++r) {
+          const int j = lane + 32 * r;
+          if (j < H8) dot8(hv[r], __ldg(wg + j));
+        }
+        for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) dot8(ld_stream_v4(hrow + j), __ldg(wg + j));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+          TokMeta m;
+          m.g = 1.0f / (1.0f + expf(-acc));
+          m.seq = pt.seq;
+          m.pos = pt.pos;
+          m.flags = pt.flags;
+          a.meta[t] = m;
+        }
+        // e_t = deq(bigram row) + deq(trigram row), fp16
+        uint4* erow = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D);
+        auto emit = [&](int j, const uint4& x, const uint4& y) {
+          uint4 o0, o1;
+          deq16(x, y, s0, s1, o0, o1);
+          erow[2 * j] = o0;
+          erow[2 * j + 1] = o1;
+        };
+#pragma unroll
+        for (int r = 0; r < kEmbedD16; ++r) {
+          const int j = lane + 32 * r;
+          if (j < D16) emit(j, ca[r], cb[r]);
+        }
+        for (int j = lane + 32 * kEmbedD16; j < D16; j += 32) emit(j, ld_stream_v4(ra + 16 * j), ld_stream_v4(rb + 16 * j));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.empty[slot]));
+    }
+    if (!state_done) state_blocks(a, blockIdx.x, gridDim.x, threadIdx.x - 32, blockDim.x - 32);
   }
-  for (int j = lane + 32 * kEmbedD16; j < D16; j += 32) emit(j, ld_stream_v4(ra + 16 * j), ld_stream_v4(rb + 16 * j));
 }
 
 // ------------------------------------------------------------------ W_proj conversion
@@ -400,20 +501,16 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
     const int64_t want = (n4 + 255) / 256;
     state_blocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
   }
-  prepare_kernel<<<token_blocks + state_blocks, 256, 0, stream>>>(a, token_blocks);
+  prepare_kernel<<<token_blocks + state_blocks, 256, 0, stream>>>(with_magic(a), token_blocks);
   return cudaGetLastError();
 }
 
 cudaError_t launch_embed(const PrepareArgs& a, const uint8_t* table, const float* scales, int32_t D, __half* e,
-                         cudaStream_t stream) {
-  const int token_blocks = (a.T + kPrepWarps - 1) / kPrepWarps;
-  int state_blocks = 1;
-  if (a.conv_in != nullptr) {
-    const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
-    const int64_t want = (n4 + 255) / 256;
-    state_blocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
-  }
-  embed_kernel<<<token_blocks + state_blocks, 256, 0, stream>>>(a, token_blocks, table, scales, D, e);
+                         int32_t num_sms, cudaStream_t stream) {
+  const bool state = a.conv_in != nullptr || a.hist_new != nullptr;
+  // small batches spread over the SMs: a few tokens per CTA, no warp taking two in turn
+  const int grid = state ? num_sms : std::min<int>(num_sms, a.T);
+  embed_pipe_kernel<<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, scales, D, e);
   return cudaGetLastError();
 }
 
