@@ -42,6 +42,8 @@ details. The readings fixed here (each marked READING) are:
        token; u before a fresh sequence is 0, else the carried state.
 * C-10 out = h + y.
 * C-12 carried state: the last two tokens and the last three u rows.
+* C-16 the NVFP4 table variant: FP4 E2M1 codes, two per byte (low nibble
+       first), an E4M3 scale per 16 codes and the C-6 row scale.
 
 Precision: every step is evaluated in float64 (library matmul for the
 projection and the gate dot product); the caller rounds the float64 result
@@ -85,6 +87,54 @@ def e4m3_decode(code: int) -> float:
 
 
 E4M3_VALUES = np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+# --------------------------------------------------------------------------------------
+# C-16  NVFP4 table rows (READING): FP4 E2M1 codes with an E4M3 scale per 16 codes
+# --------------------------------------------------------------------------------------
+# The pages' capacity variant quantises the PLE table to NVFP4, about 26.82 GiB
+# against 95.37 GiB in BF16 (deletoe.com page, section "第三条路：把 PLE 也量化，
+# 能塞下，但不够快"; DGX Spark report, section "运行时内存占用"), a packed table of
+# "NVFP4 code" and "FP8 scale" (DGX Spark report, section "小结"). 26.82 GiB for
+# the same 51.2 G elements is 4.5 bits per element: a 4-bit code per element and
+# an 8-bit scale per 16 elements. The layout is not on the pages; this build
+# reads it as: codes u8 [2][R][D/2], element 2i in the low nibble of byte i and
+# element 2i+1 in the high nibble; block scales E4M3 u8 [2][R][D/16], block j
+# covering elements [16j, 16j+16); and the per-row fp32 scale of C-6 kept as
+# the outer factor:  deq[k] = e2m1(code_k) * e4m3(block_scale[k // 16]) * scale.
+
+def e2m1_decode(code: int) -> float:
+    """Value of one FP4 E2M1 code: sign bit, 2 exponent bits (bias 1), 1 mantissa bit.
+
+    exponent field 0: (-1)^s * m * 0.5   (subnormal; m = 0 is zero)
+    otherwise:        (-1)^s * (1 + m/2) * 2^(e-1)
+    The format has no infinities and no NaN (max magnitude 6)."""
+    code = int(code) & 0xF
+    s = code >> 3
+    e = (code >> 1) & 0x3
+    m = code & 0x1
+    mag = m * 0.5 if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1)
+    return -mag if s else mag
+
+
+E2M1_VALUES = np.array([e2m1_decode(c) for c in range(16)], dtype=np.float64)
+
+
+def unpack_fp4(packed: np.ndarray) -> np.ndarray:
+    """uint8 [..., D/2] of two codes per byte -> uint8 codes [..., D] (low nibble first)."""
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def dequantise_nvfp4(packed: np.ndarray, block_scales: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """deq[i][k] = e2m1(code[i][k]) * e4m3(block_scales[i][k // 16]) * scales[i]   (C-16)."""
+    codes = unpack_fp4(packed)
+    blocks = E4M3_VALUES[np.asarray(block_scales, dtype=np.uint8)]
+    per_elem = np.repeat(blocks, 16, axis=-1)
+    return E2M1_VALUES[codes] * per_elem * np.asarray(scales, np.float64)[:, None]
 
 
 # --------------------------------------------------------------------------------------
@@ -192,14 +242,21 @@ def dequantise(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return E4M3_VALUES[np.asarray(codes, dtype=np.uint8)] * np.asarray(scales, np.float64)[:, None]
 
 
-def embed(table, ids: np.ndarray) -> np.ndarray:
-    """e_t = deq(bigram row of t) + deq(trigram row of t)   (C-7).
+def table_rows(table, order: int, rows) -> np.ndarray:
+    """Dequantised rows of sub-table ``order`` (C-6 for an FP8 table, C-16 for NVFP4).
 
-    ``table`` supplies ``codes(order, rows)`` and ``scales(order, rows)``."""
+    ``table`` supplies ``codes(order, rows)`` and ``scales(order, rows)``, and for
+    ``table.format == "nvfp4"`` also ``block_scales(order, rows)``."""
+    if getattr(table, "format", "e4m3") == "nvfp4":
+        return dequantise_nvfp4(table.codes(order, rows), table.block_scales(order, rows),
+                                table.scales(order, rows))
+    return dequantise(table.codes(order, rows), table.scales(order, rows))
+
+
+def embed(table, ids: np.ndarray) -> np.ndarray:
+    """e_t = deq(bigram row of t) + deq(trigram row of t)   (C-7)."""
     ids = np.asarray(ids, dtype=np.int64)
-    e = dequantise(table.codes(0, ids[:, 0]), table.scales(0, ids[:, 0]))
-    e = e + dequantise(table.codes(1, ids[:, 1]), table.scales(1, ids[:, 1]))
-    return e
+    return table_rows(table, 0, ids[:, 0]) + table_rows(table, 1, ids[:, 1])
 
 
 class ArrayTable:
@@ -214,6 +271,20 @@ class ArrayTable:
 
     def scales(self, order, rows):
         return self._scales[order][np.asarray(rows, dtype=np.int64)]
+
+
+class Nvfp4ArrayTable(ArrayTable):
+    """An NVFP4 table held in arrays (C-16): packed codes uint8 [2][R][D/2], block
+    scales uint8 (E4M3) [2][R][D/16], row scales float32 [2][R]."""
+
+    format = "nvfp4"
+
+    def __init__(self, codes: np.ndarray, block_scales: np.ndarray, scales: np.ndarray):
+        super().__init__(codes, scales)
+        self._block_scales = block_scales
+
+    def block_scales(self, order, rows):
+        return self._block_scales[order][np.asarray(rows, dtype=np.int64)]
 
 
 # --------------------------------------------------------------------------------------

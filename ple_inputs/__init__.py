@@ -34,7 +34,8 @@ __all__ = [
     "GAMMA", "splitmix64_stream", "table_codes", "table_scales", "SynthTable",
     "f32_to_bf16_bits", "Weights", "make_weights", "tokens_uniform", "tokens_zipf",
     "hidden_bf16", "WORKLOADS", "Workload", "workload", "prefill_batch",
-    "decode_batch", "long_chunks", "mtp_session", "fill_table_device",
+    "decode_batch", "long_chunks", "mtp_session", "fill_table_device", "nv_table_codes",
+    "nv_table_block_scales", "SynthNvTable", "fill_nv_table_device",
 ]
 
 _U64 = np.uint64
@@ -43,6 +44,9 @@ _MIX1 = 0xBF58476D1CE4E5B9
 _MIX2 = 0x94D049BB133111EB
 TAG_CODES = 1
 TAG_SCALES = 2
+TAG_NV_CODES = 3                     # NVFP4 table: packed E2M1 code bytes
+TAG_NV_BLOCKS = 4                    # NVFP4 table: E4M3 block-scale bytes
+NV_BLOCK_BASE = 0x30                 # block-scale codes 0x30..0x3F: E4M3 0.5 .. 1.875
 N_FINITE_E4M3 = 254                  # 256 codes minus the two NaN codes 0x7F / 0xFF
 
 
@@ -108,6 +112,32 @@ def table_scales(seed: int, rows_per_order: int, order: int,
     return _u64_to_scale(splitmix64_stream(seed, TAG_SCALES, idx.astype(_U64)))
 
 
+def nv_table_codes(seed: int, rows_per_order: int, row_dim: int, order: int,
+                   rows: np.ndarray) -> np.ndarray:
+    """Packed NVFP4 code bytes (two E2M1 codes each, all 16 codes equally likely)
+    of the given rows of sub-table ``order``: uint8 [len(rows)][row_dim / 2].
+
+    Byte k of row r of order n is the top byte of counter index ((n * R + r) * D/2 + k)."""
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1)
+    half = row_dim // 2
+    base = (np.int64(order) * np.int64(rows_per_order) + rows) * np.int64(half)
+    idx = base[:, None] + np.arange(half, dtype=np.int64)[None, :]
+    return (splitmix64_stream(seed, TAG_NV_CODES, idx.astype(_U64)) >> _U64(56)).astype(np.uint8)
+
+
+def nv_table_block_scales(seed: int, rows_per_order: int, row_dim: int, order: int,
+                          rows: np.ndarray) -> np.ndarray:
+    """E4M3 block-scale bytes (codes 0x30..0x3F, i.e. 0.5 .. 1.875) of the given rows:
+    uint8 [len(rows)][row_dim / 16]. Byte j of row r of order n is drawn from counter
+    index ((n * R + r) * D/16 + j): NV_BLOCK_BASE + the draw's top 4 bits."""
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1)
+    nb = row_dim // 16
+    base = (np.int64(order) * np.int64(rows_per_order) + rows) * np.int64(nb)
+    idx = base[:, None] + np.arange(nb, dtype=np.int64)[None, :]
+    u = splitmix64_stream(seed, TAG_NV_BLOCKS, idx.astype(_U64))
+    return (np.uint64(NV_BLOCK_BASE) + (u >> _U64(60))).astype(np.uint8)
+
+
 @dataclass
 class SynthTable:
     """Host view of the synthetic table [2][R][D] + scales [2][R] (rows made on demand)."""
@@ -129,6 +159,34 @@ class SynthTable:
         codes = np.stack([self.codes(0, r), self.codes(1, r)])
         scales = np.stack([self.scales(0, r), self.scales(1, r)])
         return codes, scales
+
+
+@dataclass
+class SynthNvTable:
+    """Host view of a synthetic NVFP4 table: packed codes [2][R][D/2], E4M3 block
+    scales [2][R][D/16] and the same per-row fp32 scales as the FP8 table."""
+    seed: int
+    rows_per_order: int
+    row_dim: int
+    format: str = "nvfp4"
+
+    def codes(self, order: int, rows) -> np.ndarray:
+        return nv_table_codes(self.seed, self.rows_per_order, self.row_dim, order, rows)
+
+    def block_scales(self, order: int, rows) -> np.ndarray:
+        return nv_table_block_scales(self.seed, self.rows_per_order, self.row_dim, order, rows)
+
+    def scales(self, order: int, rows) -> np.ndarray:
+        return table_scales(self.seed, self.rows_per_order, order, rows)
+
+    def full(self):
+        """The whole table as arrays (small tables only): codes, block scales, scales."""
+        r = np.arange(self.rows_per_order)
+        if self.rows_per_order * self.row_dim > (1 << 28):
+            raise ValueError("table too large to materialise on the host")
+        return (np.stack([self.codes(0, r), self.codes(1, r)]),
+                np.stack([self.block_scales(0, r), self.block_scales(1, r)]),
+                np.stack([self.scales(0, r), self.scales(1, r)]))
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -330,10 +388,23 @@ def _synth_lib():
         lib.ple_synth_fill_table.restype = ctypes.c_int
         lib.ple_synth_fill_table.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                              ctypes.c_int32, ctypes.c_uint64, ctypes.c_void_p]
+        lib.ple_synth_fill_nvfp4.restype = ctypes.c_int
+        lib.ple_synth_fill_nvfp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                             ctypes.c_int32, ctypes.c_uint64, ctypes.c_void_p]
         lib.ple_synth_stream_base.restype = ctypes.c_uint64
         lib.ple_synth_stream_base.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
         _SYNTH_LIB = lib
     return _SYNTH_LIB
+
+
+def fill_nv_table_device(codes_ptr: int, block_ptr: int, scales_ptr: int, rows_per_order: int,
+                         row_dim: int, seed: int, stream: int = 0) -> None:
+    """Fill a device NVFP4 table: codes u8[2][R][D/2], block scales u8[2][R][D/16], scales f32[2][R]."""
+    rc = _synth_lib().ple_synth_fill_nvfp4(ctypes.c_void_p(codes_ptr), ctypes.c_void_p(block_ptr),
+                                           ctypes.c_void_p(scales_ptr), rows_per_order, row_dim, seed,
+                                           ctypes.c_void_p(stream))
+    if rc != 0:
+        raise RuntimeError(f"ple_synth_fill_nvfp4 failed with CUDA error {rc}")
 
 
 def fill_table_device(table_ptr: int, scales_ptr: int, rows_per_order: int, row_dim: int,
