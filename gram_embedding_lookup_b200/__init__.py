@@ -16,7 +16,8 @@ __all__ = [
     "PleError", "PleConfig", "PleWeights", "PleState", "lib", "ple_create", "ple_destroy",
     "ple_ngram_ids", "ple_gather_rows", "ple_forward", "ple_decode_step", "ple_get_error",
     "ple_status_string", "ple_set_profiling", "ple_get_stage_times", "ple_set_forward_path",
-    "ple_launch_count", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32", "STATUS",
+    "ple_launch_count", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32",
+    "PLE_TABLE_E4M3", "PLE_TABLE_NVFP4", "STATUS",
     "STAGES", "LIB_PATH",
 ]
 
@@ -24,6 +25,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libple.so")
 
 PLE_OUT_BF16 = 0
 PLE_OUT_F32 = 1
+PLE_TABLE_E4M3 = 0
+PLE_TABLE_NVFP4 = 1
 PLE_STATIC_MAX_TOKENS = 16384   # the fixed row-ID array of ple_embed_static
 STATUS = {0: "PLE_OK", 1: "PLE_ERR_INVALID_ARG", 2: "PLE_ERR_SHAPE", 3: "PLE_ERR_ALIGN", 4: "PLE_ERR_RANGE",
           5: "PLE_ERR_OOM", 6: "PLE_ERR_CUDA", 7: "PLE_ERR_TIMEOUT", 8: "PLE_ERR_UNSUPPORTED"}
@@ -39,13 +42,13 @@ class PleError(RuntimeError):
 
 class PleConfig(ctypes.Structure):
     _fields_ = [("vocab", ctypes.c_int32), ("hidden", ctypes.c_int32), ("row_dim", ctypes.c_int32),
-                ("max_tokens", ctypes.c_int32), ("max_seqs", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int32), ("max_seqs", ctypes.c_int32), ("table_format", ctypes.c_int32),
                 ("rows", ctypes.c_int64 * 2)]
 
 
 class PleWeights(ctypes.Structure):
     _fields_ = [("table", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("w_proj", ctypes.c_void_p),
-                ("w_gate", ctypes.c_void_p), ("conv_w", ctypes.c_void_p)]
+                ("w_gate", ctypes.c_void_p), ("conv_w", ctypes.c_void_p), ("block_scales", ctypes.c_void_p)]
 
 
 class PleState(ctypes.Structure):

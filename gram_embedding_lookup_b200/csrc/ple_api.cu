@@ -129,6 +129,11 @@ bool encode_2d(ple_handle* h, CUtensorMap* map, CUtensorMapDataType dt, const vo
   return r == CUDA_SUCCESS;
 }
 
+ple::TableRef table_ref(const ple_handle* h) {
+  const bool nv = h->cfg.table_format == PLE_TABLE_NVFP4;
+  return ple::TableRef{h->w.table, nv ? h->w.block_scales : nullptr, h->w.scales, nv ? 1 : 0};
+}
+
 void free_all(ple_handle* h) {
   cudaFree(h->w16);
   cudaFree(h->e);
@@ -179,7 +184,7 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   pa.status = h->status;
   // row IDs, gate and the gathered, dequantised rows in one kernel
   ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
-    return ple::launch_embed(pa, h->w.table, h->w.scales, c.row_dim, h->e, h->num_sms, stream);
+    return ple::launch_embed(pa, table_ref(h), c.row_dim, h->e, h->num_sms, stream);
   });
   if (st != PLE_OK) return st;
 
@@ -287,7 +292,7 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   if (config == nullptr || weights == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
   *out = nullptr;
   const ple_config& c = *config;
-  if (c.reserved != 0 || c.vocab <= 0 || c.hidden <= 0 || c.row_dim <= 0 || c.max_tokens <= 0 || c.max_seqs <= 0)
+  if ((c.table_format != PLE_TABLE_E4M3 && c.table_format != PLE_TABLE_NVFP4) || c.vocab <= 0 || c.hidden <= 0 || c.row_dim <= 0 || c.max_tokens <= 0 || c.max_seqs <= 0)
     return PLE_ERR_INVALID_ARG;
   if (c.hidden % 128 != 0 || c.row_dim % 64 != 0) return PLE_ERR_UNSUPPORTED;
   for (int n = 0; n < 2; ++n)
@@ -295,8 +300,10 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   if (weights->table == nullptr || weights->scales == nullptr || weights->w_proj == nullptr ||
       weights->w_gate == nullptr || weights->conv_w == nullptr)
     return PLE_ERR_INVALID_ARG;
+  if (c.table_format == PLE_TABLE_NVFP4 && weights->block_scales == nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned(weights->table, 16) || !aligned(weights->w_proj, 16) || !aligned(weights->w_gate, 16) ||
-      !aligned(weights->conv_w, 16) || !aligned(weights->scales, 4))
+      !aligned(weights->conv_w, 16) || !aligned(weights->scales, 4) ||
+      (c.table_format == PLE_TABLE_NVFP4 && !aligned(weights->block_scales, 16)))
     return PLE_ERR_ALIGN;
 
   ple_handle* h = new (std::nothrow) ple_handle();
@@ -419,7 +426,7 @@ ple_status ple_gather_rows(ple_handle* h, const int32_t* ids, int32_t T, void* e
   if (!aligned(ids, 8) || !aligned(e_out, 16)) return PLE_ERR_ALIGN;
   const ple_config& c = h->cfg;
   return run_stage(h, PLE_STAGE_GATHER, stream, [&] {
-    return ple::launch_gather(ids, T, h->w.table, h->w.scales, c.rows[0], c.rows[1], c.row_dim,
+    return ple::launch_gather(ids, T, table_ref(h), c.rows[0], c.rows[1], c.row_dim,
                               static_cast<__half*>(e_out), true, stream);
   });
 }
@@ -467,7 +474,9 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
     a.magic0 = ple::barrett_magic(c.rows[0]);
     a.magic1 = ple::barrett_magic(c.rows[1]);
     a.table = h->w.table;
+    a.blocks = h->w.block_scales;
     a.scales = h->w.scales;
+    a.nvfp4 = c.table_format == PLE_TABLE_NVFP4 ? 1 : 0;
     a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
     a.conv_w = h->w.conv_w;
     a.hidden = static_cast<const __nv_bfloat16*>(hidden);

@@ -117,6 +117,7 @@ size_t smem_bytes(int units, int32_t D, int32_t H) {
          static_cast<size_t>(kMaxTok) * (D + 8) * sizeof(__half) + static_cast<size_t>(H) * sizeof(__nv_bfloat16);
 }
 
+template <bool NV>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecodeSmallArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();                                          // row IDs ready
   const int row_segs = (T * nsr + kWarps - 1) / kWarps;     // per warp
   for (int first = 0; first < row_segs; first += kRowBatch) {
-    uint4 xa[kRowBatch], xb[kRowBatch];
+    RowChunk<NV> xa[kRowBatch], xb[kRowBatch];
     float sa[kRowBatch], sb[kRowBatch];
 #pragma unroll
     for (int r = 0; r < kRowBatch; ++r) {
@@ -271,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = s / nsr, j = (s - t * nsr) * 32 + lane;
       if (t < T && j < dv16) {
         const int64_t ra = sm->rid[t][0], rb = sm->rid[t][1];
-        xa[r] = __ldg(reinterpret_cast<const uint4*>(a.table + ra * a.D) + j);
-        xb[r] = __ldg(reinterpret_cast<const uint4*>(a.table + rb * a.D) + j);
+        xa[r] = load_chunk<NV>(a.table, a.blocks, ra, a.D, j);
+        xb[r] = load_chunk<NV>(a.table, a.blocks, rb, a.D, j);
         sa[r] = __ldg(a.scales + ra);
         sb[r] = __ldg(a.scales + rb);
       }
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = s / nsr, j = (s - t * nsr) * 32 + lane;
       if (t < T && j < dv16) {
         uint4 lo, hi;
-        deq16(xa[r], xb[r], sa[r], sb[r], lo, hi);
+        deq_chunk<NV>(xa[r], xb[r], sa[r], sb[r], lo, hi);
         uint4* dst = reinterpret_cast<uint4*>(e16 + t * ldE + 16 * j);
         dst[0] = lo;
         dst[1] = hi;
@@ -475,8 +476,10 @@ cudaError_t launch_decode_small(const CUtensorMap& tmap_w, const DecodeSmallArgs
                                 cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(decode_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    cudaError_t e = cudaFuncSetAttribute(decode_small_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemLimit);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_small_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -490,7 +493,8 @@ cudaError_t launch_decode_small(const CUtensorMap& tmap_w, const DecodeSmallArgs
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_small_kernel, tmap_w, a);
+  if (a.nvfp4) return cudaLaunchKernelEx(&cfg, decode_small_kernel<true>, tmap_w, a);
+  return cudaLaunchKernelEx(&cfg, decode_small_kernel<false>, tmap_w, a);
 }
 
 }  // namespace ple

@@ -320,4 +320,92 @@ __device__ __forceinline__ void deq16(const uint4& a, const uint4& b, float s0, 
   o1.w = deq2(a.w, b.w, 16, s0, s1);
 }
 
+// NVFP4 rows: e = fp16(a' * s0 + b' * s1) for 16 elements of two rows, where a'
+// is an FP4 E2M1 code times its block's E4M3 scale. Codes come two per byte,
+// the low nibble first (8 bytes per 16 elements); one block scale covers the
+// 16. The product of an E2M1 value (at most 2 significant bits, magnitude
+// 0.5 .. 6) and an E4M3 value (4 bits, 2^-9 .. 448) has at most 6 significant
+// bits and lies in [2^-10, 2688], so it is exact in fp16. Then fmaf in fp32
+// and RNE to fp16 as for FP8 rows. NaN block scales stay NaN.
+__device__ __forceinline__ __half2 e2m1x2_cvt(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte & 0xFFu));
+  return *reinterpret_cast<const __half2*>(&r);
+}
+
+__device__ __forceinline__ uint32_t deq2_nv(uint32_t wa, uint32_t wb, int shift, __half2 ba, __half2 bb, float s0,
+                                            float s1) {
+  const float2 a = __half22float2(__hmul2(e2m1x2_cvt(wa >> shift), ba));
+  const float2 b = __half22float2(__hmul2(e2m1x2_cvt(wb >> shift), bb));
+  const __half2 r = __floats2half2_rn(fmaf(a.x, s0, b.x * s1), fmaf(a.y, s0, b.y * s1));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// ca, cb: the 8 code bytes of each row (16 elements); bsa, bsb: the block-scale bytes.
+__device__ __forceinline__ void deq16_nv(const uint2& ca, const uint2& cb, uint32_t bsa, uint32_t bsb, float s0,
+                                         float s1, uint4& o0, uint4& o1) {
+  const float2 bs = e4m3x2_cvt((bsa & 0xFFu) | ((bsb & 0xFFu) << 8));
+  const __half2 ba = __float2half2_rn(bs.x);          // exact: an E4M3 value is an fp16 value
+  const __half2 bb = __float2half2_rn(bs.y);
+  o0.x = deq2_nv(ca.x, cb.x, 0, ba, bb, s0, s1);
+  o0.y = deq2_nv(ca.x, cb.x, 8, ba, bb, s0, s1);
+  o0.z = deq2_nv(ca.x, cb.x, 16, ba, bb, s0, s1);
+  o0.w = deq2_nv(ca.x, cb.x, 24, ba, bb, s0, s1);
+  o1.x = deq2_nv(ca.y, cb.y, 0, ba, bb, s0, s1);
+  o1.y = deq2_nv(ca.y, cb.y, 8, ba, bb, s0, s1);
+  o1.z = deq2_nv(ca.y, cb.y, 16, ba, bb, s0, s1);
+  o1.w = deq2_nv(ca.y, cb.y, 24, ba, bb, s0, s1);
+}
+
+// ------------------------------------------------------------------ table row chunks
+// Streaming loads of data read once (no L1 allocation).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u8(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+// One 16-element chunk of a table row: E4M3 codes (16 bytes), or NVFP4 codes
+// (8 bytes) and the chunk's block-scale byte.
+template <bool NV> struct RowChunk;
+template <> struct RowChunk<false> { uint4 c; };
+template <> struct RowChunk<true> { uint2 c; uint32_t b; };
+
+// Chunk j of global row `row` (sub-table offset already added) of a table with
+// row_dim D: codes at row * D (E4M3) or row * D/2 (NVFP4), block scales at row * D/16.
+template <bool NV>
+__device__ __forceinline__ RowChunk<NV> load_chunk(const uint8_t* codes, const uint8_t* blocks, int64_t row,
+                                                   int32_t D, int j) {
+  RowChunk<NV> r;
+  if constexpr (NV) {
+    r.c = ld_stream_v2(codes + row * (D / 2) + 8 * j);
+    r.b = ld_stream_u8(blocks + row * (D / 16) + j);
+  } else {
+    (void)blocks;
+    r.c = ld_stream_v4(codes + row * D + 16 * j);
+  }
+  return r;
+}
+
+template <bool NV>
+__device__ __forceinline__ void deq_chunk(const RowChunk<NV>& a, const RowChunk<NV>& b, float s0, float s1,
+                                          uint4& o0, uint4& o1) {
+  if constexpr (NV) deq16_nv(a.c, b.c, a.b, b.b, s0, s1, o0, o1);
+  else deq16(a.c, b.c, s0, s1, o0, o1);
+}
+
 }  // namespace ple

@@ -13,6 +13,14 @@ namespace ple {
 
 struct TokMeta;
 
+// The table as the kernels see it (ple_table_format in ple.h).
+struct TableRef {
+  const uint8_t* codes;        // E4M3: one byte per element; NVFP4: two E2M1 codes per byte
+  const uint8_t* blocks;       // NVFP4: one E4M3 block scale per 16 elements; else null
+  const float* scales;         // fp32 per row
+  int32_t nvfp4;               // 1: PLE_TABLE_NVFP4
+};
+
 // Prepare stage: sequence map, n-gram row IDs, gate, state snapshot.
 struct PrepareArgs {
   const int32_t* tokens;
@@ -38,13 +46,12 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
 
 // Prepare and gather fused (one pass over HBM): ids, metadata with the gate,
 // and e[t] for the batch. num_sms sizes the persistent grid.
-cudaError_t launch_embed(const PrepareArgs& a, const uint8_t* table, const float* scales, int32_t D, __half* e,
-                         int32_t num_sms, cudaStream_t stream);
+cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
+                         cudaStream_t stream);
 
 // Gather stage: e[t] = deq(row of order 0) + deq(row of order 1), fp16.
-cudaError_t launch_gather(const int32_t* ids, int32_t T, const uint8_t* table, const float* scales,
-                          int64_t rows0, int64_t rows1, int32_t D, __half* e, bool reduce_ids,
-                          cudaStream_t stream);
+cudaError_t launch_gather(const int32_t* ids, int32_t T, const TableRef& table, int64_t rows0, int64_t rows1,
+                          int32_t D, __half* e, bool reduce_ids, cudaStream_t stream);
 
 // W_proj bf16 [D][H] -> fp16 [H][D]; *bad set to 1 when a value is outside the fp16 range.
 cudaError_t launch_convert_w(const __nv_bfloat16* w, int32_t D, int32_t H, __half* w16, int32_t* bad,
@@ -123,7 +130,9 @@ struct DecodeSmallArgs {
   int64_t rows0, rows1;
   uint64_t magic0, magic1; // barrett_magic(rows0), barrett_magic(rows1)
   const uint8_t* table;
+  const uint8_t* blocks;   // NVFP4 block scales (null for E4M3)
   const float* scales;
+  int32_t nvfp4;
   const __nv_bfloat16* w_gate;
   const float* conv_w;
   const __nv_bfloat16* hidden;

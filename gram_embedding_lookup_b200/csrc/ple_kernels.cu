@@ -175,38 +175,29 @@ __global__ void __launch_bounds__(256) prepare_kernel(const PrepareArgs a, int t
 }
 
 // ------------------------------------------------------------------ gather
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ ids, int32_t T,
-                                                     const uint8_t* __restrict__ table,
-                                                     const float* __restrict__ scales, int64_t rows0,
-                                                     int64_t rows1, int32_t D, __half* __restrict__ e,
-                                                     int reduce_ids) {
+template <bool NV>
+__global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ ids, int32_t T, const TableRef t,
+                                                     int64_t rows0, int64_t rows1, int32_t D,
+                                                     __half* __restrict__ e, int reduce_ids) {
   const int chunks = D >> 4;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= static_cast<int64_t>(T) * chunks) return;
-  const int32_t t = static_cast<int32_t>(g / chunks);
-  const int32_t c = static_cast<int32_t>(g - static_cast<int64_t>(t) * chunks);
-  int2 id = ids[t];
+  const int32_t tk = static_cast<int32_t>(g / chunks);
+  const int32_t c = static_cast<int32_t>(g - static_cast<int64_t>(tk) * chunks);
+  int2 id = ids[tk];
   if (reduce_ids) {
     id.x = static_cast<int32_t>(static_cast<uint32_t>(id.x) % static_cast<uint32_t>(rows0));
     id.y = static_cast<int32_t>(static_cast<uint32_t>(id.y) % static_cast<uint32_t>(rows1));
   }
   const int64_t row0 = id.x;
   const int64_t row1 = rows0 + id.y;
-  const uint4 a = ld_stream_v4(table + row0 * D + c * 16);
-  const uint4 b = ld_stream_v4(table + row1 * D + c * 16);
-  const float s0 = __ldg(scales + row0);
-  const float s1 = __ldg(scales + row1);
+  const RowChunk<NV> a = load_chunk<NV>(t.codes, t.blocks, row0, D, c);
+  const RowChunk<NV> b = load_chunk<NV>(t.codes, t.blocks, row1, D, c);
+  const float s0 = __ldg(t.scales + row0);
+  const float s1 = __ldg(t.scales + row1);
   uint4 o0, o1;
-  deq16(a, b, s0, s1, o0, o1);
-  uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D + c * 16);
+  deq_chunk<NV>(a, b, s0, s1, o0, o1);
+  uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(tk) * D + c * 16);
   dst[0] = o0;
   dst[1] = o1;
 }
@@ -244,9 +235,9 @@ struct PipeSmem {
   uint64_t empty[kPipeBatches];                      // consumers -> producer (count kPipeConsumers)
 };
 
+template <bool NV>
 __global__ void __launch_bounds__(kPipeThreads, 1)
-    embed_pipe_kernel(const PrepareArgs a, const uint8_t* __restrict__ table, const float* __restrict__ scales,
-                      int32_t D, __half* __restrict__ e) {
+    embed_pipe_kernel(const PrepareArgs a, const TableRef tab, int32_t D, __half* __restrict__ e) {
   __shared__ PipeSmem sm;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -300,7 +291,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     bool state_done = false;
     for (int b = 0; b < nb; ++b) {
       const int slot = b % kPipeBatches, round = b / kPipeBatches;
-      uint4 hv[kEmbedH4], ca[kEmbedD16], cb[kEmbedD16];
+      uint4 hv[kEmbedH4];
+      RowChunk<NV> ca[kEmbedD16], cb[kEmbedD16];
       auto load_hidden = [&](int t) {
         const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
 #pragma unroll
@@ -327,18 +319,17 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
         if (half > 0) load_hidden(t);
         const PipeTok pt = sm.tok[slot][i];
-        const uint8_t* ra = table + static_cast<int64_t>(pt.r0) * D;
-        const uint8_t* rb = table + (a.rows0 + pt.r1) * D;
+        const int64_t ra = pt.r0, rb = a.rows0 + pt.r1;
 #pragma unroll
         for (int r = 0; r < kEmbedD16; ++r) {
           const int j = lane + 32 * r;
           if (j < D16) {
-            ca[r] = ld_stream_v4(ra + 16 * j);
-            cb[r] = ld_stream_v4(rb + 16 * j);
+            ca[r] = load_chunk<NV>(tab.codes, tab.blocks, ra, D, j);
+            cb[r] = load_chunk<NV>(tab.codes, tab.blocks, rb, D, j);
           }
         }
-        const float s0 = __ldg(scales + pt.r0);
-        const float s1 = __ldg(scales + a.rows0 + pt.r1);
+        const float s0 = __ldg(tab.scales + ra);
+        const float s1 = __ldg(tab.scales + rb);
         // gate: g = sigmoid(w_gate . h_t), fp32
         float acc = 0.f;
         auto dot8 = [&](const uint4& hq, const uint4& wq) {
@@ -370,9 +361,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
         // e_t = deq(bigram row) + deq(trigram row), fp16
         uint4* erow = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D);
-        auto emit = [&](int j, const uint4& x, const uint4& y) {
+        auto emit = [&](int j, const RowChunk<NV>& x, const RowChunk<NV>& y) {
           uint4 o0, o1;
-          deq16(x, y, s0, s1, o0, o1);
+          deq_chunk<NV>(x, y, s0, s1, o0, o1);
           erow[2 * j] = o0;
           erow[2 * j + 1] = o1;
         };
@@ -381,7 +372,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           const int j = lane + 32 * r;
           if (j < D16) emit(j, ca[r], cb[r]);
         }
-        for (int j = lane + 32 * kEmbedD16; j < D16; j += 32) emit(j, ld_stream_v4(ra + 16 * j), ld_stream_v4(rb + 16 * j));
+        for (int j = lane + 32 * kEmbedD16; j < D16; j += 32)
+          emit(j, load_chunk<NV>(tab.codes, tab.blocks, ra, D, j), load_chunk<NV>(tab.codes, tab.blocks, rb, D, j));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.empty[slot]));
@@ -505,22 +497,27 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_embed(const PrepareArgs& a, const uint8_t* table, const float* scales, int32_t D, __half* e,
-                         int32_t num_sms, cudaStream_t stream) {
+cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
+                         cudaStream_t stream) {
   const bool state = a.conv_in != nullptr || a.hist_new != nullptr;
   // small batches spread over the SMs: a few tokens per CTA, no warp taking two in turn
   const int grid = state ? num_sms : std::min<int>(num_sms, a.T);
-  embed_pipe_kernel<<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, scales, D, e);
+  if (table.nvfp4)
+    embed_pipe_kernel<true><<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, D, e);
+  else
+    embed_pipe_kernel<false><<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, D, e);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const int32_t* ids, int32_t T, const uint8_t* table, const float* scales,
-                          int64_t rows0, int64_t rows1, int32_t D, __half* e, bool reduce_ids,
-                          cudaStream_t stream) {
+cudaError_t launch_gather(const int32_t* ids, int32_t T, const TableRef& table, int64_t rows0, int64_t rows1,
+                          int32_t D, __half* e, bool reduce_ids, cudaStream_t stream) {
   const int64_t threads = static_cast<int64_t>(T) * (D / 16);
   const int blocks = static_cast<int>((threads + 255) / 256);
-  gather_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const int2*>(ids), T, table, scales, rows0,
-                                            rows1, D, e, reduce_ids ? 1 : 0);
+  const int2* id2 = reinterpret_cast<const int2*>(ids);
+  if (table.nvfp4)
+    gather_kernel<true><<<blocks, 256, 0, stream>>>(id2, T, table, rows0, rows1, D, e, reduce_ids ? 1 : 0);
+  else
+    gather_kernel<false><<<blocks, 256, 0, stream>>>(id2, T, table, rows0, rows1, D, e, reduce_ids ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -92,8 +92,8 @@ extern "C" ple_status ple_embed_static(const int32_t* tokens, int32_t T, const i
   pa.H = 0;
   pa.status = status;
   if (ple::launch_prepare(pa, stream) != cudaSuccess) return PLE_ERR_CUDA;
-  if (ple::launch_gather(ids, T, table, scales, rows0, rows1, row_dim, static_cast<__half*>(e_out), false,
-                         stream) != cudaSuccess)
+  if (ple::launch_gather(ids, T, ple::TableRef{table, nullptr, scales, 0}, rows0, rows1, row_dim,
+                        static_cast<__half*>(e_out), false, stream) != cudaSuccess)
     return PLE_ERR_CUDA;
   if (status_out != nullptr &&
       cudaMemcpyAsync(status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, stream) != cudaSuccess)

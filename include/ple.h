@@ -21,6 +21,9 @@
  *   rows     row_n = (k_n ^ (k_n >> 32)) mod rows[n]  (unsigned 64-bit)
  *   embed    e_t[k] = E4M3(table[0][row_2][k])*scales[0][row_2]
  *                   + E4M3(table[1][row_3][k])*scales[1][row_3]
+ *            or, for an NVFP4 table (see ple_table_format),
+ *            e_t[k] = E2M1(code[0][row_2][k])*E4M3(block[0][row_2][k/16])*scales[0][row_2]
+ *                   + (the same for order 1 and row_3)
  *   project  v_t = e_t W_proj            (W_proj bf16 [row_dim][hidden])
  *   gate     g_t = sigmoid(w_gate . h_t) (one scalar per token)
  *   conv     y_t[j] = sum_{k=0..3} conv_w[j][k] * u_{t-3+k}[j],  u = g v,
@@ -67,6 +70,18 @@ typedef enum {
 
 typedef enum { PLE_OUT_BF16 = 0, PLE_OUT_F32 = 1 } ple_out_dtype;
 
+/* Table formats.
+ *   PLE_TABLE_E4M3: one FP8 E4M3 ("fn") code per element and one fp32 scale per
+ *     row (51.2 GB at 2 x 10,000,048 rows of 2560).
+ *   PLE_TABLE_NVFP4: the capacity variant of the pages, about 26.82 GiB against
+ *     95.37 GiB in BF16 (deletoe.com page, section "第三条路：把 PLE 也量化，能塞下，
+ *     但不够快"; DGX Spark report, sections "运行时内存占用" and "小结": a packed
+ *     table of NVFP4 codes and FP8 scales). The layout is not on the pages;
+ *     this library reads it as FP4 E2M1 codes, two per byte with the low
+ *     nibble first, one E4M3 block scale per 16 elements, and the same fp32
+ *     scale per row as the E4M3 table. */
+typedef enum { PLE_TABLE_E4M3 = 0, PLE_TABLE_NVFP4 = 1 } ple_table_format;
+
 /* Sizes fixed at creation. hidden % 128 == 0, row_dim % 64 == 0,
  * 0 < rows[n] < 2^31. max_tokens bounds T of every call (and B*q of a decode
  * step); max_seqs bounds S (and B). */
@@ -76,20 +91,26 @@ typedef struct {
   int32_t row_dim;
   int32_t max_tokens;
   int32_t max_seqs;
-  int32_t reserved;          /* must be 0 */
+  int32_t table_format;      /* ple_table_format */
   int64_t rows[2];           /* rows of the bigram (0) and trigram (1) sub-tables */
 } ple_config;
 
 /* Parameters. All are BORROWED: they must stay valid and unchanged for the
  * handle's lifetime, except w_proj, which is read once by ple_create. */
 typedef struct {
-  const uint8_t* table;      /* FP8-E4M3 codes; sub-table n, row r at byte offset
-                                (n*rows[0] + r)*row_dim  (so [2][rows][row_dim]
-                                when rows[0] == rows[1]); 16-byte aligned */
+  const uint8_t* table;      /* E4M3: one code per element; sub-table n, row r at byte
+                                offset (n*rows[0] + r)*row_dim ([2][rows][row_dim] when
+                                rows[0] == rows[1]).
+                                NVFP4: packed E2M1 codes, element 2i in the low nibble of
+                                byte i of the row; row r of sub-table n at byte offset
+                                (n*rows[0] + r)*row_dim/2. 16-byte aligned */
   const float* scales;       /* fp32 per-row scales; sub-table n, row r at n*rows[0] + r */
   const void* w_proj;        /* bf16 [row_dim][hidden], row-major */
   const void* w_gate;        /* bf16 [hidden] */
   const float* conv_w;       /* fp32 [hidden][4]; tap 3 multiplies the current token */
+  const uint8_t* block_scales; /* NVFP4 only (NULL for E4M3): E4M3 scale of elements
+                                [16j, 16j+16) of row r of sub-table n at byte offset
+                                (n*rows[0] + r)*row_dim/16 + j; 16-byte aligned */
 } ple_weights;
 
 /* Per-sequence carried state (caller-owned, device memory). */
@@ -119,8 +140,9 @@ ple_status ple_ngram_ids(ple_handle* handle, const int32_t* tokens, int32_t T,
                          int32_t* ids, cudaStream_t stream);
 
 /* The gather stage alone: e_out fp16 [T][row_dim] receives e_t (see top of
- * file) for the given row IDs int32 [T][2]. IDs must be in range (the call
- * reduces them mod rows[n] so that no access leaves the table). */
+ * file, in the handle's table format) for the given row IDs int32 [T][2]. IDs
+ * must be in range (the call reduces them mod rows[n] so that no access
+ * leaves the table). */
 ple_status ple_gather_rows(ple_handle* handle, const int32_t* ids, int32_t T,
                            void* e_out, cudaStream_t stream);
 
@@ -156,7 +178,8 @@ ple_status ple_decode_step(ple_handle* handle, const int32_t* tokens, int32_t B,
  * create a handle either, since ple_create allocates.
  *
  * ple_embed_static computes the n-gram row IDs of a packed batch (as
- * ple_ngram_ids) and gathers and dequantises the rows into e_out fp16
+ * ple_ngram_ids) and gathers and dequantises the rows of an E4M3 table
+ * (PLE_TABLE_E4M3 layout) into e_out fp16
  * [T][row_dim] (as ple_gather_rows). It allocates nothing: the row IDs live in
  * a fixed array inside the library image, PLE_STATIC_MAX_TOKENS x 2 int32
  * (128 KiB), which every GPU that loads the library holds until the process

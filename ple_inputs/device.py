@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 import gram_embedding_lookup_b200 as ple
-from . import Workload, fill_table_device
+from . import Workload, fill_nv_table_device, fill_table_device
 
 
 def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
@@ -25,27 +25,40 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
 
 
 class DeviceLayer:
-    """A workload's table and weights on the current device, plus a libple handle."""
+    """A workload's table and weights on the current device, plus a libple handle.
 
-    def __init__(self, w: Workload, max_tokens: int, max_seqs: int, weights=None, stream=None):
+    table_format ple.PLE_TABLE_NVFP4 builds the synthetic NVFP4 table instead
+    (packed codes in ``table``, E4M3 block scales in ``block_scales``)."""
+
+    def __init__(self, w: Workload, max_tokens: int, max_seqs: int, weights=None, stream=None,
+                 table_format: int = 0):
         self.w = w
+        self.table_format = table_format
         R, D, H = w.rows_per_order, w.row_dim, w.hidden
-        self.table = torch.empty(2 * R * D, dtype=torch.uint8, device="cuda")
-        self.scales = torch.empty(2 * R, dtype=torch.float32, device="cuda")
         s = torch.cuda.current_stream() if stream is None else stream
-        fill_table_device(self.table.data_ptr(), self.scales.data_ptr(), R, D, w.table_seed, s.cuda_stream)
+        self.scales = torch.empty(2 * R, dtype=torch.float32, device="cuda")
+        if table_format == ple.PLE_TABLE_NVFP4:
+            self.table = torch.empty(2 * R * D // 2, dtype=torch.uint8, device="cuda")
+            self.block_scales = torch.empty(2 * R * D // 16, dtype=torch.uint8, device="cuda")
+            fill_nv_table_device(self.table.data_ptr(), self.block_scales.data_ptr(), self.scales.data_ptr(), R, D,
+                                 w.table_seed, s.cuda_stream)
+        else:
+            self.table = torch.empty(2 * R * D, dtype=torch.uint8, device="cuda")
+            self.block_scales = None
+            fill_table_device(self.table.data_ptr(), self.scales.data_ptr(), R, D, w.table_seed, s.cuda_stream)
         self.host_weights = weights if weights is not None else w.weights()
         self.w_proj = bf16_tensor(self.host_weights.w_proj)
         self.w_gate = bf16_tensor(self.host_weights.w_gate)
         self.conv_w = torch.from_numpy(np.ascontiguousarray(self.host_weights.conv_w, np.float32)).cuda()
         cfg = ple.PleConfig()
         cfg.vocab, cfg.hidden, cfg.row_dim = w.vocab, H, D
-        cfg.max_tokens, cfg.max_seqs, cfg.reserved = max_tokens, max_seqs, 0
+        cfg.max_tokens, cfg.max_seqs, cfg.table_format = max_tokens, max_seqs, table_format
         cfg.rows[0] = R
         cfg.rows[1] = R
         self.config = cfg
         pw = ple.PleWeights(self.table.data_ptr(), self.scales.data_ptr(), self.w_proj.data_ptr(),
-                            self.w_gate.data_ptr(), self.conv_w.data_ptr())
+                            self.w_gate.data_ptr(), self.conv_w.data_ptr(),
+                            self.block_scales.data_ptr() if self.block_scales is not None else None)
         self.weights = pw
         self.handle = ple.ple_create(cfg, pw, s.cuda_stream)
 

@@ -72,6 +72,13 @@ def test_null_arguments_rejected_on_host(libple):
     cfg.rows[0] = cfg.rows[1] = 16
     wts.table = 17
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 3  # misaligned
+    wts.table = 16
+    cfg.table_format = 2                          # no such format
+    assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
+    cfg.table_format = ple.PLE_TABLE_NVFP4        # NVFP4 needs block scales
+    assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
+    wts.block_scales = 24                         # ... 16-byte aligned
+    assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 3
     assert libple.ple_destroy(None) == 1
     assert libple.ple_forward(None, None, 0, None, 1, None, None, 0, None, None) == 1
     assert libple.ple_decode_step(None, None, 1, 1, None, None, 0, None, None, None, None) == 1
