@@ -364,6 +364,7 @@ def main():
         line["decode"] = decode_bench(ctx, layer, stream)
         line["mtp"] = mtp_bench(ctx, layer, stream)
         line["long_context"] = long_bench(ctx, layer, stream)
+        line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks)
 
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         tokens, offsets, hidden = sets[0]["host"]
@@ -471,6 +472,68 @@ def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
     d2h = s0["out"].numel() * 2
     return {"value": s0["T"] * world * steps / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps}
+
+
+def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
+    """The NVFP4 table variant (PLE_TABLE_NVFP4): the same prefill batches and the
+    decode workload on a table of packed E2M1 codes with E4M3 block scales per 16
+    elements (28.8 GB at full scale instead of 51.2 GB)."""
+    torch, ple, pi = ctx["torch"], ctx["ple"], ctx["pi"]
+    from ple_inputs.device import DeviceLayer
+    R, D, H = w.rows_per_order, w.row_dim, w.hidden
+    need = 2 * R * (D // 2 + D // 16) + 2 * R * 4
+    free, _ = torch.cuda.mem_get_info()
+    if free < need + (4 << 30):
+        return {"skipped": f"needs {need / 1e9:.1f} GB free for the NVFP4 table, {free / 1e9:.1f} GB free"}
+    layer = DeviceLayer(w, max_tokens=16384, max_seqs=64, table_format=ple.PLE_TABLE_NVFP4)
+    h = layer.handle
+
+    def step(i):
+        s = sets[i % len(sets)]
+        ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
+                        None, stream)
+
+    for i in range(5):
+        step(i)
+    ple.ple_set_profiling(h, True)
+    ple.ple_get_stage_times(h)
+    ms = timed(ctx, stream, step, steps)
+    stage = ple.ple_get_stage_times(h)
+    ple.ple_set_profiling(h, False)
+    T = sets[0]["T"]
+    e_ms, e_n = stage["prepare"]
+    e_s = e_ms / 1e3 / max(e_n, 1)
+    row_bytes = 2 * (D // 2 + D // 16) + 8                  # both rows' codes and block scales, row scales
+    embed_bytes = T * (2 * H + row_bytes + 2 * D + 8 + 16 + 4)
+    g_ms, g_n = stage["gemm"]
+
+    wd = pi.workload("decode")
+    tokens, hidden, hist, conv = pi.decode_batch(wd)
+    B, q = tokens.shape
+    tk = torch.from_numpy(tokens).cuda()
+    hd = ctx["bf16_tensor"](hidden)
+    hs = torch.from_numpy(hist.astype(np.int32)).cuda()
+    cs = torch.from_numpy(conv).cuda()
+    out = torch.empty(B * q, H, dtype=torch.bfloat16, device="cuda")
+
+    def dstep(i):
+        ple.ple_decode_step(h, tk, B, q, hd, out, ple.PLE_OUT_BF16, hs, cs, None, stream)
+
+    for i in range(5):
+        dstep(i)
+    n_dec = 500
+    d_ms = timed(ctx, stream, dstep, n_dec)
+    status = ple.ple_get_error(h)
+    layer.close()
+    world = ctx["world"]
+    return {"workload": "full-scale prefill (the headline batches) and 8 x 1 decode on the NVFP4 table",
+            "table_bytes": int(need), "value": T * world * steps / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms / steps, "stage_ms_per_launch": {"embed": e_s * 1e3, "gemm": g_ms / max(g_n, 1)},
+            "embed_roofline": {"bound": "hbm", "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"],
+                               "algorithmic_bytes_per_launch": embed_bytes},
+            "gathered_row_gbs": T * row_bytes / e_s / 1e9,
+            "decode_us_per_step": 1e3 * d_ms / n_dec, "device_status": int(status)}
 
 
 def decode_bench(ctx, layer, stream):
