@@ -14,7 +14,8 @@ import os
 
 __all__ = [
     "PleError", "PleConfig", "PleWeights", "PleState", "lib", "ple_create", "ple_destroy",
-    "ple_ngram_ids", "ple_gather_rows", "ple_forward", "ple_decode_step", "ple_get_error",
+    "ple_ngram_ids", "ple_gather_rows", "ple_forward", "ple_prepare", "ple_forward_prepared", "ple_decode_step",
+    "ple_get_error",
     "ple_status_string", "ple_set_profiling", "ple_get_stage_times", "ple_set_forward_path",
     "ple_launch_count", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32",
     "PLE_TABLE_E4M3", "PLE_TABLE_NVFP4", "STATUS",
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
             "ple_gather_rows": ([_VP, _VP, _I32, _VP, _VP], _I32),
             "ple_forward": ([_VP, _VP, _I32, _VP, _I32, _VP, _VP, _I32, ctypes.POINTER(PleState), _VP], _I32),
             "ple_decode_step": ([_VP, _VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP, _VP, _VP], _I32),
+            "ple_prepare": ([_VP, _VP, _I32, _VP, _I32, _VP, _VP], _I32),
+            "ple_forward_prepared": ([_VP, _VP, _VP, _I32, ctypes.POINTER(PleState), _VP], _I32),
             "ple_get_error": ([_VP], _I32),
             "ple_status_string": ([_I32], ctypes.c_char_p),
             "ple_set_profiling": ([_VP, _I32], _I32),
@@ -150,6 +153,19 @@ def ple_forward(handle, tokens, T, offsets, S, hidden, out, out_dtype, state=Non
         st = ctypes.byref(PleState(_ptr(hist), _ptr(conv)))
     _check(lib().ple_forward(handle, _ptr(tokens), T, _ptr(offsets), S, _ptr(hidden), _ptr(out), out_dtype, st,
                              _stream(stream)), "ple_forward")
+
+
+def ple_prepare(handle, tokens, T, offsets, S, hist=None, stream=None) -> None:
+    _check(lib().ple_prepare(handle, _ptr(tokens), T, _ptr(offsets), S, _ptr(hist), _stream(stream)), "ple_prepare")
+
+
+def ple_forward_prepared(handle, hidden, out, out_dtype, state=None, stream=None) -> None:
+    st = None
+    if state is not None:
+        hist, conv = state
+        st = ctypes.byref(PleState(_ptr(hist), _ptr(conv)))
+    _check(lib().ple_forward_prepared(handle, _ptr(hidden), _ptr(out), out_dtype, st, _stream(stream)),
+           "ple_forward_prepared")
 
 
 def ple_decode_step(handle, tokens, B, q, hidden, out, out_dtype, hist, conv_state, n_commit=None,

@@ -57,6 +57,11 @@ struct ple_handle {
   CUtensorMap tmap_w{};
   CUtensorMap tmap_wd{};         // fp16 W_proj, 64 x 16 boxes for the decode kernel
   int32_t forward_path = 0;
+  struct Prepared {        // the batch ple_prepare left in the scratch (ids, e, meta, hist_new)
+    bool valid = false;
+    int32_t T = 0, S = 0;
+    bool with_hist = false;
+  } prepared;
   bool profiling = false;
   struct Rec { int stage; cudaEvent_t a, b; };
   std::vector<Rec> pending;
@@ -152,6 +157,10 @@ void free_all(ple_handle* h) {
   for (auto e : h->free_events) cudaEventDestroy(e);
 }
 
+ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q, const void* hidden, void* out,
+                          ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist, float* dec_conv,
+                          const int32_t* tokens, const int32_t* n_commit, cudaStream_t stream);
+
 // Runs prepare + gather + projection (+ combine) for a packed batch.
 ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
                      int32_t uniform_q, const void* hidden, void* out, ple_out_dtype dtype,
@@ -159,7 +168,6 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
                      cudaStream_t stream) {
   const ple_config& c = h->cfg;
   const bool decode = uniform_q > 0;
-  const Plan pl = plan_projection(h, T, decode ? 2 : h->forward_path, h->partial_elems);
 
   ple::PrepareArgs pa{};
   pa.tokens = tokens;
@@ -183,11 +191,24 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   }
   pa.status = h->status;
   // row IDs, gate and the gathered, dequantised rows in one kernel
-  ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
+  h->prepared.valid = false;            // the scratch now holds this call's batch
+  const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
     return ple::launch_embed(pa, table_ref(h), c.row_dim, h->e, h->num_sms, stream);
   });
   if (st != PLE_OK) return st;
+  return run_projection(h, T, S, uniform_q, hidden, out, dtype, state, dec_hist, dec_conv, tokens, n_commit, stream);
+}
 
+// The projection and everything after it, on the rows, IDs and metadata in the
+// handle's scratch (written by the embed kernel, or by ple_prepare plus the gate
+// kernel).
+ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q, const void* hidden, void* out,
+                          ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist, float* dec_conv,
+                          const int32_t* tokens, const int32_t* n_commit, cudaStream_t stream) {
+  const ple_config& c = h->cfg;
+  const bool decode = uniform_q > 0;
+  const Plan pl = plan_projection(h, T, decode ? 2 : h->forward_path, h->partial_elems);
+  ple_status st = PLE_OK;
   CUtensorMap tmap_e{}, tmap_h{}, tmap_o{}, tmap_o_head{};
   if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->e, c.row_dim, T, static_cast<uint64_t>(c.row_dim) * 2,
                  kTileK, pl.n_tok / pl.ctas, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -447,6 +468,72 @@ ple_status ple_forward(ple_handle* h, const int32_t* tokens, int32_t T, const in
   return run_layer(h, tokens, T, offsets, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, stream);
 }
 
+ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
+                       const int32_t* hist, cudaStream_t stream) {
+  if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
+  h->prepared.valid = false;
+  if (T > 0) {
+    if (tokens == nullptr || offsets == nullptr) return PLE_ERR_INVALID_ARG;
+    if (!aligned(tokens, 4) || !aligned(offsets, 4) || (hist && !aligned(hist, 4))) return PLE_ERR_ALIGN;
+    const ple_config& c = h->cfg;
+    ple::PrepareArgs pa{};
+    pa.tokens = tokens;
+    pa.T = T;
+    pa.offsets = offsets;
+    pa.S = S;
+    pa.hist = hist;
+    pa.vocab = c.vocab;
+    pa.rows0 = c.rows[0];
+    pa.rows1 = c.rows[1];
+    pa.ids = h->ids;
+    pa.hidden = nullptr;                 // the gate waits for ple_forward_prepared
+    pa.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
+    pa.H = c.hidden;
+    pa.meta = h->meta;
+    pa.hist_new = h->hist_new;
+    pa.status = h->status;
+    const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
+      return ple::launch_embed(pa, table_ref(h), c.row_dim, h->e, h->num_sms, stream);
+    });
+    if (st != PLE_OK) return st;
+  }
+  h->prepared.valid = true;
+  h->prepared.T = T;
+  h->prepared.S = S;
+  h->prepared.with_hist = hist != nullptr;
+  return PLE_OK;
+}
+
+ple_status ple_forward_prepared(ple_handle* h, const void* hidden, void* out, ple_out_dtype out_dtype,
+                                const ple_state* state, cudaStream_t stream) {
+  if (h == nullptr || !h->prepared.valid) return PLE_ERR_INVALID_ARG;
+  if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
+  if ((state != nullptr) != h->prepared.with_hist) return PLE_ERR_INVALID_ARG;
+  const int32_t T = h->prepared.T, S = h->prepared.S;
+  if (T == 0) return PLE_OK;
+  if (hidden == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
+  if (out == hidden && out_dtype != PLE_OUT_BF16) return PLE_ERR_INVALID_ARG;
+  if (state != nullptr && (state->hist == nullptr || state->conv == nullptr)) return PLE_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(out, 16) || (state && (!aligned(state->hist, 4) || !aligned(state->conv, 16))))
+    return PLE_ERR_ALIGN;
+  const ple_config& c = h->cfg;
+  ple::PrepareArgs ga{};
+  ga.T = T;
+  ga.S = S;
+  ga.hidden = static_cast<const __nv_bfloat16*>(hidden);
+  ga.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
+  ga.H = c.hidden;
+  ga.meta = h->meta;
+  if (state != nullptr) {
+    ga.conv_in = state->conv;
+    ga.conv_copy = h->conv0;
+  }
+  const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_gate(ga, stream); });
+  if (st != PLE_OK) return st;
+  return run_projection(h, T, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, nullptr, stream);
+}
+
 ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const void* hidden, void* out,
                            ple_out_dtype out_dtype, int32_t* hist, float* conv_state, const int32_t* n_commit,
                            cudaStream_t stream) {
@@ -460,6 +547,7 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
       !aligned(conv_state, 16) || (n_commit && !aligned(n_commit, 4)))
     return PLE_ERR_ALIGN;
   const ple_config& c = h->cfg;
+  h->prepared.valid = false;
   if (h->forward_path != 2 && h->decode_small && out != hidden && ple::decode_small_supported(B, q)) {
     ple::DecodeSmallArgs a{};
     a.tokens = tokens;

@@ -49,6 +49,10 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
 cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
                          cudaStream_t stream);
 
+// Gate of a prepared batch: meta[t].g from hidden (one warp per token), plus the
+// conv-state snapshot when conv_in is set.
+cudaError_t launch_gate(const PrepareArgs& a, cudaStream_t stream);
+
 // Gather stage: e[t] = deq(row of order 0) + deq(row of order 1), fp16.
 cudaError_t launch_gather(const int32_t* ids, int32_t T, const TableRef& table, int64_t rows0, int64_t rows1,
                           int32_t D, __half* e, bool reduce_ids, cudaStream_t stream);

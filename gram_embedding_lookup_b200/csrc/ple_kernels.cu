@@ -206,6 +206,70 @@ __global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ id
 constexpr int kEmbedH4 = 10;    // uint4 of h per lane held in registers (hidden <= 2560)
 constexpr int kEmbedD16 = 5;    // 16-code chunks per lane and row held in registers (rows <= 2560 codes)
 
+// g = sigmoid(w_gate . h_t) for one token, by one warp, in fp32: lane l adds
+// up the 8-element groups j = l, l + 32, l + 64, ... in that order (the first
+// kEmbedH4 of them already loaded into hv), then a butterfly reduction across
+// the lanes. The embed and gate kernels both compute the gate through this
+// function, so ple_forward and ple_prepare + ple_forward_prepared agree bit
+// for bit.
+__device__ __forceinline__ float gate_warp(const uint4 (&hv)[kEmbedH4], const uint4* hrow, const uint4* wg, int H8,
+                                           int lane) {
+  float acc = 0.f;
+  auto dot8 = [&](const uint4& hq, const uint4& wq) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
+    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 hf = __bfloat1622float2(h2[q]);
+      const float2 wf = __bfloat1622float2(w2[q]);
+      acc = fmaf(hf.x, wf.x, acc);
+      acc = fmaf(hf.y, wf.y, acc);
+    }
+  };
+#pragma unroll
+  for (int r = 0; r < kEmbedH4; ++r) {
+    const int j = lane + 32 * r;
+    if (j < H8) dot8(hv[r], __ldg(wg + j));
+  }
+  for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) dot8(ld_stream_v4(hrow + j), __ldg(wg + j));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return 1.0f / (1.0f + expf(-acc));
+}
+
+// ------------------------------------------------------------------ gate (after ple_prepare)
+// The gate of a batch whose IDs, rows and metadata ple_prepare left in the
+// scratch: one warp per token writes meta[t].g. Blocks past token_blocks take
+// the snapshot of the carried conv state, as the embed kernel's state work does.
+__global__ void __launch_bounds__(256) gate_kernel(const PrepareArgs a, int token_blocks) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (static_cast<int>(blockIdx.x) >= token_blocks) {
+    if (a.conv_in != nullptr) {
+      const int64_t n4 = static_cast<int64_t>(a.S) * 3 * a.H / 4;
+      const float4* src = reinterpret_cast<const float4*>(a.conv_in);
+      float4* dst = reinterpret_cast<float4*>(a.conv_copy);
+      const int sb = blockIdx.x - token_blocks, nsb = gridDim.x - token_blocks;
+      for (int64_t i = static_cast<int64_t>(sb) * blockDim.x + threadIdx.x; i < n4;
+           i += static_cast<int64_t>(nsb) * blockDim.x)
+        dst[i] = src[i];
+    }
+    return;
+  }
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= a.T) return;
+  const int H8 = a.H / 8;
+  const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+  uint4 hv[kEmbedH4];
+#pragma unroll
+  for (int r = 0; r < kEmbedH4; ++r) {
+    const int j = lane + 32 * r;
+    if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+  }
+  const float g = gate_warp(hv, hrow, reinterpret_cast<const uint4*>(a.w_gate), H8, lane);
+  if (lane == 0) a.meta[t].g = g;
+}
+
 // ------------------------------------------------------------------ embed, pipelined
 // n-gram row IDs, the gate dot product over h_t, and the row gather with E4M3
 // dequantisation into fp16 e_t, in one pass over HBM. One persistent CTA per
@@ -301,7 +365,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           if (j < H8) hv[r] = ld_stream_v4(hrow + j);
         }
       };
-      if (b * kPipeBatch + cw < n) load_hidden(t0 + b * kPipeBatch + cw);
+      const bool with_gate = a.hidden != nullptr;     // null: ple_prepare, the gate comes later
+      if (with_gate && b * kPipeBatch + cw < n) load_hidden(t0 + b * kPipeBatch + cw);
       if (!state_done) {
         state_blocks(a, blockIdx.x, gridDim.x, threadIdx.x - 32, blockDim.x - 32);
         state_done = true;
@@ -317,7 +382,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         if (k >= n) break;                                   // warp-uniform
         const int t = t0 + k;
         const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
-        if (half > 0) load_hidden(t);
+        if (with_gate && half > 0) load_hidden(t);
         const PipeTok pt = sm.tok[slot][i];
         const int64_t ra = pt.r0, rb = a.rows0 + pt.r1;
 #pragma unroll
@@ -330,30 +395,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
         const float s0 = __ldg(tab.scales + ra);
         const float s1 = __ldg(tab.scales + rb);
-        // gate: g = sigmoid(w_gate . h_t), fp32
-        float acc = 0.f;
-        auto dot8 = [&](const uint4& hq, const uint4& wq) {
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
-          const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 hf = __bfloat1622float2(h2[q]);
-            const float2 wf = __bfloat1622float2(w2[q]);
-            acc = fmaf(hf.x, wf.x, acc);
-            acc = fmaf(hf.y, wf.y, acc);
-          }
-        };
-#pragma unroll
-        for (int r = 0; r < kEmbedH4; ++r) {
-          const int j = lane + 32 * r;
-          if (j < H8) dot8(hv[r], __ldg(wg + j));
-        }
-        for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) dot8(ld_stream_v4(hrow + j), __ldg(wg + j));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        const float g = with_gate ? gate_warp(hv, hrow, wg, H8, lane) : 0.f;
         if (lane == 0) {
           TokMeta m;
-          m.g = 1.0f / (1.0f + expf(-acc));
+          m.g = g;
           m.seq = pt.seq;
           m.pos = pt.pos;
           m.flags = pt.flags;
@@ -506,6 +551,17 @@ cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D,
     embed_pipe_kernel<true><<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, D, e);
   else
     embed_pipe_kernel<false><<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, D, e);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate(const PrepareArgs& a, cudaStream_t stream) {
+  const int token_blocks = (a.T + 7) / 8;
+  int state_blocks = 0;
+  if (a.conv_in != nullptr) {
+    const int64_t want = (static_cast<int64_t>(a.S) * 3 * a.H / 4 + 255) / 256;
+    state_blocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
+  }
+  gate_kernel<<<token_blocks + state_blocks, 256, 0, stream>>>(a, token_blocks);
   return cudaGetLastError();
 }
 

@@ -157,6 +157,33 @@ ple_status ple_forward(ple_handle* handle, const int32_t* tokens, int32_t T,
                        const int32_t* offsets, int32_t S, const void* hidden, void* out,
                        ple_out_dtype out_dtype, const ple_state* state, cudaStream_t stream);
 
+/* The layer in two calls, for callers that know the tokens before the hidden
+ * states: the n-gram IDs and the row lookup need no hidden state (DGX Spark
+ * report, section "n-gram embedding 是一条附加的条件记忆路径"), so
+ * ple_prepare can run on a side stream while earlier layers compute hidden,
+ * and ple_forward_prepared then does the rest: the gate, the projection, the
+ * conv, the residual and the state.
+ *
+ * ple_prepare takes the arguments of ple_forward that do not depend on hidden
+ * (hist = the state's hist, or NULL for fresh sequences) and leaves the row
+ * IDs, the dequantised rows and the per-token metadata in the handle's
+ * scratch. ple_forward_prepared takes hidden, out, out_dtype and state as in
+ * ple_forward, for the batch last prepared on the handle. The result equals
+ * ple_forward's bit for bit.
+ *   - state must be non-NULL exactly when ple_prepare got a hist, and
+ *     state->hist must hold the values ple_prepare read; otherwise
+ *     PLE_ERR_INVALID_ARG.
+ *   - ple_forward_prepared without a prepared batch returns
+ *     PLE_ERR_INVALID_ARG. ple_forward and ple_decode_step reuse the scratch
+ *     and discard the prepared batch. A prepared batch stays usable for
+ *     further ple_forward_prepared calls (other hidden states) until then.
+ *   - The two calls may use different streams; ordering them (an event) is
+ *     the caller's job. */
+ple_status ple_prepare(ple_handle* handle, const int32_t* tokens, int32_t T,
+                       const int32_t* offsets, int32_t S, const int32_t* hist, cudaStream_t stream);
+ple_status ple_forward_prepared(ple_handle* handle, const void* hidden, void* out,
+                                ple_out_dtype out_dtype, const ple_state* state, cudaStream_t stream);
+
 /* One decode / speculative-verify step: B sequences with q new tokens each.
  * tokens int32 [B][q]; hidden bf16 [B*q][hidden]; out [B*q][hidden];
  * hist int32 [B][2] and conv_state fp32 [B][3][hidden] are read and updated.
@@ -211,7 +238,8 @@ const char* ple_status_string(ple_status status);
 
 /* Kernel stages of the library, in launch order within a call. In
  * ple_forward and ple_decode_step the PREPARE stage also gathers and
- * dequantises the rows (one fused kernel); GATHER counts ple_gather_rows. */
+ * dequantises the rows (one fused kernel); ple_prepare and the gate kernel of
+ * ple_forward_prepared count as PREPARE too. GATHER counts ple_gather_rows. */
 enum { PLE_STAGE_PREPARE = 0, PLE_STAGE_GATHER = 1, PLE_STAGE_GEMM = 2, PLE_STAGE_COMBINE = 3,
        PLE_NUM_STAGES = 4 };
 

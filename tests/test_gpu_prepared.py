@@ -1,0 +1,163 @@
+"""ple_prepare + ple_forward_prepared against ple_forward, through the C ABI.
+
+The two-call form computes the same layer with the gate moved to a kernel of
+its own; the tests require the outputs and the state to equal ple_forward's
+bit for bit, on every projection path, across two streams, and check the
+host-side errors for a missing or mismatched prepared batch.
+"""
+import numpy as np
+import pytest
+
+import ple_inputs as pi
+
+torch = pytest.importorskip("torch")
+ple = pytest.importorskip("gram_embedding_lookup_b200")
+
+from tests.gpu_common import MID, full_layer, mid_layer, tiny_layer  # noqa: E402,F401
+from tests.test_gpu_parity import dev_bf16, dev_i32, gpu_forward, to_bits  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+def _prepared(L, tokens, offsets, hidden_bits, out_dtype=1, state=None, path=0, stream=None):
+    ple.ple_set_forward_path(L.handle, path)
+    T, S, H = len(tokens), len(offsets) - 1, L.w.hidden
+    hid = dev_bf16(hidden_bits)
+    out = torch.empty(T, H, dtype=torch.float32 if out_dtype == 1 else torch.bfloat16, device="cuda")
+    st = None
+    if state is not None:
+        st = (dev_i32(state[0]), torch.from_numpy(np.ascontiguousarray(state[1], np.float32)).cuda())
+    tk, of = dev_i32(tokens), dev_i32(offsets)
+    torch.cuda.synchronize()
+    if stream is None:
+        ple.ple_prepare(L.handle, tk, T, of, S, None if st is None else st[0])
+        ple.ple_forward_prepared(L.handle, hid, out, out_dtype, st)
+    else:
+        side, main = stream
+        with torch.cuda.stream(side):
+            ple.ple_prepare(L.handle, tk, T, of, S, None if st is None else st[0], side)
+            ev = torch.cuda.Event()
+            ev.record(side)
+        main.wait_event(ev)
+        with torch.cuda.stream(main):
+            ple.ple_forward_prepared(L.handle, hid, out, out_dtype, st, main)
+    torch.cuda.synchronize()
+    ple.ple_set_forward_path(L.handle, 0)
+    assert ple.ple_get_error(L.handle) == 0
+    res = out.cpu().numpy() if out_dtype == 1 else to_bits(out)
+    return res, None if st is None else (st[0].cpu().numpy(), st[1].cpu().numpy())
+
+
+def _f32bits(x):
+    """fp32 bit patterns of an fp32-valued array (float64 copies convert back exactly)."""
+    return np.asarray(x, np.float32).view(np.uint32)
+
+
+def _state(rng, S, H, vocab):
+    return rng.integers(-1, vocab, (S, 2)).astype(np.int32), rng.standard_normal((S, 3, H)).astype(np.float32)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_prepared_equals_forward_tiny(tiny_layer, path, with_state):
+    w = tiny_layer.w
+    rng = np.random.default_rng(path + 10 * with_state)
+    lengths = [300, 1, 2, 700]
+    T = sum(lengths)
+    toks = rng.integers(0, w.vocab, T).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    hid = pi.hidden_bf16(rng, T, w.hidden)
+    state = _state(rng, len(lengths), w.hidden, w.vocab) if with_state else None
+    for dt in (1, 0):
+        ref, ref_st = gpu_forward(tiny_layer, toks, offs, hid, dt, state=state, path=path)
+        got, got_st = _prepared(tiny_layer, toks, offs, hid, dt, state=state, path=path)
+        assert np.array_equal(_f32bits(got), _f32bits(ref)) if dt == 1 else np.array_equal(got, ref)
+        if with_state:
+            assert np.array_equal(got_st[0], ref_st[0])
+            assert np.array_equal(_f32bits(got_st[1]), _f32bits(ref_st[1]))
+
+
+@pytest.mark.parametrize("path", [1, 3, 2])
+def test_prepared_equals_forward_mid_with_state(mid_layer, path):
+    rng = np.random.default_rng(70 + path)
+    lengths = [1000, 3, 600, 253]
+    T = sum(lengths)
+    toks = rng.integers(0, MID.vocab, T).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    hid = pi.hidden_bf16(rng, T, MID.hidden)
+    state = _state(rng, len(lengths), MID.hidden, MID.vocab)
+    ref, ref_st = gpu_forward(mid_layer, toks, offs, hid, 1, state=state, path=path)
+    got, got_st = _prepared(mid_layer, toks, offs, hid, 1, state=state, path=path)
+    assert np.array_equal(_f32bits(got), _f32bits(ref))
+    assert np.array_equal(got_st[0], ref_st[0])
+    assert np.array_equal(_f32bits(got_st[1]), _f32bits(ref_st[1]))
+
+
+def test_prepared_on_a_side_stream(tiny_layer):
+    w = tiny_layer.w
+    toks, offs, hid = pi.tiny_batch(w)
+    ref, _ = gpu_forward(tiny_layer, toks, offs, hid, 1)
+    side, main = torch.cuda.Stream(), torch.cuda.Stream()
+    got, _ = _prepared(tiny_layer, toks, offs, hid, 1, stream=(side, main))
+    assert np.array_equal(_f32bits(got), _f32bits(ref))
+
+
+def test_prepared_batch_reused_with_other_hidden(tiny_layer):
+    w = tiny_layer.w
+    rng = np.random.default_rng(3)
+    toks = rng.integers(0, w.vocab, 500).astype(np.int32)
+    offs = np.array([0, 500], np.int32)
+    h1, h2 = pi.hidden_bf16(rng, 500, w.hidden), pi.hidden_bf16(rng, 500, w.hidden)
+    ref2, _ = gpu_forward(tiny_layer, toks, offs, h2, 1)
+    ple.ple_prepare(tiny_layer.handle, dev_i32(toks), 500, dev_i32(offs), 1)
+    outs = []
+    for hb in (h1, h2):
+        out = torch.empty(500, w.hidden, dtype=torch.float32, device="cuda")
+        ple.ple_forward_prepared(tiny_layer.handle, dev_bf16(hb), out, 1)
+        torch.cuda.synchronize()
+        outs.append(out.cpu().numpy())
+    assert np.array_equal(_f32bits(outs[1]), _f32bits(ref2))
+    assert not np.array_equal(outs[0], outs[1])
+
+
+def test_prepared_host_errors(tiny_layer):
+    w = tiny_layer.w
+    h = tiny_layer.handle
+    toks, offs, hid = pi.tiny_batch(w)
+    T = len(toks)
+    out = torch.empty(T, w.hidden, dtype=torch.float32, device="cuda")
+    hd = dev_bf16(hid)
+    # a ple_forward discards the prepared batch
+    gpu_forward(tiny_layer, toks, offs, hid, 1)
+    with pytest.raises(ple.PleError) as ei:
+        ple.ple_forward_prepared(h, hd, out, 1)
+    assert ei.value.code == 1
+    # state given without a prepared history, and the reverse
+    ple.ple_prepare(h, dev_i32(toks), T, dev_i32(offs), len(offs) - 1)
+    conv = torch.zeros(1, 3, w.hidden, dtype=torch.float32, device="cuda")
+    hist = dev_i32(np.full((1, 2), -1, np.int32))
+    with pytest.raises(ple.PleError) as ei:
+        ple.ple_forward_prepared(h, hd, out, 1, (hist, conv))
+    assert ei.value.code == 1
+    ple.ple_prepare(h, dev_i32(toks), T, dev_i32(offs), len(offs) - 1, hist)
+    with pytest.raises(ple.PleError) as ei:
+        ple.ple_forward_prepared(h, hd, out, 1)
+    assert ei.value.code == 1
+    # a decode step discards it too
+    ple.ple_prepare(h, dev_i32(toks), T, dev_i32(offs), len(offs) - 1)
+    ple.ple_decode_step(h, dev_i32(toks[:2].reshape(2, 1)), 2, 1, dev_bf16(hid[:2]),
+                        torch.empty(2, w.hidden, dtype=torch.float32, device="cuda"), 1,
+                        dev_i32(np.full((2, 2), -1, np.int32)),
+                        torch.zeros(2, 3, w.hidden, dtype=torch.float32, device="cuda"))
+    with pytest.raises(ple.PleError):
+        ple.ple_forward_prepared(h, hd, out, 1)
+    torch.cuda.synchronize()
+    assert ple.ple_get_error(h) == 0
+
+
+def test_prepared_equals_forward_full(full_layer):
+    w = pi.workload("prefill")
+    toks, offs, hid = pi.prefill_batch(w)
+    ref, _ = gpu_forward(full_layer, toks, offs, hid, 0)
+    got, _ = _prepared(full_layer, toks, offs, hid, 0)
+    assert np.array_equal(got, ref)
