@@ -365,6 +365,7 @@ def main():
         line["mtp"] = mtp_bench(ctx, layer, stream)
         line["long_context"] = long_bench(ctx, layer, stream)
         line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks)
+        line["prepared"] = prepared_bench(ctx, layer, sets, stream)
 
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         tokens, offsets, hidden = sets[0]["host"]
@@ -472,6 +473,52 @@ def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
     d2h = s0["out"].numel() * 2
     return {"value": s0["T"] * world * steps / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps}
+
+
+def prepared_bench(ctx, layer, sets, stream, steps=200):
+    """The layer split in two (ple_prepare, ple_forward_prepared) on the headline
+    batches: the time of each call, and of ple_forward, with CUDA events on the
+    launching stream. ple_prepare depends only on the tokens, so a model can issue
+    it while earlier layers run; ple_forward_prepared is what is left once the
+    hidden states exist."""
+    torch, ple = ctx["torch"], ctx["ple"]
+    h = layer.handle
+
+    def prep(i):
+        s = sets[i % len(sets)]
+        ple.ple_prepare(h, s["tokens"], s["T"], s["offsets"], s["S"], None, stream)
+
+    def rest(i):
+        s = sets[i % len(sets)]
+        ple.ple_forward_prepared(h, s["hidden"], s["out"], ple.PLE_OUT_BF16, None, stream)
+
+    def whole(i):
+        s = sets[i % len(sets)]
+        ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
+                        None, stream)
+
+    for i in range(5):
+        prep(i)
+        rest(i)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        ev[i][0].record(stream)
+        prep(i)
+        ev[i][1].record(stream)
+        rest(i)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_prep = sum(a.elapsed_time(b) for a, b, _ in ev) / steps
+    t_rest = sum(b.elapsed_time(c) for _, b, c in ev) / steps
+    t_whole = timed(ctx, stream, whole, steps) / steps
+    status = ple.ple_get_error(h)
+    return {"workload": "full-scale prefill batches, the layer in two calls",
+            "prepare_ms": t_prep, "forward_prepared_ms": t_rest, "forward_ms": t_whole,
+            "after_hidden_ready_ms_saved": t_whole - t_rest, "device_status": int(status),
+            "note": "ple_prepare needs only the tokens; ple_forward_prepared (gate, projection, conv, residual) "
+                    "is the part that waits for the hidden states"}
 
 
 def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
