@@ -134,6 +134,12 @@ bool encode_2d(ple_handle* h, CUtensorMap* map, CUtensorMapDataType dt, const vo
   return r == CUDA_SUCCESS;
 }
 
+// True when the current device is not the handle's (its memory and kernels live there).
+bool wrong_device(const ple_handle* h) {
+  int dev = -1;
+  return cudaGetDevice(&dev) != cudaSuccess || dev != h->device;
+}
+
 ple::TableRef table_ref(const ple_handle* h) {
   const bool nv = h->cfg.table_format == PLE_TABLE_NVFP4;
   return ple::TableRef{h->w.table, nv ? h->w.block_scales : nullptr, h->w.scales, nv ? 1 : 0};
@@ -420,6 +426,7 @@ ple_status ple_destroy(ple_handle* h) {
 ple_status ple_ngram_ids(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
                          const int32_t* hist, int32_t* ids, cudaStream_t stream) {
   if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
   if (T == 0) return PLE_OK;
   if (tokens == nullptr || offsets == nullptr || ids == nullptr) return PLE_ERR_INVALID_ARG;
@@ -442,6 +449,7 @@ ple_status ple_ngram_ids(ple_handle* h, const int32_t* tokens, int32_t T, const 
 
 ple_status ple_gather_rows(ple_handle* h, const int32_t* ids, int32_t T, void* e_out, cudaStream_t stream) {
   if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (T == 0) return PLE_OK;
   if (ids == nullptr || e_out == nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned(ids, 8) || !aligned(e_out, 16)) return PLE_ERR_ALIGN;
@@ -456,6 +464,7 @@ ple_status ple_forward(ple_handle* h, const int32_t* tokens, int32_t T, const in
                        const void* hidden, void* out, ple_out_dtype out_dtype, const ple_state* state,
                        cudaStream_t stream) {
   if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
   if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
   if (T == 0) return PLE_OK;
@@ -471,6 +480,7 @@ ple_status ple_forward(ple_handle* h, const int32_t* tokens, int32_t T, const in
 ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
                        const int32_t* hist, cudaStream_t stream) {
   if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
   h->prepared.valid = false;
   if (T > 0) {
@@ -508,6 +518,7 @@ ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const in
 ple_status ple_forward_prepared(ple_handle* h, const void* hidden, void* out, ple_out_dtype out_dtype,
                                 const ple_state* state, cudaStream_t stream) {
   if (h == nullptr || !h->prepared.valid) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
   if ((state != nullptr) != h->prepared.with_hist) return PLE_ERR_INVALID_ARG;
   const int32_t T = h->prepared.T, S = h->prepared.S;
@@ -538,6 +549,7 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
                            ple_out_dtype out_dtype, int32_t* hist, float* conv_state, const int32_t* n_commit,
                            cudaStream_t stream) {
   if (h == nullptr) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
   if (B < 1 || q < 1 || B > h->cfg.max_seqs || static_cast<int64_t>(B) * q > h->cfg.max_tokens) return PLE_ERR_SHAPE;
   if (tokens == nullptr || hidden == nullptr || out == nullptr || hist == nullptr || conv_state == nullptr)

@@ -474,15 +474,15 @@ uint64_t barrett_magic(int64_t m) { return ~0ull / static_cast<uint64_t>(m); }
 
 cudaError_t launch_decode_small(const CUtensorMap& tmap_w, const DecodeSmallArgs& a, int32_t grid,
                                 cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_small_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static PerDeviceOnce configured;
+  const cudaError_t e = configured.run([] {
+    cudaError_t r = cudaFuncSetAttribute(decode_small_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemLimit);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_small_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(decode_small_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);

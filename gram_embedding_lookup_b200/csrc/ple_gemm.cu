@@ -535,13 +535,11 @@ template <int CTAS>
 cudaError_t launch_gemm_impl(const CUtensorMap& tmap_w, const CUtensorMap& tmap_e, const CUtensorMap& tmap_h,
                              const CUtensorMap& tmap_o, const CUtensorMap& tmap_o_head, const GemmParams& p, int grid,
                              cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_kernel<CTAS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static PerDeviceOnce configured;
+  const cudaError_t e = configured.run([] {
+    return cudaFuncSetAttribute(gemm_kernel<CTAS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(NUM_THREADS);

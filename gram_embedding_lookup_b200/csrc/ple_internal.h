@@ -7,11 +7,34 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "ple.h"
 
 namespace ple {
 
 struct TokMeta;
+
+// Kernel attributes (such as the dynamic shared-memory limit) belong to the
+// device that is current when they are set. PerDeviceOnce runs a setup once for
+// every device a process uses (devices 0..63; others run it on every call).
+class PerDeviceOnce {
+ public:
+  template <typename F>
+  cudaError_t run(F&& setup) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (bit != 0 && (done_.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = setup();
+    if (e == cudaSuccess && bit != 0) done_.fetch_or(bit, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  std::atomic<uint64_t> done_{0};
+};
 
 // The table as the kernels see it (ple_table_format in ple.h).
 struct TableRef {

@@ -44,7 +44,8 @@
  *   - errors that only the device can see (token outside [0, vocab),
  *     inconsistent offsets, an internal wait that ran out) set a sticky status
  *     word in the handle, read and cleared by ple_get_error();
- *   - a handle is used by one stream at a time.
+ *   - a handle is used by one stream at a time, with the device it was
+ *     created on current (another current device gives PLE_ERR_INVALID_ARG).
  */
 #ifndef PLE_H_
 #define PLE_H_
