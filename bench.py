@@ -227,6 +227,41 @@ def prefill_config(args, w, world):
             "l2": f"{args.sets} rotating input sets (>2x L2 per step)", "out_dtype": "bf16"}
 
 
+# ----------------------------------------------------------------------------- ranks
+class Comm:
+    """Coordination of the replicas (one process per GPU, no data-path collective):
+    a barrier around the timed region and the maximum of a time over the ranks.
+    NCCL on the GPUs; the CPU tests run the same code over gloo."""
+
+    def __init__(self, world: int, dist=None, device: str = "cuda"):
+        self.world = world
+        self.dist = dist
+        self.device = device
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def replica_value(tokens_per_step: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processes tokens_per_step per step (weak
+    scaling); the time is the slowest rank's."""
+    return tokens_per_step * world * steps / (ms_max / 1e3)
+
+
+def replica_variant(v: int, rank: int) -> int:
+    """Input-set index of rank ``rank``: each replica draws its own batches."""
+    return v + 100 * rank
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def main():
     args = parse_args()
@@ -251,16 +286,8 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    comm = Comm(world, dist, "cuda")
+    barrier, max_over_ranks = comm.barrier, comm.max
 
     ctx = dict(torch=torch, ple=ple, pi=pi, bf16_tensor=bf16_tensor, barrier=barrier,
                max_over_ranks=max_over_ranks, world=world, args=args)
@@ -274,7 +301,7 @@ def main():
 
     sets = []
     for v in range(args.sets):
-        tokens, offsets, hidden = pi.prefill_batch(w, variant=v + 100 * rank)
+        tokens, offsets, hidden = pi.prefill_batch(w, variant=replica_variant(v, rank))
         sets.append(dict(tokens=torch.from_numpy(tokens).cuda(), offsets=torch.from_numpy(offsets).cuda(),
                          hidden=bf16_tensor(hidden), out=torch.empty(len(tokens), H, dtype=torch.bfloat16,
                                                                       device="cuda"),
@@ -318,7 +345,7 @@ def main():
     ms = max_over_ranks(ev0.elapsed_time(ev1))
     T = sets[0]["T"]
     ms_per_step = ms / args.steps
-    value = T * world * args.steps / (ms / 1e3)
+    value = replica_value(T, world, args.steps, ms)
 
     peaks, peak_kind = load_peaks()
     gemm_ms, gemm_n = stage["gemm"]
