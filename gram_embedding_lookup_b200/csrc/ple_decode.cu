@@ -84,10 +84,6 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_
                : "r"(addr));
 }
 
-__device__ __forceinline__ void pdl_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Unit partition: CTA b of G owns units [u0(b), u0(b + 1)) with u0(b) = b * U / G;
 // the owner of unit u is the largest b with u0(b) <= u. 32-bit: the host

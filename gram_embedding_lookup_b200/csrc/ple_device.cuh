@@ -29,6 +29,16 @@ struct __align__(16) TokMeta {
 };
 constexpr int32_t kFlagLast = 1;
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// launch_dependents lets the next kernel in the stream (launched with
+// programmatic stream serialization) start once every CTA of this grid has
+// issued it; wait blocks until the previous grid has completed and its memory
+// is visible. Data the previous kernel writes is read only after the wait.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ smem address helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

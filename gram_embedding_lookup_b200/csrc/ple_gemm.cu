@@ -406,6 +406,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
       // bytes the even CTA's full barrier receives per stage (both CTAs' loads)
       const uint32_t tx_bytes = CTAS * (A_STAGE + static_cast<uint32_t>(p.n_tok / CTAS) * BK * 2);
       bool ok = true;
+      bool e_ready = false;
       for (int tile = unit; tile < total_tiles && ok; tile += units) {
         int m, n, ks;
         tile_coords(p, tile, m, n, ks);
@@ -420,9 +421,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
           if constexpr (CTAS == 2) {
             const uint32_t fb0 = mapa_shared(fb, 0);
             tma_load_2d_pair(sA + stage * A_STAGE, &tmap_w, kb * BK, chA, fb0);
+            if (!e_ready) { pdl_wait(); e_ready = true; }   // e comes from the previous kernel
             tma_load_2d_pair(sB + stage * C::B_STAGE, &tmap_e, kb * BK, tokB, fb0);
           } else {
             tma_load_2d(sA + stage * A_STAGE, &tmap_w, kb * BK, chA, fb);
+            if (!e_ready) { pdl_wait(); e_ready = true; }
             tma_load_2d(sB + stage * C::B_STAGE, &tmap_e, kb * BK, tokB, fb);
           }
           issued[stage] = true;
@@ -503,6 +506,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
     const TileWalk walk{unit, units, total_tiles, static_cast<int>(rank), CTAS};
     uint32_t q = 0;
     TokMeta mt_next[2];
+    // metadata, gates, the state snapshot and the new history come from the
+    // previous kernel; every output store happens after this wait
+    pdl_wait();
     if (p.fused) load_meta(p, walk, 0, et, mt_next);
     int it = 0;
     bool ok = true;
@@ -545,13 +551,17 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmap_w, const CUtensorMap& tmap_
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = kGemmSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CTAS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the prologue, W_proj and h overlap the embed
+  // kernel's tail (the kernel waits before it reads anything that kernel writes)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_kernel<CTAS>, tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, p);
 }
 

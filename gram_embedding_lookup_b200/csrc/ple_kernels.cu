@@ -317,6 +317,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  // the projection may start its prologue on SMs this kernel leaves; it reads
+  // the rows, gates and state only after this grid has completed
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ---- producer: row IDs, a lane per token
