@@ -393,6 +393,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
   if constexpr (CTAS == 2) cluster_sync();     // the peer's barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
+  // a combine kernel after the split-K form may launch now; it waits for this grid
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)

@@ -459,6 +459,7 @@ __global__ void __launch_bounds__(128) combine_forward_kernel(const CombineArgs 
   const int32_t t = blockIdx.y;
   const int32_t j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= a.H || t >= a.T) return;
+  pdl_wait();                                  // the partial sums come from the projection
   const TokMeta mt = a.meta[t];
   float u[4];                          // u[k] = u_{t-3+k}
 #pragma unroll
@@ -495,6 +496,7 @@ __global__ void __launch_bounds__(128) combine_decode_kernel(const DecodeCombine
   const int32_t b = blockIdx.y;
   const int32_t j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= a.H || b >= a.B) return;
+  pdl_wait();                                  // the partial sums come from the projection
   int32_t nc = a.n_commit ? a.n_commit[b] : a.q;
   if (nc < 1 || nc > a.q) {
     if (j == 0) set_status(a.status, PLE_ERR_RANGE);
@@ -587,16 +589,28 @@ cudaError_t launch_convert_w(const __nv_bfloat16* w, int32_t D, int32_t H, __hal
   return cudaGetLastError();
 }
 
+// Combine kernels start under programmatic dependent launch: their blocks wait
+// for the projection before they read anything it writes.
+template <typename Kernel, typename Args>
+cudaError_t launch_after_projection(Kernel kernel, dim3 grid, const Args& a, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 cudaError_t launch_combine_forward(const CombineArgs& a, cudaStream_t stream) {
-  dim3 grid((a.H + 127) / 128, a.T);
-  combine_forward_kernel<<<grid, 128, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_after_projection(combine_forward_kernel, dim3((a.H + 127) / 128, a.T), a, stream);
 }
 
 cudaError_t launch_combine_decode(const DecodeCombineArgs& a, cudaStream_t stream) {
-  dim3 grid((a.H + 127) / 128, a.B);
-  combine_decode_kernel<<<grid, 128, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_after_projection(combine_decode_kernel, dim3((a.H + 127) / 128, a.B), a, stream);
 }
 
 }  // namespace ple
