@@ -571,25 +571,8 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
     layer = DeviceLayer(w, max_tokens=16384, max_seqs=64, table_format=ple.PLE_TABLE_NVFP4)
     h = layer.handle
 
-    def step(i):
-        s = sets[i % len(sets)]
-        ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
-                        None, stream)
-
-    for i in range(5):
-        step(i)
-    ple.ple_set_profiling(h, True)
-    ple.ple_get_stage_times(h)
-    ms = timed(ctx, stream, step, steps)
-    stage = ple.ple_get_stage_times(h)
-    ple.ple_set_profiling(h, False)
-    T = sets[0]["T"]
-    e_ms, e_n = stage["prepare"]
-    e_s = e_ms / 1e3 / max(e_n, 1)
-    row_bytes = 2 * (D // 2 + D // 16) + 8                  # both rows' codes and block scales, row scales
-    embed_bytes = T * (2 * H + row_bytes + 2 * D + 8 + 16 + 4)
-    g_ms, g_n = stage["gemm"]
-
+    # the decode step first, before the prefill loop heats the GPU into its power cap
+    # (the headline decode line also runs on a GPU that has been mostly idle)
     wd = pi.workload("decode")
     tokens, hidden, hist, conv = pi.decode_batch(wd)
     B, q = tokens.shape
@@ -606,6 +589,29 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
         dstep(i)
     n_dec = 500
     d_ms = timed(ctx, stream, dstep, n_dec)
+
+    def step(i):
+        s = sets[i % len(sets)]
+        ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
+                        None, stream)
+
+    for i in range(5):
+        step(i)
+    ms = timed(ctx, stream, step, steps)            # no events between the kernels
+    ple.ple_set_profiling(h, True)                  # then per-kernel durations
+    ple.ple_get_stage_times(h)
+    for i in range(min(steps, 100)):
+        step(i)
+    torch.cuda.synchronize()
+    stage = ple.ple_get_stage_times(h)
+    ple.ple_set_profiling(h, False)
+    T = sets[0]["T"]
+    e_ms, e_n = stage["prepare"]
+    e_s = e_ms / 1e3 / max(e_n, 1)
+    row_bytes = 2 * (D // 2 + D // 16) + 8                  # both rows' codes and block scales, row scales
+    embed_bytes = T * (2 * H + row_bytes + 2 * D + 8 + 16 + 4)
+    g_ms, g_n = stage["gemm"]
+
     status = ple.ple_get_error(h)
     layer.close()
     world = ctx["world"]
