@@ -472,8 +472,14 @@ def gather_bench(ctx, layer, sets, stream, peaks):
 
 
 def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
-    """Same metric through the C ABI with host buffers: H2D of the step's inputs from
-    pinned memory, the layer, D2H of the output, all inside the timed region."""
+    """Same metric through the C ABI with host buffers: every step's inputs go up from
+    pinned host memory and its output comes back down, all inside the timed region.
+
+    As a serving loop would run it, the copies overlap the layer. Step i+1's inputs
+    go up on one copy stream and step i-1's output comes down on another while step i
+    runs on the compute stream. The input sets form a ring of device buffers, and
+    events order each buffer's upload, layer call and download. The same steps run
+    in series on one stream are reported beside it."""
     import torch
     hosts = []
     for s in sets:
@@ -481,9 +487,33 @@ def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
         hosts.append(dict(tokens=torch.from_numpy(tokens).pin_memory(), offsets=torch.from_numpy(offsets).pin_memory(),
                           hidden=torch.from_numpy(hidden.view(np.int16)).view(torch.bfloat16).pin_memory(),
                           out=torch.empty_like(s["out"], device="cpu").pin_memory()))
+    nb = len(sets)
+    s_up, s_down = torch.cuda.Stream(), torch.cuda.Stream()
+    up_done = [torch.cuda.Event() for _ in range(nb)]
+    comp_done = [torch.cuda.Event() for _ in range(nb)]
+    down_done = [torch.cuda.Event() for _ in range(nb)]
 
-    def step(i):
-        s, hs = sets[i % len(sets)], hosts[i % len(sets)]
+    def step_overlapped(i):
+        b = i % nb
+        s, hs = sets[b], hosts[b]
+        s_up.wait_event(comp_done[b])           # the layer is done with this buffer's inputs
+        with torch.cuda.stream(s_up):
+            s["tokens"].copy_(hs["tokens"], non_blocking=True)
+            s["offsets"].copy_(hs["offsets"], non_blocking=True)
+            s["hidden"].copy_(hs["hidden"], non_blocking=True)
+        up_done[b].record(s_up)
+        stream.wait_event(up_done[b])
+        stream.wait_event(down_done[b])         # this buffer's previous output is down
+        ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
+                        None, stream)
+        comp_done[b].record(stream)
+        s_down.wait_event(comp_done[b])
+        with torch.cuda.stream(s_down):
+            hs["out"].copy_(s["out"], non_blocking=True)
+        down_done[b].record(s_down)
+
+    def step_serial(i):
+        s, hs = sets[i % nb], hosts[i % nb]
         s["tokens"].copy_(hs["tokens"], non_blocking=True)
         s["offsets"].copy_(hs["offsets"], non_blocking=True)
         s["hidden"].copy_(hs["hidden"], non_blocking=True)
@@ -491,24 +521,32 @@ def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
                         None, stream)
         hs["out"].copy_(s["out"], non_blocking=True)
 
-    for i in range(max(args.warmup, 3)):
-        step(i)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
     steps = 20
-    for i in range(steps):
-        step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+
+    def timed_steps(step, first, last):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(first)
+        for i in range(steps):
+            step(i)
+        last.wait_stream(stream)
+        e1.record(last)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    ms = timed_steps(step_overlapped, s_up, s_down)
+    ms_serial = timed_steps(step_serial, stream, stream)
     s0 = sets[0]
     h2d = s0["tokens"].numel() * 4 + s0["offsets"].numel() * 4 + s0["hidden"].numel() * 2
     d2h = s0["out"].numel() * 2
     return {"value": s0["T"] * world * steps / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps}
+            "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps,
+            "copies": "overlapped with the layer (copy streams, ring of 3 buffer sets)",
+            "serial": {"value": s0["T"] * world * steps / (ms_serial / 1e3), "ms_per_step": ms_serial / steps}}
 
 
 def prepared_bench(ctx, layer, sets, stream, steps=200):
