@@ -402,6 +402,7 @@ def main():
         line["long_context"] = long_bench(ctx, layer, stream)
         line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks)
         line["prepared"] = prepared_bench(ctx, layer, sets, stream)
+        line["gather_fused"] = gather_fused_bench(ctx, layer, sets, stream, peaks)
 
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         tokens, offsets, hidden = sets[0]["host"]
@@ -547,6 +548,45 @@ def e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier):
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps,
             "copies": "overlapped with the layer (copy streams, ring of 3 buffer sets)",
             "serial": {"value": s0["T"] * world * steps / (ms_serial / 1e3), "ms_per_step": ms_serial / steps}}
+
+
+def gather_fused_bench(ctx, layer, sets, stream, peaks, steps=300):
+    """Forward path 4 on the headline batches: the rows are gathered and
+    dequantised inside the projection kernel (the fp16 rows never reach HBM),
+    after a kernel that computes only the row IDs and the gate. Step time with
+    no events in between, then per-kernel times from a pass with stage events."""
+    torch, ple = ctx["torch"], ctx["ple"]
+    h = layer.handle
+    D, H = layer.w.row_dim, layer.w.hidden
+
+    def step(i):
+        s = sets[i % len(sets)]
+        ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
+                        None, stream)
+
+    ple.ple_set_forward_path(h, 4)
+    try:
+        for i in range(5):
+            step(i)
+        ms = timed(ctx, stream, step, steps) / steps
+        ple.ple_set_profiling(h, True)
+        ple.ple_get_stage_times(h)
+        for i in range(min(steps, 100)):
+            step(i)
+        torch.cuda.synchronize()
+        st = ple.ple_get_stage_times(h)
+        ple.ple_set_profiling(h, False)
+    finally:
+        ple.ple_set_forward_path(h, 0)
+    status = ple.ple_get_error(h)
+    T = sets[0]["T"]
+    gemm_ms = st["gemm"][0] / max(st["gemm"][1], 1)
+    tf = 2.0 * D * H * T / (gemm_ms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    return {"workload": "full-scale prefill batches, forward path 4 (gather fused into the projection)",
+            "value": T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "stage_ms_per_launch": {k: v[0] / max(v[1], 1) for k, v in st.items() if v[1]},
+            "gemm_tflops": tf, "gemm_frac_of_sustained_peak": tf / peak, "device_status": int(status)}
 
 
 def prepared_bench(ctx, layer, sets, stream, steps=200):

@@ -77,7 +77,8 @@ Plan plan_projection(const ple_handle* h, int T, int path, int64_t partial_cap) 
   const int m_tiles = h->cfg.hidden / kTileM;
   const int num_kb = h->cfg.row_dim / kTileK;
   const int fused_tiles_n = ceil_div(T, kFusedRows - kHalo);
-  bool fused = (path == 1 || path == 3) || (path == 0 && static_cast<int64_t>(m_tiles) * fused_tiles_n >= h->num_sms);
+  bool fused = (path == 1 || path == 3 || path == 4) ||
+               (path == 0 && static_cast<int64_t>(m_tiles) * fused_tiles_n >= h->num_sms);
   if (!fused) {
     const int n_tok = std::min(256, ceil_div(T, 16) * 16);
     const int n_tiles = ceil_div(T, n_tok);
@@ -90,6 +91,20 @@ Plan plan_projection(const ple_handle* h, int T, int path, int64_t partial_cap) 
   }
   const int ctas = (path != 3 && h->cfg.hidden % (2 * kTileM) == 0 && h->num_sms >= 2) ? 2 : 1;
   return Plan{true, kFusedRows, kFusedRows - kHalo, -kHalo, kHalo, fused_tiles_n, 1, ctas};
+}
+
+// Whether ple_forward on T tokens runs the gather-fused projection (the token
+// operand gathered from the table inside the projection kernel, never written
+// to HBM): path 4, E4M3 tables, SM-pair tiles. It is not the automatic choice:
+// the kernel dequantises each token's rows once per 256-channel tile (ten
+// times at hidden 2560) inside the tensor-bound kernel, and measures slower
+// than the embed kernel followed by the TMA-fed projection.
+bool gather_fused(const ple_handle* h, int T) {
+  if (h->forward_path != 4 || h->cfg.table_format != PLE_TABLE_E4M3) return false;
+  if (h->cfg.rows[0] + h->cfg.rows[1] >= (int64_t(1) << 31)) return false;   // rows are int32 in the kernel
+  if (!ple::gather_fused_supported(h->cfg.row_dim / kTileK)) return false;
+  const Plan pl = plan_projection(h, T, 4, h->partial_elems);
+  return pl.fused && pl.ctas == 2;
 }
 
 cudaEvent_t take_event(ple_handle* h) {
@@ -165,7 +180,7 @@ void free_all(ple_handle* h) {
 
 ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q, const void* hidden, void* out,
                           ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist, float* dec_conv,
-                          const int32_t* tokens, const int32_t* n_commit, cudaStream_t stream);
+                          const int32_t* tokens, const int32_t* n_commit, bool gather, cudaStream_t stream);
 
 // Runs prepare + gather + projection (+ combine) for a packed batch.
 ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
@@ -196,24 +211,29 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
     pa.hist_new = h->hist_new;
   }
   pa.status = h->status;
-  // row IDs, gate and the gathered, dequantised rows in one kernel
+  // row IDs, gate and the gathered, dequantised rows in one kernel; for the
+  // gather-fused projection, IDs and gate only
+  const bool gather = !decode && gather_fused(h, T);
   h->prepared.valid = false;            // the scratch now holds this call's batch
   const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
-    return ple::launch_embed(pa, table_ref(h), c.row_dim, h->e, h->num_sms, stream);
+    return ple::launch_embed(pa, table_ref(h), c.row_dim, gather ? nullptr : h->e, h->num_sms, stream);
   });
   if (st != PLE_OK) return st;
-  return run_projection(h, T, S, uniform_q, hidden, out, dtype, state, dec_hist, dec_conv, tokens, n_commit, stream);
+  return run_projection(h, T, S, uniform_q, hidden, out, dtype, state, dec_hist, dec_conv, tokens, n_commit, gather,
+                        stream);
 }
 
 // The projection and everything after it, on the rows, IDs and metadata in the
 // handle's scratch (written by the embed kernel, or by ple_prepare plus the gate
-// kernel).
+// kernel). gather: the rows are not in the scratch; the projection gathers them
+// from the table by the IDs.
 ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q, const void* hidden, void* out,
                           ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist, float* dec_conv,
-                          const int32_t* tokens, const int32_t* n_commit, cudaStream_t stream) {
+                          const int32_t* tokens, const int32_t* n_commit, bool gather, cudaStream_t stream) {
   const ple_config& c = h->cfg;
   const bool decode = uniform_q > 0;
-  const Plan pl = plan_projection(h, T, decode ? 2 : h->forward_path, h->partial_elems);
+  const Plan pl = plan_projection(h, T, decode ? 2 : (gather ? 4 : h->forward_path), h->partial_elems);
+  if (gather && !(pl.fused && pl.ctas == 2)) return PLE_ERR_UNSUPPORTED;
   ple_status st = PLE_OK;
   CUtensorMap tmap_e{}, tmap_h{}, tmap_o{}, tmap_o_head{};
   if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->e, c.row_dim, T, static_cast<uint64_t>(c.row_dim) * 2,
@@ -254,9 +274,16 @@ ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q
   gp.out_f32 = dtype == PLE_OUT_F32 ? 1 : 0;
   gp.partial = h->partial;
   gp.status = h->status;
+  if (gather) {
+    gp.ids = reinterpret_cast<const int2*>(h->ids);
+    gp.codes = h->w.table;
+    gp.scales = h->w.scales;
+    gp.rows0 = c.rows[0];
+  }
   const int total = gp.m_tiles * gp.n_tiles * gp.k_splits;
   const int grid = pl.ctas == 2 ? 2 * std::min(total, h->num_sms / 2) : std::min(total, h->num_sms);
-  st = run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_gemm(h->tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, gp, grid, pl.ctas, stream);
+  st = run_stage(h, PLE_STAGE_GEMM, stream, [&] {
+    return ple::launch_gemm(h->tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, gp, grid, pl.ctas, gather, stream);
   });
   if (st != PLE_OK || pl.fused) return st;
 
@@ -542,7 +569,7 @@ ple_status ple_forward_prepared(ple_handle* h, const void* hidden, void* out, pl
   }
   const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_gate(ga, stream); });
   if (st != PLE_OK) return st;
-  return run_projection(h, T, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, nullptr, stream);
+  return run_projection(h, T, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, nullptr, false, stream);
 }
 
 ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const void* hidden, void* out,
@@ -634,7 +661,7 @@ ple_status ple_get_stage_times(ple_handle* h, float* ms, int64_t* launches) {
 }
 
 ple_status ple_set_forward_path(ple_handle* h, int32_t path) {
-  if (h == nullptr || path < 0 || path > 3) return PLE_ERR_INVALID_ARG;
+  if (h == nullptr || path < 0 || path > 4) return PLE_ERR_INVALID_ARG;
   h->forward_path = path;
   return PLE_OK;
 }

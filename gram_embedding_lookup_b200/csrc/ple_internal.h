@@ -68,7 +68,8 @@ struct PrepareArgs {
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
 
 // Prepare and gather fused (one pass over HBM): ids, metadata with the gate,
-// and e[t] for the batch. num_sms sizes the persistent grid.
+// and e[t] for the batch. num_sms sizes the persistent grid. With e null it
+// writes only the ids and the metadata (the gather-fused projection follows).
 cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
                          cudaStream_t stream);
 
@@ -103,15 +104,26 @@ struct GemmParams {
   int32_t out_f32;
   float* partial;        // [k_splits][T][H]
   int32_t* status;
+  // gather-fused form only: the kernel builds the token operand itself from
+  // the E4M3 table rows named by ids
+  const int2* ids;       // [T] (row of order 0, row of order 1)
+  const uint8_t* codes;  // [2][R][D]; order 1 starts at row rows0
+  const float* scales;   // [2][R]
+  int64_t rows0;
 };
 constexpr int kGemmSmemBytes = 227 * 1024;   // the sm_100 per-block maximum
 // tmap_o / tmap_o_head: bf16 output tiles of 32 and of 29 tokens (the first
 // chunk of a fused tile without its halo rows).
 // ctas = 2: SM-pair tiles (clusters of two CTAs, 256 channels per tile, grid even,
 // m_tiles = hidden / 256, tmap_e boxes of n_tok / 2 rows); ctas = 1: single-SM tiles.
+// gather = true (ctas = 2, fused, n_tok = 256 only): the token operand is
+// gathered and dequantised from the table inside the kernel (p.ids, p.codes,
+// p.scales, p.rows0); tmap_e is not read.
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_e, const CUtensorMap& tmap_h,
                         const CUtensorMap& tmap_o, const CUtensorMap& tmap_o_head, const GemmParams& p, int grid,
-                        int ctas, cudaStream_t stream);
+                        int ctas, bool gather, cudaStream_t stream);
+// Whether the gather-fused form takes rows of num_kb K-stages (64 codes each).
+bool gather_fused_supported(int32_t num_kb);
 
 // Combine split-K partials + gate + conv + residual (+ state) for a packed batch.
 struct CombineArgs {

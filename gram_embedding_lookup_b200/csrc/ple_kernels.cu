@@ -280,7 +280,8 @@ __global__ void __launch_bounds__(256) gate_kernel(const PrepareArgs a, int toke
 // loads at once: its hidden row and its two table rows (plain 16-byte loads,
 // which keep more bytes in flight per SM than bulk copies of single rows do).
 // Then come the gate dot product (fp32, lane-strided, then a warp reduction),
-// the dequantisation into fp16 e_t and the metadata. Batches go through the
+// the dequantisation into fp16 e_t and the metadata (with e null the rows are
+// skipped: the gather-fused projection reads them itself). Batches go through the
 // ring in order, so every parity wait is for the phase after the one last
 // released.
 constexpr int kPipeConsumers = 15;                   // 16 warps in all: 128 registers per thread
@@ -369,6 +370,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
       };
       const bool with_gate = a.hidden != nullptr;     // null: ple_prepare, the gate comes later
+      const bool with_rows = e != nullptr;            // null: the projection gathers the rows itself
       if (with_gate && b * kPipeBatch + cw < n) load_hidden(t0 + b * kPipeBatch + cw);
       if (!state_done) {
         state_blocks(a, blockIdx.x, gridDim.x, threadIdx.x - 32, blockDim.x - 32);
@@ -391,13 +393,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 #pragma unroll
         for (int r = 0; r < kEmbedD16; ++r) {
           const int j = lane + 32 * r;
-          if (j < D16) {
+          if (with_rows && j < D16) {
             ca[r] = load_chunk<NV>(tab.codes, tab.blocks, ra, D, j);
             cb[r] = load_chunk<NV>(tab.codes, tab.blocks, rb, D, j);
           }
         }
-        const float s0 = __ldg(tab.scales + ra);
-        const float s1 = __ldg(tab.scales + rb);
+        const float s0 = with_rows ? __ldg(tab.scales + ra) : 0.f;
+        const float s1 = with_rows ? __ldg(tab.scales + rb) : 0.f;
         const float g = with_gate ? gate_warp(hv, hrow, wg, H8, lane) : 0.f;
         if (lane == 0) {
           TokMeta m;
@@ -407,6 +409,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           m.flags = pt.flags;
           a.meta[t] = m;
         }
+        if (!with_rows) continue;                            // warp-uniform
         // e_t = deq(bigram row) + deq(trigram row), fp16
         uint4* erow = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D);
         auto emit = [&](int j, const RowChunk<NV>& x, const RowChunk<NV>& y) {

@@ -239,7 +239,8 @@ const char* ple_status_string(ple_status status);
 
 /* Kernel stages of the library, in launch order within a call. In
  * ple_forward and ple_decode_step the PREPARE stage also gathers and
- * dequantises the rows (one fused kernel); ple_prepare and the gate kernel of
+ * dequantises the rows (one fused kernel), except on the gather-fused path,
+ * where the GEMM stage does; ple_prepare and the gate kernel of
  * ple_forward_prepared count as PREPARE too. GATHER counts ple_gather_rows. */
 enum { PLE_STAGE_PREPARE = 0, PLE_STAGE_GATHER = 1, PLE_STAGE_GEMM = 2, PLE_STAGE_COMBINE = 3,
        PLE_NUM_STAGES = 4 };
@@ -257,9 +258,16 @@ ple_status ple_get_stage_times(ple_handle* handle, float* ms, int64_t* launches)
  * (gate, conv and residual inside the projection kernel, conv halo
  * recomputed per tile; SM-pair tiles of 256 channels when hidden % 256 == 0),
  * 2 = split-K projection followed by a combine kernel, 3 = fused epilogue with
- * single-SM tiles of 128 channels. For ple_decode_step: steps of B * q <= 16
- * tokens with out != hidden run as one kernel unless path is 2, which forces
- * the split-K path. */
+ * single-SM tiles of 128 channels, 4 = as 1, but with the row gather and
+ * dequantisation inside the projection kernel: the first kernel computes only
+ * the row IDs and the gate, and the projection reads the FP8 rows itself into
+ * its shared-memory operand tiles, so the fp16 rows never reach HBM (E4M3
+ * tables, SM-pair tiles, row_dim >= 128; elsewhere path 4 runs as
+ * path 1). Paths 1 and 4 give identical bits; path 4 is never chosen
+ * automatically, because on B200 it is slower (each token's rows are
+ * dequantised once per 256-channel tile inside the tensor-bound kernel). For ple_decode_step: steps of B * q <= 16 tokens with
+ * out != hidden run as one kernel unless path is 2, which forces the split-K
+ * path. */
 ple_status ple_set_forward_path(ple_handle* handle, int32_t path);
 
 /* Total number of kernels the handle has launched since creation. */
