@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e, decode and clocks measurements")
     ap.add_argument("--ref-tokens", type=int, default=512, help="tokens per reference-arm step")
+    ap.add_argument("--path", type=int, default=0,
+                    help="forward path of the timed prefill steps (ple_set_forward_path; 0 = automatic, "
+                         "4 = gather fused into the projection)")
     return ap.parse_args()
 
 
@@ -224,7 +227,8 @@ def prefill_config(args, w, world):
                         "Zipf(1.1) tokens over 248,320, hidden 2560, 2 x 10,000,048 x 2560 FP8 table in HBM",
             "model": "PLE n-gram embedding layer", "global_batch": 16384 * world, "seq_len": 16384,
             "table_rows_per_order": w.rows_per_order, "parallelism": f"replicas x{world}",
-            "l2": f"{args.sets} rotating input sets (>2x L2 per step)", "out_dtype": "bf16"}
+            "l2": f"{args.sets} rotating input sets (>2x L2 per step)", "out_dtype": "bf16",
+            "forward_path": args.path}
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -312,6 +316,7 @@ def main():
         ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
                         None, stream)
 
+    ple.ple_set_forward_path(h, args.path)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -349,6 +354,7 @@ def main():
     torch.cuda.synchronize()
     stage = ple.ple_get_stage_times(h)
     ple.ple_set_profiling(h, False)
+    ple.ple_set_forward_path(h, 0)
     status = ple.ple_get_error(h)
     ms = max_over_ranks(ev0.elapsed_time(ev1))
     T = sets[0]["T"]
@@ -372,8 +378,11 @@ def main():
                 "algorithmic_flops_per_launch": flops, "launch_ms": gemm_s * 1e3}
     e_ms, e_n = stage["prepare"]
     e_s = e_ms / 1e3 / max(e_n, 1)
-    embed_bytes = T * (2 * H + 2 * D + 8 + 2 * D + 8 + 16 + 4)   # h, rows, scales in; e, ids, meta out; tokens
-    embed = {"kernel": "embed_kernel (ids + gate + row gather/dequant)", "bound": "hbm",
+    if args.path == 4:      # the first kernel computes only IDs and gate: h and tokens in; ids, meta out
+        embed_bytes, embed_name = T * (2 * H + 8 + 16 + 4), "embed_kernel without rows (ids + gate)"
+    else:                   # h, rows, scales in; e, ids, meta out; tokens
+        embed_bytes, embed_name = T * (2 * H + 2 * D + 8 + 2 * D + 8 + 16 + 4), "embed_kernel (ids + gate + row gather/dequant)"
+    embed = {"kernel": embed_name, "bound": "hbm",
              "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
              "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"], "launch_ms": e_s * 1e3,
              "algorithmic_bytes_per_launch": embed_bytes,
