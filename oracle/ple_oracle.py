@@ -44,6 +44,11 @@ details. The readings fixed here (each marked READING) are:
 * C-12 carried state: the last two tokens and the last three u rows.
 * C-16 the NVFP4 table variant: FP4 E2M1 codes, two per byte (low nibble
        first), an E4M3 scale per 16 codes and the C-6 row scale.
+* C-17 the multi-head row layout (the SSD-stream model card's geometry: 16
+       table lookups per token of 160-byte rows): 8 heads per order, head j of
+       order n reads sub-table 8n + j at row fold(k_n ^ j*HEAD_MIX) mod R'
+       (head 0 is the C-4 row), each row carries its own scale, and e is the
+       16 dequantised rows concatenated in head order.
 
 Precision: every step is evaluated in float64 (library matmul for the
 projection and the gate dot product); the caller rounds the float64 result
@@ -235,6 +240,46 @@ def ngram_ids(tokens, offsets, rows, hist=None) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
+# C-17  the multi-head row layout (READING)
+# --------------------------------------------------------------------------------------
+# The SSD-stream model card (bittide.aicompass.dev mirror, section "技术细节")
+# says the model makes 16 deterministic table lookups per generated token and
+# that each FP8 row is 160 bytes; the same card gives the table as one file of
+# 51,200,245,760 bytes, which is 16 sub-tables x 20,000,096 rows x 160 bytes.
+# The main reading of this build (C-13) keeps 2 lookups of 2560-byte rows; this
+# variant reads the card literally: each order (bigram, trigram) has 8 hash
+# heads, head j of order n owns sub-table 8n + j, and the 16 rows of a token,
+# each dequantised with its own row scale, are concatenated in head order to
+# the 2560-wide e (16 x 160). Heads are separated by xor-ing a per-head
+# multiple of an odd constant into the order's key before the fold, so head 0
+# is exactly the C-4 row.
+
+HEADS_PER_ORDER = 8
+HEAD_MIX = 0xFF51AFD7ED558CCD   # odd 64-bit constant (MurmurHash3's 64-bit finaliser multiplier)
+
+
+def ngram_ids_heads(tokens, offsets, rows_per_head, hist=None, heads=HEADS_PER_ORDER) -> np.ndarray:
+    """Row IDs [T][2 * heads]: column n * heads + j is head j of order n (C-17)."""
+    x0, x1, x2 = ngram_contexts(tokens, offsets, hist)
+    R = int(rows_per_head)
+    ids = np.zeros((len(x0), 2 * heads), dtype=np.int64)
+    for t in range(len(x0)):
+        keys = ngram_keys(x0[t], x1[t], x2[t])
+        for n in range(2):
+            for j in range(heads):
+                ids[t, n * heads + j] = fold(keys[n] ^ ((j * HEAD_MIX) & _MASK64)) % R
+    return ids
+
+
+def row_ids(tokens, offsets, rows, hist, table) -> np.ndarray:
+    """The token's row IDs for the table's layout: [T][2] (C-4) or [T][16] (C-17)."""
+    if getattr(table, "format", "e4m3") == "heads":
+        return ngram_ids_heads(tokens, offsets, rows if np.isscalar(rows) else rows[0], hist,
+                               table.heads_per_order)
+    return ngram_ids(tokens, offsets, rows, hist)
+
+
+# --------------------------------------------------------------------------------------
 # C-5..C-7  gather, dequantise, sum the orders
 # --------------------------------------------------------------------------------------
 def dequantise(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
@@ -254,8 +299,12 @@ def table_rows(table, order: int, rows) -> np.ndarray:
 
 
 def embed(table, ids: np.ndarray) -> np.ndarray:
-    """e_t = deq(bigram row of t) + deq(trigram row of t)   (C-7)."""
+    """e_t = deq(bigram row of t) + deq(trigram row of t)   (C-7); for the
+    multi-head layout the 16 dequantised rows side by side in head order (C-17)."""
     ids = np.asarray(ids, dtype=np.int64)
+    if getattr(table, "format", "e4m3") == "heads":
+        return np.concatenate([dequantise(table.codes(h, ids[:, h]), table.scales(h, ids[:, h]))
+                               for h in range(ids.shape[1])], axis=1)
     return table_rows(table, 0, ids[:, 0]) + table_rows(table, 1, ids[:, 1])
 
 
@@ -271,6 +320,17 @@ class ArrayTable:
 
     def scales(self, order, rows):
         return self._scales[order][np.asarray(rows, dtype=np.int64)]
+
+
+class HeadsArrayTable(ArrayTable):
+    """A multi-head table held in arrays (C-17): codes uint8 [2 * heads][R'][D / (2 * heads)],
+    scales float32 [2 * heads][R']; ``codes(h, rows)`` reads sub-table h."""
+
+    format = "heads"
+
+    def __init__(self, codes: np.ndarray, scales: np.ndarray, heads_per_order: int = HEADS_PER_ORDER):
+        super().__init__(codes, scales)
+        self.heads_per_order = heads_per_order
 
 
 class Nvfp4ArrayTable(ArrayTable):
@@ -330,14 +390,17 @@ def ple_forward(tokens, offsets, hidden_bits, w_proj_bits, w_gate_bits, conv_w, 
     ``sample`` (optional): token indices whose outputs are wanted; only the
     rows those outputs depend on are gathered and projected.
 
-    Returns a dict: ``ids`` [T][2]; ``out`` float64 [len(sample) or T][H];
+    ``rows`` is the rows per order (C-4), or per head sub-table for a table of
+    the multi-head layout (C-17).
+
+    Returns a dict: ``ids`` [T][2] ([T][16] for C-17); ``out`` float64 [len(sample) or T][H];
     ``hist_out`` [S][2] and ``conv_out`` [S][3][H] (the state after each sequence).
     """
     tokens = np.asarray(tokens).reshape(-1)
     offsets = np.asarray(offsets, dtype=np.int64)
     T = tokens.shape[0]
     S = offsets.shape[0] - 1
-    ids = ngram_ids(tokens, offsets, rows, hist)
+    ids = row_ids(tokens, offsets, rows, hist, table)
     seq, pos = sequence_map(offsets, T)
     H = np.asarray(w_gate_bits).shape[0]
     conv0 = np.zeros((S, 3, H)) if conv_state is None else np.asarray(conv_state, np.float64)

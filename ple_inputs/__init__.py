@@ -162,6 +162,34 @@ class SynthTable:
 
 
 @dataclass
+class SynthHeadsTable:
+    """Host view of a synthetic table of the multi-head layout: 2 * heads sub-tables
+    of ``rows_per_head`` rows of ``head_dim`` FP8 codes, one fp32 scale per row.
+    Code k of row r of sub-table h has counter index ((h * R' + r) * head_dim + k),
+    so the bytes are those of the [2][heads * R'][head_dim] table the device filler
+    writes."""
+    seed: int
+    rows_per_head: int
+    head_dim: int
+    heads_per_order: int = 8
+    format: str = "heads"
+
+    def codes(self, head: int, rows) -> np.ndarray:
+        return table_codes(self.seed, self.rows_per_head, self.head_dim, head, rows)
+
+    def scales(self, head: int, rows) -> np.ndarray:
+        return table_scales(self.seed, self.rows_per_head, head, rows)
+
+    def full(self):
+        """codes [2 * heads][R'][head_dim], scales [2 * heads][R'] (small tables only)."""
+        r = np.arange(self.rows_per_head)
+        n = 2 * self.heads_per_order
+        if n * self.rows_per_head * self.head_dim > (1 << 28):
+            raise ValueError("table too large to materialise on the host")
+        return (np.stack([self.codes(h, r) for h in range(n)]), np.stack([self.scales(h, r) for h in range(n)]))
+
+
+@dataclass
 class SynthNvTable:
     """Host view of a synthetic NVFP4 table: packed codes [2][R][D/2], E4M3 block
     scales [2][R][D/16] and the same per-row fp32 scales as the FP8 table."""
@@ -254,6 +282,12 @@ class Workload:
     def table(self) -> SynthTable:
         return SynthTable(self.table_seed, self.rows_per_order, self.row_dim)
 
+    def heads_table(self, heads_per_order: int = 8) -> "SynthHeadsTable":
+        """The table of the multi-head layout: rows_per_order is then the rows per
+        head sub-table, and row_dim the width of e (2 * heads rows side by side)."""
+        return SynthHeadsTable(self.table_seed, self.rows_per_order, self.row_dim // (2 * heads_per_order),
+                               heads_per_order)
+
     def weights(self) -> Weights:
         return make_weights(self.table_seed, self.row_dim, self.hidden)
 
@@ -284,8 +318,17 @@ WORKLOADS = {
 }
 
 
+# The multi-head layout (16 sub-tables of 20,000,096 rows x 160 codes: the same
+# 51,200,245,760 bytes as the two-order table) and a small one for the tests.
+HEADS_FULL_ROWS = 20_000_096
+HEADS_WORKLOADS = {
+    "heads_tiny": Workload("heads_tiny", 1000, 512, 256, 128, table_seed=5, seed=5),
+    "heads_full": Workload("heads_full", FULL_VOCAB, HEADS_FULL_ROWS, FULL_DIM, FULL_DIM, FULL_TABLE_SEED, seed=6),
+}
+
+
 def workload(name: str) -> Workload:
-    return WORKLOADS[name]
+    return WORKLOADS[name] if name in WORKLOADS else HEADS_WORKLOADS[name]
 
 
 def prefill_batch(w: Workload, variant: int = 0, lengths=None, zipf: bool = True):

@@ -102,3 +102,50 @@ def test_wrong_subnormal_decode_caught(monkeypatch):
 def test_wrong_fold_shift_caught_by_brute_force(monkeypatch, shift):
     _patch(monkeypatch, "fold", lambda k: k ^ (k >> shift))
     assert _fails(pins.test_layer_matches_brute_force_tiny)
+
+
+# ------------------------------------------------------------------ multi-head layout (C-17)
+import tests.test_oracle_heads as heads_pins  # noqa: E402
+
+
+def _bad_heads(mix_of_head, key_of_head):
+    def bad(tokens, offsets, rows_per_head, hist=None, heads=OP.HEADS_PER_ORDER):
+        x0, x1, x2 = OP.ngram_contexts(tokens, offsets, hist)
+        ids = np.zeros((len(x0), 2 * heads), dtype=np.int64)
+        for t in range(len(x0)):
+            keys = OP.ngram_keys(x0[t], x1[t], x2[t])
+            for n in range(2):
+                for j in range(heads):
+                    k = keys[key_of_head(n)] ^ (mix_of_head(j) * OP.HEAD_MIX & OP._MASK64)
+                    ids[t, n * heads + j] = OP.fold(k) % int(rows_per_head)
+        return ids
+    return bad
+
+
+def test_heads_trigram_from_bigram_key_caught(monkeypatch):
+    _patch(monkeypatch, "ngram_ids_heads", _bad_heads(lambda j: j, lambda n: 0))
+    assert _fails(heads_pins.test_heads_dependence_structure)
+
+
+def test_heads_mix_offset_caught(monkeypatch):
+    _patch(monkeypatch, "ngram_ids_heads", _bad_heads(lambda j: j + 1, lambda n: n))
+    assert _fails(heads_pins.test_head_zero_is_the_two_order_row)
+
+
+def test_heads_without_mix_caught(monkeypatch):
+    _patch(monkeypatch, "ngram_ids_heads", _bad_heads(lambda j: 0, lambda n: n))
+    assert _fails(heads_pins.test_head_zero_is_the_two_order_row)
+
+
+def test_heads_reversed_concatenation_caught(monkeypatch):
+    orig = OP.embed
+
+    def bad(table, ids):
+        e = orig(table, ids)
+        if getattr(table, "format", "") != "heads":
+            return e
+        n = np.asarray(ids).shape[1]
+        return np.concatenate(np.split(e, n, axis=1)[::-1], axis=1)
+    _patch(monkeypatch, "embed", bad)
+    assert _fails(heads_pins.test_heads_embed_concatenates_in_head_order)
+    assert _fails(heads_pins.test_heads_layer_matches_brute_force)
