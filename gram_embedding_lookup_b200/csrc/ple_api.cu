@@ -155,9 +155,21 @@ bool wrong_device(const ple_handle* h) {
   return cudaGetDevice(&dev) != cudaSuccess || dev != h->device;
 }
 
+bool heads_layout(const ple_handle* h) { return h->cfg.table_format == PLE_TABLE_E4M3_HEADS; }
+int ids_per_token(const ple_config& c) { return c.table_format == PLE_TABLE_E4M3_HEADS ? 16 : 2; }
+
+// The kernel computing the row IDs (and, as the arguments ask, gate, metadata,
+// state and e) for the handle's table layout.
+cudaError_t launch_embed_for(const ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream);
+
 ple::TableRef table_ref(const ple_handle* h) {
   const bool nv = h->cfg.table_format == PLE_TABLE_NVFP4;
   return ple::TableRef{h->w.table, nv ? h->w.block_scales : nullptr, h->w.scales, nv ? 1 : 0};
+}
+
+cudaError_t launch_embed_for(const ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream) {
+  if (heads_layout(h)) return ple::launch_embed_heads(pa, table_ref(h), h->cfg.row_dim, e, stream);
+  return ple::launch_embed(pa, table_ref(h), h->cfg.row_dim, e, h->num_sms, stream);
 }
 
 void free_all(ple_handle* h) {
@@ -216,7 +228,7 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   const bool gather = !decode && gather_fused(h, T);
   h->prepared.valid = false;            // the scratch now holds this call's batch
   const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
-    return ple::launch_embed(pa, table_ref(h), c.row_dim, gather ? nullptr : h->e, h->num_sms, stream);
+    return launch_embed_for(h, pa, gather ? nullptr : h->e, stream);
   });
   if (st != PLE_OK) return st;
   return run_projection(h, T, S, uniform_q, hidden, out, dtype, state, dec_hist, dec_conv, tokens, n_commit, gather,
@@ -346,9 +358,16 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   if (config == nullptr || weights == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
   *out = nullptr;
   const ple_config& c = *config;
-  if ((c.table_format != PLE_TABLE_E4M3 && c.table_format != PLE_TABLE_NVFP4) || c.vocab <= 0 || c.hidden <= 0 || c.row_dim <= 0 || c.max_tokens <= 0 || c.max_seqs <= 0)
+  if ((c.table_format != PLE_TABLE_E4M3 && c.table_format != PLE_TABLE_NVFP4 &&
+       c.table_format != PLE_TABLE_E4M3_HEADS) ||
+      c.vocab <= 0 || c.hidden <= 0 || c.row_dim <= 0 || c.max_tokens <= 0 || c.max_seqs <= 0)
     return PLE_ERR_INVALID_ARG;
   if (c.hidden % 128 != 0 || c.row_dim % 64 != 0) return PLE_ERR_UNSUPPORTED;
+  if (c.table_format == PLE_TABLE_E4M3_HEADS) {
+    // 16 head rows of row_dim / 16 codes, a whole number of 16-byte chunks each
+    if (c.row_dim % 256 != 0) return PLE_ERR_UNSUPPORTED;
+    if (c.rows[1] != c.rows[0]) return PLE_ERR_INVALID_ARG;
+  }
   for (int n = 0; n < 2; ++n)
     if (c.rows[n] <= 0 || c.rows[n] >= (int64_t(1) << 31)) return PLE_ERR_INVALID_ARG;
   if (weights->table == nullptr || weights->scales == nullptr || weights->w_proj == nullptr ||
@@ -389,13 +408,15 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   const int64_t e_rows = std::max<int64_t>(c.max_tokens, 256);
   bool ok = cudaMalloc(&h->w16, static_cast<size_t>(c.row_dim) * c.hidden * 2) == cudaSuccess &&
             cudaMalloc(&h->e, static_cast<size_t>(e_rows) * c.row_dim * 2) == cudaSuccess &&
-            cudaMalloc(&h->ids, static_cast<size_t>(c.max_tokens) * 2 * 4) == cudaSuccess &&
+            cudaMalloc(&h->ids, static_cast<size_t>(c.max_tokens) * ids_per_token(c) * 4) == cudaSuccess &&
             cudaMalloc(&h->meta, static_cast<size_t>(c.max_tokens) * sizeof(ple::TokMeta)) == cudaSuccess &&
             cudaMalloc(&h->partial, static_cast<size_t>(cap) * 4) == cudaSuccess &&
             cudaMalloc(&h->conv0, static_cast<size_t>(c.max_seqs) * 3 * c.hidden * 4) == cudaSuccess &&
             cudaMalloc(&h->hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess &&
             cudaMalloc(&h->status, 8) == cudaSuccess;
-  h->decode_small = ok && ple::decode_small_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
+  // the single-kernel decode step gathers two-order rows; the multi-head layout takes the split-K steps
+  h->decode_small = ok && c.table_format != PLE_TABLE_E4M3_HEADS &&
+                    ple::decode_small_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
   if (h->decode_small) {
     ok = cudaMalloc(&h->decode_partial,
                     static_cast<size_t>(ple::decode_small_partial_elems(h->decode_plan, c.hidden)) * 4) == cudaSuccess &&
@@ -471,6 +492,8 @@ ple_status ple_ngram_ids(ple_handle* h, const int32_t* tokens, int32_t T, const 
   pa.ids = ids;
   pa.H = h->cfg.hidden;
   pa.status = h->status;
+  if (heads_layout(h))            // [T][16]: the row IDs alone (no metadata, no rows)
+    return run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return launch_embed_for(h, pa, nullptr, stream); });
   return run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_prepare(pa, stream); });
 }
 
@@ -481,6 +504,10 @@ ple_status ple_gather_rows(ple_handle* h, const int32_t* ids, int32_t T, void* e
   if (ids == nullptr || e_out == nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned(ids, 8) || !aligned(e_out, 16)) return PLE_ERR_ALIGN;
   const ple_config& c = h->cfg;
+  if (heads_layout(h))
+    return run_stage(h, PLE_STAGE_GATHER, stream, [&] {
+      return ple::launch_gather_heads(ids, T, table_ref(h), c.rows[0], c.row_dim, static_cast<__half*>(e_out), stream);
+    });
   return run_stage(h, PLE_STAGE_GATHER, stream, [&] {
     return ple::launch_gather(ids, T, table_ref(h), c.rows[0], c.rows[1], c.row_dim,
                               static_cast<__half*>(e_out), true, stream);
@@ -530,9 +557,7 @@ ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const in
     pa.meta = h->meta;
     pa.hist_new = h->hist_new;
     pa.status = h->status;
-    const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
-      return ple::launch_embed(pa, table_ref(h), c.row_dim, h->e, h->num_sms, stream);
-    });
+    const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return launch_embed_for(h, pa, h->e, stream); });
     if (st != PLE_OK) return st;
   }
   h->prepared.valid = true;

@@ -376,6 +376,25 @@ __device__ __forceinline__ void deq16(const uint4& a, const uint4& b, float s0, 
   o1.w = deq2(a.w, b.w, 16, s0, s1);
 }
 
+// One row on its own (the multi-head layout): e = fp16(a * s) for 16 codes,
+// the product in fp32, rounded to nearest even.
+__device__ __forceinline__ uint32_t deq2_one(uint32_t wa, int shift, float s) {
+  const float2 a = e4m3x2_cvt(wa >> shift);
+  const __half2 r = __floats2half2_rn(a.x * s, a.y * s);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void deq16_one(const uint4& a, float s, uint4& o0, uint4& o1) {
+  o0.x = deq2_one(a.x, 0, s);
+  o0.y = deq2_one(a.x, 16, s);
+  o0.z = deq2_one(a.y, 0, s);
+  o0.w = deq2_one(a.y, 16, s);
+  o1.x = deq2_one(a.z, 0, s);
+  o1.y = deq2_one(a.z, 16, s);
+  o1.z = deq2_one(a.w, 0, s);
+  o1.w = deq2_one(a.w, 16, s);
+}
+
 // NVFP4 rows: e = fp16(a' * s0 + b' * s1) for 16 elements of two rows, where a'
 // is an FP4 E2M1 code times its block's E4M3 scale. Codes come two per byte,
 // the low nibble first (8 bytes per 16 elements); one block scale covers the

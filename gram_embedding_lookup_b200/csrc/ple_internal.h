@@ -73,6 +73,17 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
 cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
                          cudaStream_t stream);
 
+// The multi-head layout (PLE_TABLE_E4M3_HEADS): one warp per token computes the
+// 16 head rows (ids [T][16]), the gate and metadata when a.meta is set, and
+// e[t] (the 16 dequantised rows side by side) when e is set; extra blocks do
+// the offsets check and the state work. a.rows0 is the rows per head sub-table.
+cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
+                               cudaStream_t stream);
+
+// Gather stage of the multi-head layout: ids [T][16] -> e [T][D].
+cudaError_t launch_gather_heads(const int32_t* ids, int32_t T, const TableRef& table, int64_t rows, int32_t D,
+                                __half* e, cudaStream_t stream);
+
 // Gate of a prepared batch: meta[t].g from hidden (one warp per token), plus the
 // conv-state snapshot when conv_in is set.
 cudaError_t launch_gate(const PrepareArgs& a, cudaStream_t stream);

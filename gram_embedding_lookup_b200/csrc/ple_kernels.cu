@@ -49,10 +49,11 @@ PrepareArgs with_magic(const PrepareArgs& in) {
   return a;
 }
 
-// Sequence, position, last-token flag and the two row IDs of token t (every
-// lane of the calling warp computes the same values; lane 0 reports errors).
-__device__ __forceinline__ void sequence_and_rows(const PrepareArgs& a, int t, int lane, int32_t& s, int32_t& pos,
-                                                  int32_t& last, int32_t& r0, int32_t& r1) {
+// Sequence, position, last-token flag and the bigram and trigram keys of token
+// t (every lane of the calling warp computes the same values; lane 0 reports
+// errors).
+__device__ __forceinline__ void sequence_and_keys(const PrepareArgs& a, int t, int lane, int32_t& s, int32_t& pos,
+                                                  int32_t& last, uint64_t& k2, uint64_t& k3) {
   if (a.uniform_q > 0) {
     s = t / a.uniform_q;
     pos = t - s * a.uniform_q;
@@ -83,8 +84,15 @@ __device__ __forceinline__ void sequence_and_rows(const PrepareArgs& a, int t, i
   };
   const uint64_t x1 = pos >= 1 ? context_of(a.tokens[t - 1]) : carried(1);
   const uint64_t x2 = pos >= 2 ? context_of(a.tokens[t - 2]) : (pos == 1 ? carried(1) : carried(2));
-  const uint64_t k2 = (x0 * kP0) ^ (x1 * kP1);
-  const uint64_t k3 = k2 ^ (x2 * kP2);
+  k2 = (x0 * kP0) ^ (x1 * kP1);
+  k3 = k2 ^ (x2 * kP2);
+}
+
+// ... and the two row IDs of token t.
+__device__ __forceinline__ void sequence_and_rows(const PrepareArgs& a, int t, int lane, int32_t& s, int32_t& pos,
+                                                  int32_t& last, int32_t& r0, int32_t& r1) {
+  uint64_t k2, k3;
+  sequence_and_keys(a, t, lane, s, pos, last, k2, k3);
   r0 = static_cast<int32_t>(mod_barrett(fold64(k2), static_cast<uint64_t>(a.rows0), a.magic0));
   r1 = static_cast<int32_t>(mod_barrett(fold64(k3), static_cast<uint64_t>(a.rows1), a.magic1));
 }
@@ -268,6 +276,104 @@ __global__ void __launch_bounds__(256) gate_kernel(const PrepareArgs a, int toke
   }
   const float g = gate_warp(hv, hrow, reinterpret_cast<const uint4*>(a.w_gate), H8, lane);
   if (lane == 0) a.meta[t].g = g;
+}
+
+// ------------------------------------------------------------------ multi-head layout
+// The row geometry of the SSD-stream model card ("Qwen3.8 Flash-Next NVFP4 -
+// SSD Stream", section "技术细节": 16 table lookups per token, 160-byte rows):
+// 8 hash heads per order; head j of order n reads sub-table 8n + j at row
+// fold(k_n ^ j * kHeadMix) mod rows (head 0 is the two-order row), and e is the
+// 16 dequantised rows side by side.
+constexpr uint64_t kHeadMix = 0xFF51AFD7ED558CCDull;   // odd constant separating the heads
+constexpr int kHeads = 16;
+
+// One warp per token. Lane l < 16 owns head l: its row ID and its row's scale;
+// the gather then spreads the token's D / 16 chunks of 16 codes over the lanes,
+// each taking its chunk's row and scale from the owning lane. Blocks past
+// token_blocks do the offsets check and the state work.
+__global__ void __launch_bounds__(256) embed_heads_kernel(const PrepareArgs a, const TableRef tab, int32_t D,
+                                                          __half* __restrict__ e, int token_blocks) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (static_cast<int>(blockIdx.x) >= token_blocks) {
+    state_blocks(a, blockIdx.x - token_blocks, gridDim.x - token_blocks, threadIdx.x, blockDim.x);
+    return;
+  }
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= a.T) return;
+  int32_t s, pos, last;
+  uint64_t k2, k3;
+  sequence_and_keys(a, t, lane, s, pos, last, k2, k3);
+  const int hh = lane & (kHeads - 1);
+  const uint64_t k = ((hh >> 3) ? k3 : k2) ^ (static_cast<uint64_t>(hh & 7) * kHeadMix);
+  const int32_t row = static_cast<int32_t>(mod_barrett(fold64(k), static_cast<uint64_t>(a.rows0), a.magic0));
+  if (lane < kHeads) a.ids[static_cast<int64_t>(t) * kHeads + lane] = row;
+  if (a.meta != nullptr) {
+    float g = 0.f;
+    if (a.hidden != nullptr) {
+      const int H8 = a.H / 8;
+      const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+      uint4 hv[kEmbedH4];
+#pragma unroll
+      for (int r = 0; r < kEmbedH4; ++r) {
+        const int j = lane + 32 * r;
+        if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+      }
+      g = gate_warp(hv, hrow, reinterpret_cast<const uint4*>(a.w_gate), H8, lane);
+    }
+    if (lane == 0) {
+      TokMeta m;
+      m.g = g;
+      m.seq = s;
+      m.pos = pos;
+      m.flags = last ? kFlagLast : 0;
+      a.meta[t] = m;
+    }
+  }
+  if (e == nullptr) return;
+  const int hd = D / kHeads;                 // codes per head row
+  const int cph = hd / 16;                   // 16-code chunks per head row
+  const int nch = D / 16;
+  const int64_t srow = static_cast<int64_t>(hh) * a.rows0 + row;
+  const float sc = __ldg(tab.scales + srow);
+  for (int base = 0; base < nch; base += 32) {
+    const int c = base + lane;
+    const int h = min(c, nch - 1) / cph;
+    const int r = __shfl_sync(0xffffffffu, row, h);
+    const float sh = __shfl_sync(0xffffffffu, sc, h);
+    if (c < nch) {
+      const int cc = c - h * cph;
+      const uint4 v = ld_stream_v4(tab.codes + (static_cast<int64_t>(h) * a.rows0 + r) * hd + cc * 16);
+      uint4 o0, o1;
+      deq16_one(v, sh, o0, o1);
+      uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D + c * 16);
+      dst[0] = o0;
+      dst[1] = o1;
+    }
+  }
+}
+
+// Gather stage of the multi-head layout: one thread per 16-code chunk.
+__global__ void __launch_bounds__(256) gather_heads_kernel(const int32_t* __restrict__ ids, int32_t T,
+                                                           const TableRef t, int64_t rows, int32_t D,
+                                                           __half* __restrict__ e) {
+  const int nch = D / 16;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= static_cast<int64_t>(T) * nch) return;
+  const int32_t tk = static_cast<int32_t>(g / nch);
+  const int c = static_cast<int>(g - static_cast<int64_t>(tk) * nch);
+  const int hd = D / kHeads;
+  const int cph = hd / 16;
+  const int h = c / cph;
+  const int cc = c - h * cph;
+  const uint32_t r = static_cast<uint32_t>(ids[static_cast<int64_t>(tk) * kHeads + h]) % static_cast<uint32_t>(rows);
+  const int64_t row = static_cast<int64_t>(h) * rows + r;
+  const uint4 v = ld_stream_v4(t.codes + row * hd + cc * 16);
+  uint4 o0, o1;
+  deq16_one(v, __ldg(t.scales + row), o0, o1);
+  uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(tk) * D + c * 16);
+  dst[0] = o0;
+  dst[1] = o1;
 }
 
 // ------------------------------------------------------------------ embed, pipelined
@@ -559,6 +665,25 @@ cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D,
     embed_pipe_kernel<true><<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, D, e);
   else
     embed_pipe_kernel<false><<<grid, kPipeThreads, 0, stream>>>(with_magic(a), table, D, e);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
+                               cudaStream_t stream) {
+  const int token_blocks = (a.T + 7) / 8;
+  int sblocks = 1;
+  if (a.conv_in != nullptr) {
+    const int64_t want = (static_cast<int64_t>(a.S) * 3 * a.H / 4 + 255) / 256;
+    sblocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
+  }
+  embed_heads_kernel<<<token_blocks + sblocks, 256, 0, stream>>>(with_magic(a), table, D, e, token_blocks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_heads(const int32_t* ids, int32_t T, const TableRef& table, int64_t rows, int32_t D,
+                                __half* e, cudaStream_t stream) {
+  const int64_t threads = static_cast<int64_t>(T) * (D / 16);
+  gather_heads_kernel<<<static_cast<int>((threads + 255) / 256), 256, 0, stream>>>(ids, T, table, rows, D, e);
   return cudaGetLastError();
 }
 

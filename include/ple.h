@@ -80,8 +80,18 @@ typedef enum { PLE_OUT_BF16 = 0, PLE_OUT_F32 = 1 } ple_out_dtype;
  *     table of NVFP4 codes and FP8 scales). The layout is not on the pages;
  *     this library reads it as FP4 E2M1 codes, two per byte with the low
  *     nibble first, one E4M3 block scale per 16 elements, and the same fp32
- *     scale per row as the E4M3 table. */
-typedef enum { PLE_TABLE_E4M3 = 0, PLE_TABLE_NVFP4 = 1 } ple_table_format;
+ *     scale per row as the E4M3 table.
+ *   PLE_TABLE_E4M3_HEADS: the row geometry of the SSD-stream model card
+ *     ("Qwen3.8 Flash-Next NVFP4 - SSD Stream", section "技术细节": 16 table
+ *     lookups per token, 160-byte FP8 rows). 16 sub-tables (8 hash heads per
+ *     order) of rows[0] rows of row_dim/16 E4M3 codes, one fp32 scale per row;
+ *     head j of order n (sub-table 8n + j) takes row
+ *     (k ^ (k >> 32)) mod rows[0] with k = k_n ^ (j * 0xFF51AFD7ED558CCD) mod 2^64
+ *     (k_n the order's key below; head 0 is the two-order row), and e is the
+ *     16 dequantised rows side by side in sub-table order. rows[1] must equal
+ *     rows[0]; row_dim % 256 == 0. The same 51,200,245,760 bytes hold
+ *     16 x 20,000,096 rows of 160. Row IDs are [T][16] for this format. */
+typedef enum { PLE_TABLE_E4M3 = 0, PLE_TABLE_NVFP4 = 1, PLE_TABLE_E4M3_HEADS = 2 } ple_table_format;
 
 /* Sizes fixed at creation. hidden % 128 == 0, row_dim % 64 == 0,
  * 0 < rows[n] < 2^31. max_tokens bounds T of every call (and B*q of a decode
@@ -104,7 +114,9 @@ typedef struct {
                                 rows[0] == rows[1]).
                                 NVFP4: packed E2M1 codes, element 2i in the low nibble of
                                 byte i of the row; row r of sub-table n at byte offset
-                                (n*rows[0] + r)*row_dim/2. 16-byte aligned */
+                                (n*rows[0] + r)*row_dim/2.
+                                E4M3_HEADS: sub-table h (0..15), row r at byte offset
+                                (h*rows[0] + r)*(row_dim/16). 16-byte aligned */
   const float* scales;       /* fp32 per-row scales; sub-table n, row r at n*rows[0] + r */
   const void* w_proj;        /* bf16 [row_dim][hidden], row-major */
   const void* w_gate;        /* bf16 [hidden] */
@@ -135,15 +147,16 @@ ple_status ple_destroy(ple_handle* handle);
 /* N-gram row IDs only. tokens int32 [T]; offsets int32 [S+1] with
  * offsets[0] = 0, offsets[S] = T, non-decreasing (sequence s covers
  * [offsets[s], offsets[s+1])); hist int32 [S][2] or NULL (all absent);
- * ids int32 [T][2] receives (bigram row, trigram row), each in [0, rows[n]). */
+ * ids int32 [T][2] receives (bigram row, trigram row), each in [0, rows[n]);
+ * for PLE_TABLE_E4M3_HEADS, ids int32 [T][16] receives the 16 head rows. */
 ple_status ple_ngram_ids(ple_handle* handle, const int32_t* tokens, int32_t T,
                          const int32_t* offsets, int32_t S, const int32_t* hist,
                          int32_t* ids, cudaStream_t stream);
 
 /* The gather stage alone: e_out fp16 [T][row_dim] receives e_t (see top of
- * file, in the handle's table format) for the given row IDs int32 [T][2]. IDs
- * must be in range (the call reduces them mod rows[n] so that no access
- * leaves the table). */
+ * file, in the handle's table format) for the given row IDs int32 [T][2]
+ * ([T][16] for PLE_TABLE_E4M3_HEADS). IDs must be in range (the call reduces
+ * them mod rows[n] so that no access leaves the table). */
 ple_status ple_gather_rows(ple_handle* handle, const int32_t* ids, int32_t T,
                            void* e_out, cudaStream_t stream);
 

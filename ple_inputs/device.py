@@ -28,7 +28,9 @@ class DeviceLayer:
     """A workload's table and weights on the current device, plus a libple handle.
 
     table_format ple.PLE_TABLE_NVFP4 builds the synthetic NVFP4 table instead
-    (packed codes in ``table``, E4M3 block scales in ``block_scales``)."""
+    (packed codes in ``table``, E4M3 block scales in ``block_scales``);
+    ple.PLE_TABLE_E4M3_HEADS builds the multi-head table (16 sub-tables of
+    rows_per_order rows of row_dim / 16 codes)."""
 
     def __init__(self, w: Workload, max_tokens: int, max_seqs: int, weights=None, stream=None,
                  table_format: int = 0):
@@ -36,8 +38,15 @@ class DeviceLayer:
         self.table_format = table_format
         R, D, H = w.rows_per_order, w.row_dim, w.hidden
         s = torch.cuda.current_stream() if stream is None else stream
-        self.scales = torch.empty(2 * R, dtype=torch.float32, device="cuda")
-        if table_format == ple.PLE_TABLE_NVFP4:
+        heads = table_format == ple.PLE_TABLE_E4M3_HEADS
+        self.scales = torch.empty((16 if heads else 2) * R, dtype=torch.float32, device="cuda")
+        if heads:
+            # 16 sub-tables of R rows x D/16 codes: the bytes of a [2][8R][D/16] table
+            self.table = torch.empty(R * D, dtype=torch.uint8, device="cuda")
+            self.block_scales = None
+            fill_table_device(self.table.data_ptr(), self.scales.data_ptr(), 8 * R, D // 16, w.table_seed,
+                              s.cuda_stream)
+        elif table_format == ple.PLE_TABLE_NVFP4:
             self.table = torch.empty(2 * R * D // 2, dtype=torch.uint8, device="cuda")
             self.block_scales = torch.empty(2 * R * D // 16, dtype=torch.uint8, device="cuda")
             fill_nv_table_device(self.table.data_ptr(), self.block_scales.data_ptr(), self.scales.data_ptr(), R, D,

@@ -73,8 +73,14 @@ def test_null_arguments_rejected_on_host(libple):
     wts.table = 17
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 3  # misaligned
     wts.table = 16
-    cfg.table_format = 2                          # no such format
+    cfg.table_format = 3                          # no such format
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
+    cfg.table_format = ple.PLE_TABLE_E4M3_HEADS   # 16 head rows need row_dim % 256 == 0 ...
+    assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 8
+    cfg.row_dim = 256
+    cfg.rows[1] = 17                              # ... and equal rows per head sub-table
+    assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
+    cfg.row_dim, cfg.rows[1] = 64, 16
     cfg.table_format = ple.PLE_TABLE_NVFP4        # NVFP4 needs block scales
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
     wts.block_scales = 24                         # ... 16-byte aligned
