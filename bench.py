@@ -410,6 +410,7 @@ def main():
         line["mtp"] = mtp_bench(ctx, layer, stream)
         line["long_context"] = long_bench(ctx, layer, stream)
         line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks)
+        line["heads"] = heads_bench(ctx, sets, stream, peaks)
         line["prepared"] = prepared_bench(ctx, layer, sets, stream)
         line["gather_fused"] = gather_fused_bench(ctx, layer, sets, stream, peaks)
 
@@ -642,6 +643,71 @@ def prepared_bench(ctx, layer, sets, stream, steps=200):
             "after_hidden_ready_ms_saved": t_whole - t_rest, "device_status": int(status),
             "note": "ple_prepare needs only the tokens; ple_forward_prepared (gate, projection, conv, residual) "
                     "is the part that waits for the hidden states"}
+
+
+def heads_bench(ctx, sets, stream, peaks, steps=300):
+    """The multi-head row layout (PLE_TABLE_E4M3_HEADS: 16 lookups of 160-byte rows
+    per token, 16 sub-tables of 20,000,096 rows, the same 51.2 GB): the headline
+    prefill batches and the 8 x 1 decode workload (a split-K step on this layout)."""
+    torch, ple, pi = ctx["torch"], ctx["ple"], ctx["pi"]
+    from ple_inputs.device import DeviceLayer
+    w = pi.workload("heads_full")
+    R, D, H = w.rows_per_order, w.row_dim, w.hidden
+    need = R * D + 16 * R * 4
+    free, _ = torch.cuda.mem_get_info()
+    if free < need + (4 << 30):
+        return {"skipped": f"needs {need / 1e9:.1f} GB free for the multi-head table, {free / 1e9:.1f} GB free"}
+    layer = DeviceLayer(w, max_tokens=16384, max_seqs=64, table_format=ple.PLE_TABLE_E4M3_HEADS)
+    h = layer.handle
+    tokens, hidden, hist, conv = pi.decode_batch(pi.workload("decode"))
+    B, q = tokens.shape
+    tk = torch.from_numpy(tokens).cuda()
+    hd = ctx["bf16_tensor"](hidden)
+    hs = torch.from_numpy(hist.astype(np.int32)).cuda()
+    cs = torch.from_numpy(conv).cuda()
+    out = torch.empty(B * q, H, dtype=torch.bfloat16, device="cuda")
+
+    def dstep(i):
+        ple.ple_decode_step(h, tk, B, q, hd, out, ple.PLE_OUT_BF16, hs, cs, None, stream)
+
+    for i in range(5):
+        dstep(i)
+    n_dec = 500
+    d_ms = timed(ctx, stream, dstep, n_dec)
+
+    def step(i):
+        s = sets[i % len(sets)]
+        ple.ple_forward(h, s["tokens"], s["T"], s["offsets"], s["S"], s["hidden"], s["out"], ple.PLE_OUT_BF16,
+                        None, stream)
+
+    for i in range(5):
+        step(i)
+    ms = timed(ctx, stream, step, steps)
+    ple.ple_set_profiling(h, True)
+    ple.ple_get_stage_times(h)
+    for i in range(min(steps, 100)):
+        step(i)
+    torch.cuda.synchronize()
+    stage = ple.ple_get_stage_times(h)
+    ple.ple_set_profiling(h, False)
+    T = sets[0]["T"]
+    e_ms, e_n = stage["prepare"]
+    e_s = e_ms / 1e3 / max(e_n, 1)
+    row_bytes = D + 16 * 4                        # 16 rows of D / 16 codes and their scales
+    embed_bytes = T * (2 * H + row_bytes + 2 * D + 16 * 4 + 16 + 4)   # h, rows in; e, ids, meta out; tokens
+    g_ms, g_n = stage["gemm"]
+    status = ple.ple_get_error(h)
+    layer.close()
+    world = ctx["world"]
+    return {"workload": "full-scale prefill (the headline batches) and 8 x 1 decode on the multi-head table "
+                        "(16 x 20,000,096 rows x 160 codes)",
+            "table_bytes": int(need), "value": T * world * steps / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms / steps, "stage_ms_per_launch": {"embed": e_s * 1e3, "gemm": g_ms / max(g_n, 1)},
+            "embed_roofline": {"bound": "hbm", "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"],
+                               "algorithmic_bytes_per_launch": embed_bytes},
+            "gathered_row_gbs": T * row_bytes / e_s / 1e9,
+            "decode_us_per_step": d_ms / n_dec * 1e3, "device_status": int(status)}
 
 
 def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
