@@ -453,31 +453,41 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     }
   } else {
     // ---- consumers: two tokens of every batch, lane-parallel within the warp.
-    //      A token's hidden row does not depend on its row IDs, so the loads of
-    //      the first one are issued before the wait for the batch (the first
-    //      time, the conv-state snapshot, the new token history and the offsets
-    //      check run meanwhile). Every warp waits for every batch, so that its
-    //      release of a slot always counts in the slot's current round.
+    //      A token's hidden row does not depend on its row IDs, so its loads
+    //      are issued right after the warp's previous gate, before the wait for
+    //      the token's batch (the first time, the conv-state snapshot, the new
+    //      token history and the offsets check run meanwhile). Every warp waits
+    //      for every batch, so that its release of a slot always counts in the
+    //      slot's current round.
     const int cw = warp - 1;
     const int H8 = a.H / 8;
     const int D16 = D / 16;
     const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+    const bool with_gate = a.hidden != nullptr;       // null: ple_prepare, the gate comes later
+    const bool with_rows = e != nullptr;              // null: the projection gathers the rows itself
+    // hv holds the hidden row of the warp's next token; it is loaded as soon as
+    // the previous token's gate has used it, so the load runs under that
+    // token's dequantisation and stores (and, for a batch's first token, under
+    // the wait for the batch's row IDs)
+    uint4 hv[kEmbedH4];
+    auto load_hidden = [&](int t) {
+      const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+#pragma unroll
+      for (int r = 0; r < kEmbedH4; ++r) {
+        const int j = lane + 32 * r;
+        if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+      }
+    };
+    // the k-th token (in the CTA's range) this warp handles after token k
+    auto next_token = [&](int b, int half) {
+      return half + 1 < kPipeBatch / kPipeConsumers ? b * kPipeBatch + cw + kPipeConsumers * (half + 1)
+                                                    : (b + 1) * kPipeBatch + cw;
+    };
+    if (with_gate && cw < n) load_hidden(t0 + cw);
     bool state_done = false;
     for (int b = 0; b < nb; ++b) {
       const int slot = b % kPipeBatches, round = b / kPipeBatches;
-      uint4 hv[kEmbedH4];
       RowChunk<NV> ca[kEmbedD16], cb[kEmbedD16];
-      auto load_hidden = [&](int t) {
-        const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
-#pragma unroll
-        for (int r = 0; r < kEmbedH4; ++r) {
-          const int j = lane + 32 * r;
-          if (j < H8) hv[r] = ld_stream_v4(hrow + j);
-        }
-      };
-      const bool with_gate = a.hidden != nullptr;     // null: ple_prepare, the gate comes later
-      const bool with_rows = e != nullptr;            // null: the projection gathers the rows itself
-      if (with_gate && b * kPipeBatch + cw < n) load_hidden(t0 + b * kPipeBatch + cw);
       if (!state_done) {
         state_blocks(a, blockIdx.x, gridDim.x, threadIdx.x - 32, blockDim.x - 32);
         state_done = true;
@@ -493,7 +503,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         if (k >= n) break;                                   // warp-uniform
         const int t = t0 + k;
         const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
-        if (with_gate && half > 0) load_hidden(t);
         const PipeTok pt = sm.tok[slot][i];
         const int64_t ra = pt.r0, rb = a.rows0 + pt.r1;
 #pragma unroll
@@ -507,6 +516,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const float s0 = with_rows ? __ldg(tab.scales + ra) : 0.f;
         const float s1 = with_rows ? __ldg(tab.scales + rb) : 0.f;
         const float g = with_gate ? gate_warp(hv, hrow, wg, H8, lane) : 0.f;
+        const int kn = next_token(b, half);
+        if (with_gate && kn < n) load_hidden(t0 + kn);
         if (lane == 0) {
           TokMeta m;
           m.g = g;
