@@ -17,7 +17,7 @@ __all__ = [
     "ple_ngram_ids", "ple_gather_rows", "ple_forward", "ple_prepare", "ple_forward_prepared", "ple_decode_step",
     "ple_get_error",
     "ple_status_string", "ple_set_profiling", "ple_get_stage_times", "ple_set_forward_path",
-    "ple_launch_count", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32",
+    "ple_launch_count", "ple_wait_selftest", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32",
     "PLE_TABLE_E4M3", "PLE_TABLE_NVFP4", "PLE_TABLE_E4M3_HEADS", "STATUS",
     "STAGES", "LIB_PATH",
 ]
@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
             "ple_get_stage_times": ([_VP, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int64)], _I32),
             "ple_set_forward_path": ([_VP, _I32], _I32),
             "ple_launch_count": ([_VP], ctypes.c_int64),
+            "ple_wait_selftest": ([_VP, ctypes.c_int64, _VP], _I32),
             "ple_embed_static": ([_VP, _I32, _VP, _I32, _VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, _I32, _I32,
                                   _VP, _VP, _VP], _I32),
         }
@@ -198,6 +199,12 @@ def ple_set_forward_path(handle, path: int) -> None:
 
 def ple_launch_count(handle) -> int:
     return int(lib().ple_launch_count(handle))
+
+
+def ple_wait_selftest(handle, limit_cycles: int, stream=None) -> None:
+    """Run one bounded device wait that nothing completes (see include/ple.h); the
+    handle's status then reads PLE_ERR_TIMEOUT."""
+    _check(lib().ple_wait_selftest(handle, int(limit_cycles), _stream(stream)), "ple_wait_selftest")
 
 
 def ple_embed_static(tokens, T, offsets, S, hist, table, scales, rows0, rows1, row_dim, vocab, e_out,

@@ -693,4 +693,10 @@ ple_status ple_set_forward_path(ple_handle* h, int32_t path) {
 
 int64_t ple_launch_count(const ple_handle* h) { return h ? h->launches : -1; }
 
+ple_status ple_wait_selftest(ple_handle* h, int64_t limit_cycles, cudaStream_t stream) {
+  if (h == nullptr || limit_cycles <= 0 || limit_cycles > ple::kWaitLimitCycles) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
+  return ple::launch_wait_selftest(h->status, limit_cycles, stream) == cudaSuccess ? PLE_OK : PLE_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -86,13 +86,14 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 // Waits for the phase with the given parity to complete. Returns false if the
-// wait ran out (the caller records PLE_ERR_TIMEOUT and abandons its work).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// wait ran out after `limit` SM cycles (the caller records PLE_ERR_TIMEOUT and
+// abandons its work).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long start = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - start > kWaitLimitCycles) return false;
+    if (clock64() - start > limit) return false;
   }
 }
 

@@ -84,6 +84,10 @@ cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int3
 cudaError_t launch_gather_heads(const int32_t* ids, int32_t T, const TableRef& table, int64_t rows, int32_t D,
                                 __half* e, cudaStream_t stream);
 
+// Failure-detection self-test: one bounded mbarrier wait that runs out after
+// limit_cycles and records PLE_ERR_TIMEOUT in *status.
+cudaError_t launch_wait_selftest(int32_t* status, long long limit_cycles, cudaStream_t stream);
+
 // Gate of a prepared batch: meta[t].g from hidden (one warp per token), plus the
 // conv-state snapshot when conv_in is set.
 cudaError_t launch_gate(const PrepareArgs& a, cudaStream_t stream);

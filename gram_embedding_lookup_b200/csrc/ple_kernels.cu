@@ -550,6 +550,20 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ bounded-wait self-test
+// One warp waits, through the same bounded wait the library's kernels use, on
+// an mbarrier that expects one arrival nobody makes. The wait runs out after
+// `limit` cycles; the kernel then records PLE_ERR_TIMEOUT and returns.
+__global__ void wait_selftest_kernel(int32_t* status, long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (!mbar_wait(smem_u32(&bar), 0, limit) && threadIdx.x == 0) set_status(status, PLE_ERR_TIMEOUT);
+}
+
 // ------------------------------------------------------------------ W_proj conversion
 __global__ void convert_w_kernel(const __nv_bfloat16* __restrict__ w, int32_t D, int32_t H,
                                  __half* __restrict__ w16, int32_t* bad) {
@@ -695,6 +709,11 @@ cudaError_t launch_gather_heads(const int32_t* ids, int32_t T, const TableRef& t
                                 __half* e, cudaStream_t stream) {
   const int64_t threads = static_cast<int64_t>(T) * (D / 16);
   gather_heads_kernel<<<static_cast<int>((threads + 255) / 256), 256, 0, stream>>>(ids, T, table, rows, D, e);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(int32_t* status, long long limit_cycles, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_cycles);
   return cudaGetLastError();
 }
 

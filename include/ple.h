@@ -286,6 +286,16 @@ ple_status ple_set_forward_path(ple_handle* handle, int32_t path);
 /* Total number of kernels the handle has launched since creation. */
 int64_t ple_launch_count(const ple_handle* handle);
 
+/* Failure-detection self-test. Every wait inside the library's kernels is
+ * bounded: when one runs out, the kernel records PLE_ERR_TIMEOUT in the
+ * handle's sticky status, abandons its work and returns, so the CUDA context
+ * stays usable and ple_get_error reports the failure. This call exercises that
+ * path on demand: it launches one small kernel (stream-ordered) whose wait on
+ * an mbarrier that nothing completes runs out after limit_cycles SM cycles
+ * (0 < limit_cycles <= 2e9, about one second at B200 clocks). Returns
+ * PLE_ERR_INVALID_ARG for a null handle or a limit out of range. */
+ple_status ple_wait_selftest(ple_handle* handle, int64_t limit_cycles, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

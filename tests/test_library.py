@@ -92,6 +92,7 @@ def test_null_arguments_rejected_on_host(libple):
     assert libple.ple_gather_rows(None, None, 0, None, None) == 1
     assert libple.ple_get_error(None) == 1
     assert libple.ple_launch_count(None) == -1
+    assert libple.ple_wait_selftest(None, 1000, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
