@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--sets", type=int, default=3, help="rotating input sets")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e, decode and clocks measurements")
+    ap.add_argument("--extras", default="e2e,decode,mtp,long,nvfp4,heads,prepared,gather_fused",
+                    help="comma-separated extra lines to measure (for profiling one of them alone)")
     ap.add_argument("--ref-tokens", type=int, default=512, help="tokens per reference-arm step")
     ap.add_argument("--path", type=int, default=0,
                     help="forward path of the timed prefill steps (ple_set_forward_path; 0 = automatic, "
@@ -405,14 +407,23 @@ def main():
     line["gather_roofline"] = gather_bench(ctx, layer, sets, stream, peaks)
 
     if not args.no_extras:
-        line["e2e"] = e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier)
-        line["decode"] = decode_bench(ctx, layer, stream)
-        line["mtp"] = mtp_bench(ctx, layer, stream)
-        line["long_context"] = long_bench(ctx, layer, stream)
-        line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks)
-        line["heads"] = heads_bench(ctx, sets, stream, peaks)
-        line["prepared"] = prepared_bench(ctx, layer, sets, stream)
-        line["gather_fused"] = gather_fused_bench(ctx, layer, sets, stream, peaks)
+        want = set(args.extras.split(","))
+        if "e2e" in want:
+            line["e2e"] = e2e_prefill(args, ple, h, sets, stream, world, max_over_ranks, barrier)
+        if "decode" in want:
+            line["decode"] = decode_bench(ctx, layer, stream)
+        if "mtp" in want:
+            line["mtp"] = mtp_bench(ctx, layer, stream)
+        if "long" in want:
+            line["long_context"] = long_bench(ctx, layer, stream)
+        if "nvfp4" in want:
+            line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks)
+        if "heads" in want:
+            line["heads"] = heads_bench(ctx, sets, stream, peaks)
+        if "prepared" in want:
+            line["prepared"] = prepared_bench(ctx, layer, sets, stream)
+        if "gather_fused" in want:
+            line["gather_fused"] = gather_fused_bench(ctx, layer, sets, stream, peaks)
 
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         tokens, offsets, hidden = sets[0]["host"]
