@@ -4,9 +4,10 @@ graphs) replays to the same bits as eager launches.
 Every call is stream-ordered and does its host work (argument checks, tensor
 maps, launch planning) at capture time; the kernels keep no state between
 launches that a replay could see stale (the single-kernel decode step resets
-its tile counters itself). Three forms are captured: a decode step (one
-kernel under programmatic dependent launch), a prefill on SM-pair tiles and a
-small forward on the split-K path (projection then combine).
+its tile counters itself). Four forms are captured: a decode step (one
+kernel under programmatic dependent launch), an MTP-style decode step on the
+split-K path, a prefill on SM-pair tiles and a small forward on the split-K
+path (projection then combine).
 """
 import numpy as np
 import pytest
@@ -102,3 +103,41 @@ def test_forward_graph_replay_matches_eager(mid_layer, lengths, path):  # noqa: 
         del graph
     finally:
         ple.ple_set_forward_path(L.handle, 0)
+
+
+def test_split_decode_step_graph_replay_matches_eager(mid_layer):  # noqa: F811
+    """A decode step of more than 16 tokens (an MTP-style step with n_commit) takes
+    the split-K path: embed, projection and combine, three kernels chained by
+    programmatic dependent launch. Captured once, it replays to the same bits."""
+    from ple_inputs.device import bf16_tensor
+    L = mid_layer
+    B, q = 24, 3
+    rng = np.random.default_rng(32)
+    tok = rng.integers(0, MID.vocab, (B, q)).astype(np.int32)
+    hid = pi.hidden_bf16(rng, B * q, MID.hidden)
+    hist0 = rng.integers(0, MID.vocab, (B, 2)).astype(np.int32)
+    conv0 = rng.standard_normal((B, 3, MID.hidden)).astype(np.float32)
+    nc = _i32(rng.integers(1, q + 1, B))
+    hs, cs = _i32(hist0), torch.from_numpy(conv0).cuda()
+    ref = torch.empty(B * q, MID.hidden, dtype=torch.float32, device="cuda")
+    n0 = ple.ple_launch_count(L.handle)
+    ple.ple_decode_step(L.handle, _i32(tok), B, q, bf16_tensor(hid), ref, 1, hs, cs, nc)
+    torch.cuda.synchronize()
+    assert ple.ple_get_error(L.handle) == 0
+    assert ple.ple_launch_count(L.handle) - n0 == 3
+    s_tok, s_hid = _i32(tok), bf16_tensor(hid)
+    s_hs, s_cs = _i32(hist0), torch.from_numpy(conv0).cuda()
+    out = torch.empty_like(ref)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        ple.ple_decode_step(L.handle, s_tok, B, q, s_hid, out, 1, s_hs, s_cs, nc, torch.cuda.current_stream().cuda_stream)
+    s_hs.copy_(_i32(hist0))
+    s_cs.copy_(torch.from_numpy(conv0).cuda())
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert torch.equal(s_hs, hs) and torch.equal(s_cs, cs)
+    assert ple.ple_get_error(L.handle) == 0
+    del graph
