@@ -414,9 +414,7 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
             cudaMalloc(&h->conv0, static_cast<size_t>(c.max_seqs) * 3 * c.hidden * 4) == cudaSuccess &&
             cudaMalloc(&h->hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess &&
             cudaMalloc(&h->status, 8) == cudaSuccess;
-  // the single-kernel decode step gathers two-order rows; the multi-head layout takes the split-K steps
-  h->decode_small = ok && c.table_format != PLE_TABLE_E4M3_HEADS &&
-                    ple::decode_small_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
+  h->decode_small = ok && ple::decode_small_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
   if (h->decode_small) {
     ok = cudaMalloc(&h->decode_partial,
                     static_cast<size_t>(ple::decode_small_partial_elems(h->decode_plan, c.hidden)) * 4) == cudaSuccess &&
@@ -629,6 +627,7 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
     a.blocks = h->w.block_scales;
     a.scales = h->w.scales;
     a.nvfp4 = c.table_format == PLE_TABLE_NVFP4 ? 1 : 0;
+    a.heads = c.table_format == PLE_TABLE_E4M3_HEADS ? 1 : 0;
     a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
     a.conv_w = h->w.conv_w;
     a.hidden = static_cast<const __nv_bfloat16*>(hidden);

@@ -16,7 +16,9 @@
 //     this fetch overlaps the previous step's tail;
 //   - every CTA computes the T row-ID pairs and gates and gathers and
 //     dequantises the T row pairs into shared memory (the same rounding to fp16
-//     as the prefill path), all warps sharing the loads;
+//     as the prefill path), all warps sharing the loads; for the multi-head
+//     layout, 16 head rows per token (a thread per token and head hashes),
+//     dequantised row by row and laid side by side;
 //   - the 16 x T x 64 products of a unit run on the tensor cores with mma.sync
 //     m16n8k16 (fp16 inputs, fp32 accumulation), the W_proj operand read with
 //     ldmatrix from the 128-byte-swizzled TMA tiles;
@@ -55,6 +57,8 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr uint64_t kQ0 = 0x9E3779B97F4A7C15ull;
 constexpr uint64_t kQ1 = 0xC2B2AE3D27D4EB4Full;
 constexpr uint64_t kQ2 = 0x165667B19E3779F9ull;
+constexpr uint64_t kHeadMix = 0xFF51AFD7ED558CCDull;   // separates the 8 hash heads of an order
+constexpr int kHeads = 16;                             // multi-head layout: 2 orders x 8 heads
 
 __device__ __forceinline__ uint64_t ctx_of(int32_t tok) {
   return static_cast<uint64_t>(static_cast<uint32_t>(tok)) + 1ull;
@@ -99,6 +103,7 @@ struct __align__(16) DecodeSmem {
   float res[kMaxTok][kChan];                           // and its residual (hidden)
   float gacc[kMaxTok];                                 // gate pre-activations
   int64_t rid[kMaxTok][2];                             // row IDs (into the stacked table)
+  int32_t rid16[kMaxTok][kHeads];                      // multi-head layout: row of each head
   uint64_t bar[kMaxUnits];                             // one mbarrier per W_proj unit
   int32_t fin[kMaxLocalTiles];
   int32_t last;
@@ -113,9 +118,12 @@ size_t smem_bytes(int units, int32_t D, int32_t H) {
          static_cast<size_t>(kMaxTok) * (D + 8) * sizeof(__half) + static_cast<size_t>(H) * sizeof(__nv_bfloat16);
 }
 
-template <bool NV>
+// FMT: 0 = E4M3 rows (two orders), 1 = NVFP4 rows, 2 = the multi-head E4M3 layout.
+template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecodeSmallArgs a) {
+  constexpr bool NV = FMT == 1;
+  constexpr bool HEADS = FMT == 2;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
@@ -238,11 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     uint4 hv[kGateBatch];
     gate_load(hv, 0);
-    if (threadIdx.x < T) {
-      const int t = threadIdx.x;
+    if (threadIdx.x < (HEADS ? T * kHeads : T)) {
+      const int t = HEADS ? threadIdx.x / kHeads : threadIdx.x;
+      const int hh = HEADS ? threadIdx.x % kHeads : 0;
       const int b = t / a.q, i = t - b * a.q;
       const int32_t tok = a.tokens[t];
-      if (blockIdx.x == 0 && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
+      if (blockIdx.x == 0 && hh == 0 && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
       const int32_t h0 = a.hist[2 * b], h1 = a.hist[2 * b + 1];
       auto carried = [](int32_t h) -> uint64_t { return h < 0 ? 0ull : ctx_of(h); };
       const uint64_t x0 = ctx_of(tok);
@@ -250,16 +259,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t x2 = i >= 2 ? ctx_of(a.tokens[t - 2]) : (i == 1 ? carried(h1) : carried(h0));
       const uint64_t k2 = (x0 * kQ0) ^ (x1 * kQ1);
       const uint64_t k3 = k2 ^ (x2 * kQ2);
-      const int64_t r0 = static_cast<int64_t>(mod_barrett(k2 ^ (k2 >> 32), a.rows0, a.magic0));
-      const int64_t r1 = a.rows0 + static_cast<int64_t>(mod_barrett(k3 ^ (k3 >> 32), a.rows1, a.magic1));
-      sm->rid[t][0] = r0;
-      sm->rid[t][1] = r1;
+      if constexpr (HEADS) {
+        // head hh of order hh / 8 reads sub-table hh: fold(k_n ^ (hh % 8) * kHeadMix) mod rows
+        const uint64_t k = ((hh >> 3) ? k3 : k2) ^ (static_cast<uint64_t>(hh & 7) * kHeadMix);
+        sm->rid16[t][hh] = static_cast<int32_t>(mod_barrett(k ^ (k >> 32), a.rows0, a.magic0));
+      } else {
+        const int64_t r0 = static_cast<int64_t>(mod_barrett(k2 ^ (k2 >> 32), a.rows0, a.magic0));
+        const int64_t r1 = a.rows0 + static_cast<int64_t>(mod_barrett(k3 ^ (k3 >> 32), a.rows1, a.magic1));
+        sm->rid[t][0] = r0;
+        sm->rid[t][1] = r1;
+      }
     }
     gate_use(hv, 0);
   }
   __syncthreads();                                          // row IDs ready
   const int row_segs = (T * nsr + kWarps - 1) / kWarps;     // per warp
-  for (int first = 0; first < row_segs; first += kRowBatch) {
+  if constexpr (HEADS) {
+    // chunk j of a token (16 codes) comes from head row j / (chunks per head)
+    const int hd = a.D / kHeads, cph = hd / 16;
+    for (int first = 0; first < row_segs; first += kRowBatch) {
+      uint4 xh[kRowBatch];
+      float sh[kRowBatch];
+#pragma unroll
+      for (int r = 0; r < kRowBatch; ++r) {
+        const int s = warp + kWarps * (first + r);
+        const int t = s / nsr, j = (s - t * nsr) * 32 + lane;
+        if (t < T && j < dv16) {
+          const int h = j / cph;
+          const int64_t row = static_cast<int64_t>(h) * a.rows0 + sm->rid16[t][h];
+          xh[r] = ld_stream_v4(a.table + row * hd + (j - h * cph) * 16);
+          sh[r] = __ldg(a.scales + row);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kRowBatch; ++r) {
+        const int s = warp + kWarps * (first + r);
+        const int t = s / nsr, j = (s - t * nsr) * 32 + lane;
+        if (t < T && j < dv16) {
+          uint4 lo, hi;
+          deq16_one(xh[r], sh[r], lo, hi);
+          uint4* dst = reinterpret_cast<uint4*>(e16 + t * ldE + 16 * j);
+          dst[0] = lo;
+          dst[1] = hi;
+        }
+      }
+    }
+  }
+  for (int first = 0; first < (HEADS ? 0 : row_segs); first += kRowBatch) {
     RowChunk<NV> xa[kRowBatch], xb[kRowBatch];
     float sa[kRowBatch], sb[kRowBatch];
 #pragma unroll
@@ -472,10 +518,12 @@ cudaError_t launch_decode_small(const CUtensorMap& tmap_w, const DecodeSmallArgs
                                 cudaStream_t stream) {
   static PerDeviceOnce configured;
   const cudaError_t e = configured.run([] {
-    cudaError_t r = cudaFuncSetAttribute(decode_small_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t r = cudaFuncSetAttribute(decode_small_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemLimit);
     if (r == cudaSuccess)
-      r = cudaFuncSetAttribute(decode_small_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+      r = cudaFuncSetAttribute(decode_small_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(decode_small_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     return r;
   });
   if (e != cudaSuccess) return e;
@@ -489,8 +537,9 @@ cudaError_t launch_decode_small(const CUtensorMap& tmap_w, const DecodeSmallArgs
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.nvfp4) return cudaLaunchKernelEx(&cfg, decode_small_kernel<true>, tmap_w, a);
-  return cudaLaunchKernelEx(&cfg, decode_small_kernel<false>, tmap_w, a);
+  if (a.heads) return cudaLaunchKernelEx(&cfg, decode_small_kernel<2>, tmap_w, a);
+  if (a.nvfp4) return cudaLaunchKernelEx(&cfg, decode_small_kernel<1>, tmap_w, a);
+  return cudaLaunchKernelEx(&cfg, decode_small_kernel<0>, tmap_w, a);
 }
 
 }  // namespace ple

@@ -187,6 +187,7 @@ struct DecodeSmallArgs {
   const uint8_t* blocks;   // NVFP4 block scales (null for E4M3)
   const float* scales;
   int32_t nvfp4;
+  int32_t heads;           // 1: PLE_TABLE_E4M3_HEADS (rows0 = rows per head sub-table)
   const __nv_bfloat16* w_gate;
   const float* conv_w;
   const __nv_bfloat16* hidden;

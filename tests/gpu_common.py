@@ -55,18 +55,38 @@ def tiny_layer():
     L.close()
 
 
+_SHARED = {}
+
+
+def release_device_memory(layer):
+    """Close a layer, drop its device tensors and return the cached blocks to the
+    driver, so that the next module's full-scale table finds the memory free."""
+    import gc
+    import torch
+    layer.close()
+    for name in ("table", "scales", "block_scales", "w_proj", "w_gate", "conv_w"):
+        if hasattr(layer, name):
+            setattr(layer, name, None)
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
 @pytest.fixture(scope="session")
 def full_layer():
+    """The full-scale table (51.2 GB) and weights, created once per test process.
+    Every test module imports this fixture, and pytest would otherwise build one
+    instance per importing module."""
     import torch
     from ple_inputs.device import DeviceLayer
-    w = pi.workload("prefill")
-    free, _ = torch.cuda.mem_get_info()
-    if free < w.table_bytes + (8 << 30):
-        pytest.skip(f"needs {w.table_bytes / 1e9:.0f} GB for the full table, {free / 1e9:.0f} GB free")
-    L = DeviceLayer(w, max_tokens=16384, max_seqs=64)
-    L.host_table = w.table()
-    yield L
-    L.close()
+    if "full" not in _SHARED:
+        w = pi.workload("prefill")
+        free, _ = torch.cuda.mem_get_info()
+        if free < w.table_bytes + (8 << 30):
+            pytest.skip(f"needs {w.table_bytes / 1e9:.0f} GB for the full table, {free / 1e9:.0f} GB free")
+        L = DeviceLayer(w, max_tokens=16384, max_seqs=64)
+        L.host_table = w.table()
+        _SHARED["full"] = L
+    return _SHARED["full"]
 
 
 MID = pi.Workload("mid", 5000, 8192, 128, 256, table_seed=7, seed=7)

@@ -11,7 +11,7 @@ import pytest
 
 import oracle as O
 import ple_inputs as pi
-from tests.gpu_common import assert_bf16_close, assert_close
+from tests.gpu_common import assert_bf16_close, assert_close, release_device_memory
 
 torch = pytest.importorskip("torch")
 ple = pytest.importorskip("gram_embedding_lookup_b200")
@@ -40,7 +40,7 @@ def heads_full_layer():
     L = DeviceLayer(w, max_tokens=16384, max_seqs=64, table_format=ple.PLE_TABLE_E4M3_HEADS)
     L.host_table = w.heads_table()
     yield L
-    L.close()
+    release_device_memory(L)
 
 
 def dev_i32(a):

@@ -14,7 +14,7 @@ import ple_inputs as pi
 torch = pytest.importorskip("torch")
 ple = pytest.importorskip("gram_embedding_lookup_b200")
 
-from tests.gpu_common import MID, assert_bf16_close, assert_close  # noqa: E402
+from tests.gpu_common import MID, assert_bf16_close, assert_close, release_device_memory  # noqa: E402
 from tests.test_gpu_parity import _sample, dev_bf16, dev_i32, gpu_decode, gpu_forward, to_bits  # noqa: E402
 
 pytestmark = pytest.mark.gpu
@@ -53,7 +53,7 @@ def nv_full():
     L = _layer(w, 16384, 64)
     L.host_table = pi.SynthNvTable(w.table_seed, w.rows_per_order, w.row_dim)
     yield L
-    L.close()
+    release_device_memory(L)
 
 
 def _gather(L, ids):
