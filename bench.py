@@ -378,6 +378,7 @@ def main():
                 "frac_of_burst_peak": achieved_tf / peaks["bf16_tflops"],
                 "traffic": load_traffic("gemm", "prefill", source_hash(GEMM_SOURCES)),
                 "algorithmic_flops_per_launch": flops, "launch_ms": gemm_s * 1e3}
+    roofline["library_same_shape"] = library_gemm_same_shape(torch, T, D, H)
     e_ms, e_n = stage["prepare"]
     e_s = e_ms / 1e3 / max(e_n, 1)
     if args.path == 4:      # the first kernel computes only IDs and gate: h and tokens in; ids, meta out
@@ -445,6 +446,33 @@ def main():
     layer.close()
     if world > 1:
         dist.destroy_process_group()
+
+
+def library_gemm_same_shape(torch, T, D, H, n=300):
+    """Context for the projection's roofline: cuBLAS (torch.matmul) on a plain fp16
+    GEMM of the same shape, [T x D] @ [D x H] with fp32 accumulation, timed back
+    to back like the layer's loop. The library kernel has no gate, conv or
+    residual epilogue; it is a measurement beside the layer, not part of it."""
+    prev = torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    try:
+        a = torch.randn(T, D, device="cuda").to(torch.float16)
+        b = torch.randn(D, H, device="cuda").to(torch.float16)
+        c = torch.empty(T, H, device="cuda", dtype=torch.float16)
+        for _ in range(10):
+            torch.matmul(a, b, out=c)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            torch.matmul(a, b, out=c)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+    finally:
+        torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = prev
+    return {"kernel": "cuBLAS fp16 GEMM via torch.matmul (no epilogue)", "ms": ms,
+            "tflops": 2.0 * T * D * H / (ms / 1e3) / 1e12, "launches": n}
 
 
 def timed(ctx, stream, fn, n):
@@ -702,6 +730,7 @@ def heads_bench(ctx, sets, stream, peaks, steps=300):
     stage = ple.ple_get_stage_times(h)
     ple.ple_set_profiling(h, False)
     T = sets[0]["T"]
+    roofline["library_same_shape"] = library_gemm_same_shape(torch, T, D, H)
     e_ms, e_n = stage["prepare"]
     e_s = e_ms / 1e3 / max(e_n, 1)
     row_bytes = D + 16 * 4                        # 16 rows of D / 16 codes and their scales
@@ -770,6 +799,7 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
     stage = ple.ple_get_stage_times(h)
     ple.ple_set_profiling(h, False)
     T = sets[0]["T"]
+    roofline["library_same_shape"] = library_gemm_same_shape(torch, T, D, H)
     e_ms, e_n = stage["prepare"]
     e_s = e_ms / 1e3 / max(e_n, 1)
     row_bytes = 2 * (D // 2 + D // 16) + 8                  # both rows' codes and block scales, row scales
