@@ -158,18 +158,21 @@ bool wrong_device(const ple_handle* h) {
 bool heads_layout(const ple_handle* h) { return h->cfg.table_format == PLE_TABLE_E4M3_HEADS; }
 int ids_per_token(const ple_config& c) { return c.table_format == PLE_TABLE_E4M3_HEADS ? 16 : 2; }
 
-// The kernel computing the row IDs (and, as the arguments ask, gate, metadata,
+// The kernels computing the row IDs (and, as the arguments ask, gate, metadata,
 // state and e) for the handle's table layout.
-cudaError_t launch_embed_for(const ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream);
+cudaError_t launch_embed_for(ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream);
 
 ple::TableRef table_ref(const ple_handle* h) {
   const bool nv = h->cfg.table_format == PLE_TABLE_NVFP4;
   return ple::TableRef{h->w.table, nv ? h->w.block_scales : nullptr, h->w.scales, nv ? 1 : 0};
 }
 
-cudaError_t launch_embed_for(const ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream) {
+cudaError_t launch_embed_for(ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream) {
   if (heads_layout(h)) return ple::launch_embed_heads(pa, table_ref(h), h->cfg.row_dim, e, stream);
-  return ple::launch_embed(pa, table_ref(h), h->cfg.row_dim, e, h->num_sms, stream);
+  int kernels = 1;
+  const cudaError_t r = ple::launch_embed(pa, table_ref(h), h->cfg.row_dim, e, h->num_sms, stream, &kernels);
+  h->launches += kernels - 1;           // the stage counts one launch; large batches take two kernels
+  return r;
 }
 
 void free_all(ple_handle* h) {

@@ -71,7 +71,8 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream);
 // and e[t] for the batch. num_sms sizes the persistent grid. With e null it
 // writes only the ids and the metadata (the gather-fused projection follows).
 cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
-                         cudaStream_t stream);
+                         cudaStream_t stream,
+                         int* kernels = nullptr);
 
 // The multi-head layout (PLE_TABLE_E4M3_HEADS): one warp per token computes the
 // 16 head rows (ids [T][16]), the gate and metadata when a.meta is set, and

@@ -49,33 +49,38 @@ PrepareArgs with_magic(const PrepareArgs& in) {
   return a;
 }
 
-// Sequence, position, last-token flag and the bigram and trigram keys of token
-// t (every lane of the calling warp computes the same values; lane 0 reports
-// errors).
-__device__ __forceinline__ void sequence_and_keys(const PrepareArgs& a, int t, int lane, int32_t& s, int32_t& pos,
-                                                  int32_t& last, uint64_t& k2, uint64_t& k3) {
+// Sequence, position and last-token flag of token t. `report` decides which
+// caller records a range error.
+__device__ __forceinline__ void sequence_of(const PrepareArgs& a, int t, bool report, int32_t& s, int32_t& pos,
+                                            int32_t& last) {
   if (a.uniform_q > 0) {
     s = t / a.uniform_q;
     pos = t - s * a.uniform_q;
     last = (pos == a.uniform_q - 1);
-  } else {
-    int lo = 0, hi = a.S - 1;
-    while (lo < hi) {                         // largest s with offsets[s] <= t
-      const int mid = (lo + hi + 1) >> 1;
-      if (a.offsets[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    s = lo;
-    const int32_t begin = a.offsets[s];
-    const int32_t end = a.offsets[s + 1];
-    pos = t - begin;
-    if (pos < 0 || t >= end) {                // inconsistent offsets: keep every access in bounds
-      if (lane == 0) set_status(a.status, PLE_ERR_RANGE);
-      pos = max(0, min(pos, t));
-    }
-    last = (t == end - 1);
+    return;
   }
+  int lo = 0, hi = a.S - 1;
+  while (lo < hi) {                           // largest s with offsets[s] <= t
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.offsets[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  s = lo;
+  const int32_t begin = a.offsets[s];
+  const int32_t end = a.offsets[s + 1];
+  pos = t - begin;
+  if (pos < 0 || t >= end) {                  // inconsistent offsets: keep every access in bounds
+    if (report) set_status(a.status, PLE_ERR_RANGE);
+    pos = max(0, min(pos, t));
+  }
+  last = (t == end - 1);
+}
+
+// The bigram and trigram keys of token t at position pos of sequence s. Before
+// the sequence start the carried history, or nothing, stands in.
+__device__ __forceinline__ void keys_of(const PrepareArgs& a, int t, int32_t s, int32_t pos, bool report,
+                                        uint64_t& k2, uint64_t& k3) {
   const int32_t tok = a.tokens[t];
-  if (lane == 0 && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
+  if (report && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
   const uint64_t x0 = context_of(tok);
   auto carried = [&](int k) -> uint64_t {     // the token k places before the sequence start
     if (a.hist == nullptr) return 0ull;
@@ -88,7 +93,15 @@ __device__ __forceinline__ void sequence_and_keys(const PrepareArgs& a, int t, i
   k3 = k2 ^ (x2 * kP2);
 }
 
-// ... and the two row IDs of token t.
+// Sequence, position, last-token flag and the bigram and trigram keys of token
+// t (every lane of the calling warp computes the same values; lane 0 reports
+// errors).
+__device__ __forceinline__ void sequence_and_keys(const PrepareArgs& a, int t, int lane, int32_t& s, int32_t& pos,
+                                                  int32_t& last, uint64_t& k2, uint64_t& k3) {
+  sequence_of(a, t, lane == 0, s, pos, last);
+  keys_of(a, t, s, pos, lane == 0, k2, k3);
+}
+
 __device__ __forceinline__ void sequence_and_rows(const PrepareArgs& a, int t, int lane, int32_t& s, int32_t& pos,
                                                   int32_t& last, int32_t& r0, int32_t& r1) {
   uint64_t k2, k3;
@@ -550,6 +563,118 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ embed as independent work units
+// The same results as embed_pipe_kernel, from two launches whose work units do
+// not wait on one another, for large batches.
+//
+// ids_meta_kernel: a thread per token computes the sequence map, the row IDs
+// and the token's sequence, position and last-token flag (the gate field of
+// the metadata is left to the gate blocks), and extra blocks do the state
+// work. It lets the next grid launch at once.
+//
+// embed_split_kernel (launched as that grid's programmatic dependent): the
+// gate blocks come first, a warp per token; they stream h and write g with no
+// wait, since h does not depend on the IDs, and so cover the IDs kernel's
+// latency. The gather blocks follow: each waits for the IDs, then a thread
+// dequantises two 16-code chunks of both rows into e. They walk the tokens from
+// the end, so the first tokens' rows are the last written and still in L2 when
+// the projection starts on them. A gather block waiting for the IDs grid means
+// this grid completes only after that one, which the projection relies on; a
+// grid of gate blocks alone waits in its gate blocks.
+constexpr int kIdsThreads = 256;
+constexpr int kSplitThreads = 256;
+constexpr int kSplitGateTokens = kSplitThreads / 32;          // tokens per gate block
+constexpr int kSplitGatherChunks = 2 * kSplitThreads;         // 16-code chunks per gather block
+constexpr int kSplitMinTokens = 4096;                        // below this the one-kernel form is faster
+
+__global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs a, int token_blocks) {
+  pdl_launch_dependents();
+  if (static_cast<int>(blockIdx.x) >= token_blocks) {
+    state_blocks(a, blockIdx.x - token_blocks, gridDim.x - token_blocks, threadIdx.x, blockDim.x);
+    return;
+  }
+  const int t = blockIdx.x * kIdsThreads + threadIdx.x;
+  if (t >= a.T) return;
+  int32_t s, pos, last, r0, r1;
+  sequence_of(a, t, true, s, pos, last);
+  uint64_t k2, k3;
+  keys_of(a, t, s, pos, true, k2, k3);
+  r0 = static_cast<int32_t>(mod_barrett(fold64(k2), static_cast<uint64_t>(a.rows0), a.magic0));
+  r1 = static_cast<int32_t>(mod_barrett(fold64(k3), static_cast<uint64_t>(a.rows1), a.magic1));
+  reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
+  if (a.meta == nullptr) return;
+  if (a.hidden == nullptr) {                  // no gate blocks: the gate field is written later, by the gate kernel
+    TokMeta m;
+    m.g = 0.f;
+    m.seq = s;
+    m.pos = pos;
+    m.flags = last ? kFlagLast : 0;
+    a.meta[t] = m;
+  } else {                                    // every field but g, which a gate block writes meanwhile
+    int32_t* m = reinterpret_cast<int32_t*>(a.meta + t);
+    m[1] = s;
+    reinterpret_cast<int2*>(m)[1] = make_int2(pos, last ? kFlagLast : 0);
+  }
+}
+
+template <bool NV>
+__global__ void __launch_bounds__(kSplitThreads, 4)
+    embed_split_kernel(const PrepareArgs a, const TableRef tab, int32_t D, __half* __restrict__ e, int32_t n_gate,
+                       int32_t n_blocks) {
+  pdl_launch_dependents();
+  const int64_t b = blockIdx.x;
+  if (b < n_gate) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = static_cast<int>(b) * kSplitGateTokens + warp;
+    if (t < a.T) {
+      const int H8 = a.H / 8;
+      const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+      uint4 hv[kEmbedH4];
+#pragma unroll
+      for (int r = 0; r < kEmbedH4; ++r) {
+        const int j = lane + 32 * r;
+        if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+      }
+      const float g = gate_warp(hv, hrow, reinterpret_cast<const uint4*>(a.w_gate), H8, lane);
+      if (lane == 0) a.meta[t].g = g;
+    }
+    if (n_blocks == n_gate) pdl_wait();                          // no gather block waits for the IDs grid
+    return;
+  }
+  pdl_wait();                                                    // the row IDs
+  const int D16 = D / 16;
+  const int64_t n_chunks = static_cast<int64_t>(a.T) * D16;
+  const int64_t base = (n_blocks - 1 - b) * kSplitGatherChunks + threadIdx.x;
+  RowChunk<NV> ca[2], cb[2];
+  float sa[2], sb[2];
+  int64_t idx[2];
+  // both chunks' loads first, then both dequantisations
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    idx[u] = base + u * kSplitThreads;
+    if (idx[u] < n_chunks) {
+      const int32_t t = static_cast<int32_t>(idx[u] / D16);
+      const int c = static_cast<int>(idx[u] - static_cast<int64_t>(t) * D16);
+      const int2 id = reinterpret_cast<const int2*>(a.ids)[t];
+      const int64_t row0 = id.x, row1 = a.rows0 + id.y;
+      ca[u] = load_chunk<NV>(tab.codes, tab.blocks, row0, D, c);
+      cb[u] = load_chunk<NV>(tab.codes, tab.blocks, row1, D, c);
+      sa[u] = __ldg(tab.scales + row0);
+      sb[u] = __ldg(tab.scales + row1);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    if (idx[u] < n_chunks) {
+      uint4 o0, o1;
+      deq_chunk<NV>(ca[u], cb[u], sa[u], sb[u], o0, o1);
+      uint4* dst = reinterpret_cast<uint4*>(e + idx[u] * 16);
+      dst[0] = o0;
+      dst[1] = o1;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ bounded-wait self-test
 // One warp waits, through the same bounded wait the library's kernels use, on
 // an mbarrier that expects one arrival nobody makes. The wait runs out after
@@ -682,7 +807,37 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, int* kernels) {
+  if (kernels != nullptr) *kernels = 1;
+  if (a.T >= kSplitMinTokens) {
+    // large batches: IDs kernel, then gate and gather blocks as its dependent
+    const PrepareArgs am = with_magic(a);
+    const int token_blocks = (a.T + kIdsThreads - 1) / kIdsThreads;
+    int sblocks = 1;
+    if (a.conv_in != nullptr) {
+      const int64_t want = (static_cast<int64_t>(a.S) * 3 * a.H / 4 + kIdsThreads - 1) / kIdsThreads;
+      sblocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
+    }
+    ids_meta_kernel<<<token_blocks + sblocks, kIdsThreads, 0, stream>>>(am, token_blocks);
+    cudaError_t r = cudaGetLastError();
+    if (r != cudaSuccess) return r;
+    const int64_t n_gate = a.hidden != nullptr && a.meta != nullptr ? (a.T + kSplitGateTokens - 1) / kSplitGateTokens : 0;
+    const int64_t n_gather = e != nullptr ? (static_cast<int64_t>(a.T) * (D / 16) + kSplitGatherChunks - 1) / kSplitGatherChunks : 0;
+    if (n_gate + n_gather == 0) return cudaSuccess;
+    if (kernels != nullptr) *kernels = 2;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_gate + n_gather));
+    cfg.blockDim = dim3(kSplitThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int32_t ng = static_cast<int32_t>(n_gate), nblk = static_cast<int32_t>(n_gate + n_gather);
+    if (table.nvfp4) return cudaLaunchKernelEx(&cfg, embed_split_kernel<true>, am, table, D, e, ng, nblk);
+    return cudaLaunchKernelEx(&cfg, embed_split_kernel<false>, am, table, D, e, ng, nblk);
+  }
   const bool state = a.conv_in != nullptr || a.hist_new != nullptr;
   // small batches spread over the SMs: a few tokens per CTA, no warp taking two in turn
   const int grid = state ? num_sms : std::min<int>(num_sms, a.T);
