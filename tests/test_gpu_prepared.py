@@ -161,3 +161,33 @@ def test_prepared_equals_forward_full(full_layer):
     ref, _ = gpu_forward(full_layer, toks, offs, hid, 0)
     got, _ = _prepared(full_layer, toks, offs, hid, 0)
     assert np.array_equal(got, ref)
+
+
+def test_two_launch_embed_ragged_state_full(full_layer):
+    """Batches of 4,096 tokens or more take the two-launch embed: an IDs kernel,
+    then gate blocks and gather blocks. A ragged batch of 5,001 tokens (the last
+    gate block holds one token, the last gather block is partial) with empty
+    sequences and carried history and conv state, on samples against the
+    oracle; the two-call form of the same batch, whose embed grid has no gate
+    blocks, gives the same bits and the same state."""
+    from tests.gpu_common import assert_close
+    from tests.test_gpu_parity import _sample, check_state, oracle_forward
+    w = pi.workload("prefill")
+    lengths = [1, 0, 2, 2500, 0, 2495, 3]
+    rng = np.random.default_rng(91)
+    T, S = sum(lengths), len(lengths)
+    toks = rng.integers(0, w.vocab, T).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    hid = pi.hidden_bf16(rng, T, w.hidden)
+    hist0 = rng.integers(-1, w.vocab, (S, 2)).astype(np.int32)
+    hist0[1] = [-1, -1]
+    conv0 = rng.standard_normal((S, 3, w.hidden)).astype(np.float32)
+    out, st = gpu_forward(full_layer, toks, offs, hid, 1, state=(hist0, conv0))
+    sample = _sample(T, offs, 300, 92)
+    ref = oracle_forward(full_layer, toks, offs, hid, hist=hist0, conv=conv0, sample=sample)
+    assert_close(out[sample], ref["out"], "ragged 5,001-token prefill with state")
+    check_state(st, ref)
+    got, got_st = _prepared(full_layer, toks, offs, hid, 1, state=(hist0, conv0))
+    assert np.array_equal(_f32bits(got), _f32bits(out))
+    assert np.array_equal(got_st[0], st[0])
+    assert np.array_equal(_f32bits(got_st[1]), _f32bits(st[1]))
