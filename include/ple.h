@@ -252,19 +252,22 @@ const char* ple_status_string(ple_status status);
 
 /* Kernel stages of the library, in launch order within a call. In
  * ple_forward and ple_decode_step the PREPARE stage also gathers and
- * dequantises the rows (one fused kernel), except on the gather-fused path,
- * where the GEMM stage does; ple_prepare and the gate kernel of
- * ple_forward_prepared count as PREPARE too. GATHER counts ple_gather_rows. */
+ * dequantises the rows, except on the gather-fused path, where the GEMM stage
+ * does. PREPARE is one fused kernel, or, for a batch of 4,096 tokens or more,
+ * a row-ID kernel followed by the gate-and-gather kernel. ple_prepare and the
+ * gate kernel of ple_forward_prepared count as PREPARE too. GATHER counts
+ * ple_gather_rows. */
 enum { PLE_STAGE_PREPARE = 0, PLE_STAGE_GATHER = 1, PLE_STAGE_GEMM = 2, PLE_STAGE_COMBINE = 3,
        PLE_NUM_STAGES = 4 };
 
-/* enable != 0: record CUDA events around every kernel the handle launches
- * (on the call's stream) so that ple_get_stage_times can report them. */
+/* enable != 0: record CUDA events around every stage the handle runs (on the
+ * call's stream) so that ple_get_stage_times can report them. */
 ple_status ple_set_profiling(ple_handle* handle, int32_t enable);
 
-/* Synchronises the recorded events and writes, per stage, the summed kernel
- * time in milliseconds (ms[PLE_NUM_STAGES]) and the number of launches
- * (launches[PLE_NUM_STAGES]) since the last call; then resets the counters. */
+/* Synchronises the recorded events and writes, per stage, the summed time in
+ * milliseconds (ms[PLE_NUM_STAGES]) and the number of times the stage ran
+ * (launches[PLE_NUM_STAGES]) since the last call; then resets the counters.
+ * ple_launch_count counts kernels. */
 ple_status ple_get_stage_times(ple_handle* handle, float* ms, int64_t* launches);
 
 /* Path selection. For ple_forward: 0 = automatic, 1 = fused epilogue
