@@ -87,16 +87,6 @@ def test_dequantise_nvfp4_brute_force():
             assert got[r, k] == v
 
 
-def test_nvfp4_table_size_matches_the_pages():
-    """Two sub-tables of 10,000,048 rows of 2560 elements at 4.5 bits per element."""
-    R, D = 10_000_048, 2560
-    code_bytes = 2 * R * D // 2
-    block_bytes = 2 * R * D // 16
-    gib = (code_bytes + block_bytes) / 2 ** 30
-    assert round(gib, 2) == 26.82
-    assert round(2 * R * D * 2 / 2 ** 30, 2) == 95.37     # the BF16 table it replaces
-
-
 def test_embed_nvfp4_sums_orders():
     rng = np.random.default_rng(5)
     codes, blocks, scales = _small_nv_table(rng)
