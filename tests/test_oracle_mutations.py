@@ -149,3 +149,12 @@ def test_heads_reversed_concatenation_caught(monkeypatch):
     _patch(monkeypatch, "embed", bad)
     assert _fails(heads_pins.test_heads_embed_concatenates_in_head_order)
     assert _fails(heads_pins.test_heads_layer_matches_brute_force)
+
+
+@pytest.mark.parametrize("bad", [0x9E3779B9, 0x9E3779B97F4A7C13, 0x9E3779B97F4A7C17])
+def test_mistyped_hash_multiplier_caught(monkeypatch, bad):
+    """The 32-bit golden-ratio constant, or the 64-bit one off in its last digit:
+    the structural ID pins still hold for either, the closed-form pin does not."""
+    monkeypatch.setattr(OP, "P0", bad)
+    monkeypatch.setattr(O, "P0", bad)
+    assert _fails(pins.test_hash_multiplier_is_the_golden_ratio_constant)

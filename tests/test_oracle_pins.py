@@ -59,6 +59,14 @@ def _ids(tokens, offsets=None, hist=None, rows=R):
     return O.ngram_ids(np.array(tokens, dtype=np.int32), offsets, rows, hist)
 
 
+def test_hash_multiplier_is_the_golden_ratio_constant():
+    """P0 is floor(2^64 (sqrt 5 - 1) / 2), the multiplier of Knuth's multiplicative
+    hashing, computed here in exact integer arithmetic. P1 and P2 are odd, so each
+    product is a bijection of the 64-bit contexts."""
+    assert O.P0 == (math.isqrt(5 << 128) - (1 << 64)) // 2
+    assert O.P1 % 2 == 1 and O.P2 % 2 == 1
+
+
 def test_ids_dependence_structure():
     """Bigram row depends on (t, t-1) only; trigram row on (t, t-1, t-2) only."""
     base = [11, 22, 33, 44, 55]
