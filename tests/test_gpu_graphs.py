@@ -4,12 +4,10 @@ graphs) replays to the same bits as eager launches.
 Every call is stream-ordered and does its host work (argument checks, tensor
 maps, launch planning) at capture time; the kernels keep no state between
 launches that a replay could see stale (the single-kernel decode step resets
-its tile counters itself). Five forms are captured: a decode step (one
+its tile counters itself). Four forms are captured: a decode step (one
 kernel under programmatic dependent launch), an MTP-style decode step on the
-split-K path, a prefill on SM-pair tiles, a 4,096-token prefill whose embed
-stage is two launches (IDs, then gate and gather, chained to the projection
-by programmatic dependent launch) and a small forward on the split-K path
-(projection then combine).
+split-K path, a prefill on SM-pair tiles and a small forward on the split-K
+path (projection then combine).
 """
 import numpy as np
 import pytest
@@ -75,7 +73,7 @@ def test_decode_step_graph_replay_matches_eager(mid_layer):  # noqa: F811
     del graph
 
 
-@pytest.mark.parametrize("lengths,path", [([1500, 700, 1], 1), ([40, 3, 5], 2), ([2000, 0, 2096], 1)])
+@pytest.mark.parametrize("lengths,path", [([1500, 700, 1], 1), ([40, 3, 5], 2)])
 def test_forward_graph_replay_matches_eager(mid_layer, lengths, path):  # noqa: F811
     from ple_inputs.device import bf16_tensor
     L = mid_layer
