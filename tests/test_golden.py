@@ -16,6 +16,21 @@ import oracle as O
 import ple_inputs as pi
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "page_figures.txt")
+HASH_EXAMPLE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hash_worked_example.txt")
+
+
+def hash_worked_example():
+    """The worked example of the n-gram hash: [(rows, tokens, [(bigram row, trigram row), ...]), ...]
+    for one sequence each with no carried history (``tests/golden/hash_worked_example.txt``)."""
+    cases = []
+    with open(HASH_EXAMPLE, encoding="utf-8") as f:
+        for line in f:
+            if not line.strip() or line.startswith("#"):
+                continue
+            rows, toks, ids = (part.split() for part in line.split("|"))
+            pairs = [tuple(int(v) for v in pair.split(",")) for pair in ids]
+            cases.append((int(rows[0]), [int(t) for t in toks], pairs))
+    return cases
 
 
 def _figures():
@@ -71,3 +86,11 @@ def test_model_dimensions():
     w = pi.workload("prefill")
     assert w.hidden == F["hidden"]
     assert w.vocab == F["vocab"]
+
+
+def test_hash_worked_example_fixture_shape():
+    cases = hash_worked_example()
+    assert [(r, len(t)) for r, t, _ in cases] == [(4096, 5), (10_000_048, 5), (10_000_048, 3)]
+    for rows, toks, ids in cases:
+        assert len(ids) == len(toks)
+        assert all(0 <= a < rows and 0 <= b < rows for a, b in ids)

@@ -138,6 +138,40 @@ def test_ids_full_scale_workloads(full_layer, name):
     assert np.array_equal(gpu_ids(full_layer, toks, offs, hist), O.ngram_ids(toks, offs, R, hist))
 
 
+def test_ids_hash_worked_example(tiny_layer, full_layer):  # noqa: F811
+    """The worked example of the hash (``tests/golden/hash_worked_example.txt``, written down
+    from the definition before any implementation) through the library's own copy of the
+    constants: ple_ngram_ids on tables of 4,096 and of 10,000,048 rows per order."""
+    from tests.test_golden import hash_worked_example
+    layers = {4096: tiny_layer, 10_000_048: full_layer}
+    for rows, toks, expect in hash_worked_example():
+        L = layers[rows]
+        assert L.w.rows_per_order == rows
+        got = gpu_ids(L, np.array(toks, np.int32), [0, len(toks)])
+        assert [tuple(int(v) for v in r) for r in got] == expect, (rows, toks)
+
+
+def test_decode_hash_worked_example(tiny_layer):
+    """The decode kernel hashes with its own code: one sequence of the worked example's tokens
+    with no history, as a single 1 x 5 decode step, must gather the worked example's rows, so it
+    matches the oracle run on those literal row IDs."""
+    from tests.test_golden import hash_worked_example
+    rows, toks, expect = hash_worked_example()[0]
+    assert rows == tiny_layer.w.rows_per_order
+    w = tiny_layer.w
+    hid = pi.hidden_bf16(np.random.default_rng(11), len(toks), w.hidden)
+    tk = np.array([toks], np.int32)
+    out, _, _ = gpu_decode(tiny_layer, tk, hid, np.full((1, 2), -1, np.int32), np.zeros((1, 3, w.hidden), np.float32))
+    W = tiny_layer.host_weights
+    e = O.embed(tiny_layer.host_table, np.array(expect, np.int64))
+    v = O.project(e, O.bf16_bits_to_f64(W.w_proj))
+    g = O.gate(O.bf16_bits_to_f64(hid), O.bf16_bits_to_f64(W.w_gate))
+    u = g[:, None] * v
+    u_hist = np.concatenate([np.zeros((3, w.hidden)), u])
+    y = O.short_conv(u_hist, W.conv_w)
+    assert_close(out, O.bf16_bits_to_f64(hid) + y, "decode step on the worked example")
+
+
 # ----------------------------------------------------------------------------- gather
 def _gather(L, ids):
     T = ids.shape[0]

@@ -158,3 +158,17 @@ def test_mistyped_hash_multiplier_caught(monkeypatch, bad):
     monkeypatch.setattr(OP, "P0", bad)
     monkeypatch.setattr(O, "P0", bad)
     assert _fails(pins.test_hash_multiplier_is_the_golden_ratio_constant)
+
+
+@pytest.mark.parametrize("name,delta", [("P0", 1 << 8), ("P1", 1 << 36), ("P2", 1 << 4), ("P1", 0x30 << 56)])
+def test_one_digit_hash_constant_change_caught(monkeypatch, name, delta):
+    """Changing one hex digit of a hash multiplier (kept odd) moves some worked-example row."""
+    monkeypatch.setattr(OP, name, getattr(OP, name) ^ delta)
+    assert getattr(OP, name) % 2 == 1
+    assert _fails(pins.test_ids_match_the_hash_worked_example)
+
+
+def test_context_offset_dropped_caught(monkeypatch):
+    """Contexts without the +1 (token 0 indistinguishable from an absent position)."""
+    monkeypatch.setattr(OP, "_context_value", lambda token: int(token) & 0xFFFFFFFF)
+    assert _fails(pins.test_ids_match_the_hash_worked_example)

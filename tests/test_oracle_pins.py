@@ -67,6 +67,20 @@ def test_hash_multiplier_is_the_golden_ratio_constant():
     assert O.P1 % 2 == 1 and O.P2 % 2 == 1
 
 
+def test_ids_match_the_hash_worked_example():
+    """The row IDs of the worked example in ``tests/golden/hash_worked_example.txt``, written
+    down from the hash definition in exact integer arithmetic before the oracle existed.
+    This pins every constant and step of the hash (all three multipliers, the context offset,
+    the fold, the mod) from outside the oracle: a one-digit change to any of them moves some
+    row. Positions 2 and 4 share the bigram context (17, 42) and so the bigram row, while
+    their trigram rows differ; at the first two positions the trigram key equals the bigram
+    key."""
+    from tests.test_golden import hash_worked_example
+    for rows, toks, expect in hash_worked_example():
+        got = [tuple(int(v) for v in r) for r in _ids(toks, rows=rows)]
+        assert got == expect, (rows, toks)
+
+
 def test_ids_dependence_structure():
     """Bigram row depends on (t, t-1) only; trigram row on (t, t-1, t-2) only."""
     base = [11, 22, 33, 44, 55]
