@@ -9,6 +9,7 @@
 // allocates. This entry point takes every input and the output from the
 // caller and keeps its only intermediate (the row IDs) in a fixed array that
 // lives in the library image.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -25,30 +26,72 @@ static __device__ __align__(256) int32_t g_static_ids[2 * PLE_STATIC_MAX_TOKENS]
 static __device__ __align__(256) int32_t g_static_status[64];
 
 constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-int32_t* g_ids_ptr[kMaxDevices] = {};
-int32_t* g_status_ptr[kMaxDevices] = {};
+constexpr int32_t kMaxRowDim = 65536;   // the widest row the gather's index arithmetic is sized for
 
-// Device addresses of the arrays on the current device. In host code the
-// arrays' names are host-side stand-ins, not device addresses; the addresses
-// come from cudaGetSymbolAddress, looked up once per device.
+// The arrays' device addresses, looked up once per device and context. In host
+// code the arrays' names are host-side stand-ins, not device addresses; the
+// addresses come from cudaGetSymbolAddress with the device current. After
+// cudaDeviceReset the library's image is loaded into a new context at other
+// addresses, so the cache is keyed by the context's unique ID and the lookup
+// runs again when that ID changes.
+struct DeviceScratch {
+  unsigned long long ctx_id = 0;
+  int32_t* ids = nullptr;
+  int32_t* status = nullptr;
+};
+std::mutex g_setup_mutex;
+DeviceScratch g_scratch[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique ID of the current context (0 if the driver cannot say). The runtime
+// call before it makes sure the device's primary context exists.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa{}, qb{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+    cudaGetLastError();
+  });
+  if (get_current == nullptr || get_id == nullptr || cudaFree(nullptr) != cudaSuccess) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 ple_status static_scratch(int32_t** ids, int32_t** status) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PLE_ERR_CUDA;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_ids_ptr[dev] == nullptr) {
+  DeviceScratch& d = g_scratch[dev];
+  if (d.ids == nullptr || ctx == 0 || ctx != d.ctx_id) {
     void* a = nullptr;
     void* b = nullptr;
     if (cudaGetSymbolAddress(&a, g_static_ids) != cudaSuccess ||
         cudaGetSymbolAddress(&b, g_static_status) != cudaSuccess || a == nullptr || b == nullptr) {
       cudaGetLastError();
+      d = DeviceScratch{};
       return PLE_ERR_CUDA;
     }
-    g_ids_ptr[dev] = static_cast<int32_t*>(a);
-    g_status_ptr[dev] = static_cast<int32_t*>(b);
+    d.ctx_id = ctx;
+    d.ids = static_cast<int32_t*>(a);
+    d.status = static_cast<int32_t*>(b);
   }
-  *ids = g_ids_ptr[dev];
-  *status = g_status_ptr[dev];
+  *ids = d.ids;
+  *status = d.status;
   return PLE_OK;
 }
 
@@ -64,8 +107,14 @@ extern "C" ple_status ple_embed_static(const int32_t* tokens, int32_t T, const i
       rows1 >= (int64_t(1) << 31))
     return PLE_ERR_INVALID_ARG;
   if (T > PLE_STATIC_MAX_TOKENS) return PLE_ERR_SHAPE;
-  if (row_dim % 16 != 0) return PLE_ERR_UNSUPPORTED;
-  if (T == 0) return PLE_OK;
+  if (row_dim % 16 != 0 || row_dim > kMaxRowDim) return PLE_ERR_UNSUPPORTED;
+  if (status_out != nullptr && !aligned(status_out, 4)) return PLE_ERR_ALIGN;
+  if (T == 0) {
+    // nothing to look up; the caller's status word still reports this call
+    if (status_out != nullptr && cudaMemsetAsync(status_out, 0, sizeof(int32_t), stream) != cudaSuccess)
+      return PLE_ERR_CUDA;
+    return PLE_OK;
+  }
   if (tokens == nullptr || offsets == nullptr || table == nullptr || scales == nullptr || e_out == nullptr)
     return PLE_ERR_INVALID_ARG;
   if (!aligned(tokens, 4) || !aligned(offsets, 4) || (hist && !aligned(hist, 4)) || !aligned(table, 16) ||

@@ -227,15 +227,20 @@ ple_status ple_decode_step(ple_handle* handle, const int32_t* tokens, int32_t B,
  * exits. The caller passes all inputs and the output; table and scales are
  * laid out as in ple_weights, with rows0 / rows1 rows in the two sub-tables.
  *   - T > PLE_STATIC_MAX_TOKENS returns PLE_ERR_SHAPE; nothing is launched.
+ *     row_dim must be a multiple of 16 and at most 65536 (else
+ *     PLE_ERR_UNSUPPORTED).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture. After cudaDeviceReset the next call on that
+ *     device looks the address up again (the library image then lives in a
+ *     new context), so that call too belongs outside a capture.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents. Calls that overlap on the GPU (other streams, other threads)
  *     race on it: order them on one stream.
  *   - status_out (device int32, may be NULL) receives the call's device status:
  *     PLE_ERR_RANGE for a token outside [0, vocab) or inconsistent offsets,
- *     else PLE_OK. The status word is cleared at the start of every call. */
+ *     else PLE_OK. Every call that returns PLE_OK writes it, T == 0 included
+ *     (which launches nothing else and writes PLE_OK). */
 #define PLE_STATIC_MAX_TOKENS 16384
 ple_status ple_embed_static(const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
                             const int32_t* hist, const uint8_t* table, const float* scales,

@@ -9,12 +9,15 @@ library and gathers the dequantised rows into the caller's buffer.
 This test checks it through the C ABI against the handle-based entry points
 (ple_ngram_ids followed by ple_gather_rows) on two calls in a row, the second
 one smaller than the first, so that contents the fixed array keeps from the
-earlier call cannot leak into a later result. The file's name makes pytest
-collect it last.
+earlier call cannot leak into a later result; against the CPU oracle (the
+n-gram row IDs, then the dequantised rows, within one fp16 ulp) with unequal
+sub-table sizes and carried history; and that a call allocates no device
+memory. The file's name makes pytest collect it last.
 """
 import numpy as np
 import pytest
 
+import oracle as O
 import ple_inputs as pi
 
 torch = pytest.importorskip("torch")
@@ -94,3 +97,91 @@ def test_embed_static_reports_range_errors():
         assert status == 0                      # the status word is cleared by each call
     finally:
         layer.close()
+
+
+def _static_call(tokens, offsets, hist, table, scales, rows0, rows1, row_dim, vocab, e, status):
+    ple.ple_embed_static(_i32(tokens), len(tokens), _i32(offsets), len(offsets) - 1,
+                         None if hist is None else _i32(hist), table, scales, rows0, rows1, row_dim, vocab, e, status)
+
+
+def test_embed_static_matches_oracle_unequal_sub_tables():
+    """Rows within one fp16 ulp of the oracle's e = deq(bigram row) + deq(trigram row), with
+    sub-tables of 3,001 and 4,000 rows laid back to back in one buffer (order 1 starts at row
+    3,001) and carried history, on two calls in a row."""
+    w = pi.workload("tiny")
+    D = w.row_dim
+    codes, scales = w.table().full()                  # [2][4096][D], [2][4096]
+    flat_codes = codes.reshape(-1, D)
+    flat_scales = scales.reshape(-1)
+    rows0, rows1 = 3001, 4000
+    host = O.ArrayTable([flat_codes[:rows0], flat_codes[rows0:rows0 + rows1]],
+                        [flat_scales[:rows0], flat_scales[rows0:rows0 + rows1]])
+    table = torch.from_numpy(np.ascontiguousarray(flat_codes)).cuda()
+    sc = torch.from_numpy(np.ascontiguousarray(flat_scales)).cuda()
+    rng = np.random.default_rng(77)
+    calls = [
+        (rng.integers(0, w.vocab, 900), [0, 1, 1, 2, 450, 900],
+         np.array([[-1, -1], [5, 6], [-1, 9], [7, 8], [100, 200]])),
+        (rng.integers(0, w.vocab, 64), [0, 64], np.array([[12, 13]])),
+    ]
+    for tokens, offsets, hist in calls:
+        T = len(tokens)
+        e = torch.full((T, D), float("nan"), dtype=torch.float16, device="cuda")
+        status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+        _static_call(tokens, offsets, hist, table, sc, rows0, rows1, D, w.vocab, e, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        ids = O.ngram_ids(np.asarray(tokens, np.int32), offsets, (rows0, rows1), hist)
+        ref16 = O.embed(host, ids).astype(np.float16)
+        a = e.cpu().numpy().view(np.uint16).astype(np.int32)
+        b = ref16.view(np.uint16).astype(np.int32)
+        ulp = np.abs(np.where(a & 0x8000, -(a & 0x7FFF), a & 0x7FFF) - np.where(b & 0x8000, -(b & 0x7FFF), b & 0x7FFF))
+        assert ulp.max() <= 1, ulp.max()
+
+
+def test_embed_static_allocates_nothing():
+    """After a first call on the device, a call changes neither the device's free memory nor
+    torch's allocated bytes: its only scratch is the library's fixed array."""
+    w = pi.workload("tiny")
+    codes, scales = w.table().full()
+    table = torch.from_numpy(np.ascontiguousarray(codes.reshape(-1))).cuda()
+    sc = torch.from_numpy(np.ascontiguousarray(scales.reshape(-1))).cuda()
+    rng = np.random.default_rng(5)
+    tokens = _i32(rng.integers(0, w.vocab, 4096))
+    offsets = _i32([0, 1000, 4096])
+    e = torch.empty(4096, w.row_dim, dtype=torch.float16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    R = w.rows_per_order
+
+    def call():
+        ple.ple_embed_static(tokens, 4096, offsets, 2, None, table, sc, R, R, w.row_dim, w.vocab, e, status)
+
+    call()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0
+    assert int(status.item()) == 0
+
+
+def test_embed_static_empty_batch_writes_status():
+    """T == 0 launches no lookup but still reports PLE_OK in the caller's status word."""
+    w = pi.workload("tiny")
+    status = torch.full((1,), -7, dtype=torch.int32, device="cuda")
+    offsets = _i32([0, 0])
+    R = w.rows_per_order
+    ple.ple_embed_static(0, 0, offsets, 1, None, 0, 0, R, R, w.row_dim, w.vocab, 0, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
+def test_embed_static_rejects_oversize_rows():
+    w = pi.workload("tiny")
+    code = ple.lib().ple_embed_static(None, 4, None, 1, None, None, None, w.rows_per_order, w.rows_per_order,
+                                      65536 + 16, w.vocab, None, None, None)
+    assert code == 8
