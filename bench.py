@@ -88,78 +88,149 @@ def load_traffic(kernel: str, workload: str, src_hash: str):
 
 
 _SAMPLER = r"""
-import sys, time, pynvml
-pynvml.nvmlInit()
-bus, idx, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
-dev = None
-if bus != "-":
-    try:
-        dev = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-    except Exception:
-        dev = None
-if dev is None:
-    dev = pynvml.nvmlDeviceGetHandleByIndex(idx)
-print("max", pynvml.nvmlDeviceGetMaxClockInfo(dev, pynvml.NVML_CLOCK_SM), flush=True)
+import sys, time
+try:
+    import pynvml
+    pynvml.nvmlInit()
+    bus, idx, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+    dev = None
+    if bus != "-":
+        try:
+            dev = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            dev = None
+    if dev is None:
+        dev = pynvml.nvmlDeviceGetHandleByIndex(idx)
+    print("max", pynvml.nvmlDeviceGetMaxClockInfo(dev, pynvml.NVML_CLOCK_SM), flush=True)
+except Exception as exc:
+    print("error", type(exc).__name__, str(exc).replace(chr(10), " ")[:200], flush=True)
+    sys.exit(0)
 while True:
     try:
         print(pynvml.nvmlDeviceGetClockInfo(dev, pynvml.NVML_CLOCK_SM),
               pynvml.nvmlDeviceGetCurrentClocksEventReasons(dev), flush=True)
-    except Exception:
-        pass
+    except Exception as exc:
+        print("error", type(exc).__name__, str(exc).replace(chr(10), " ")[:200], flush=True)
     time.sleep(period)
 """
 
+_SMI_QUERY = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
 
 class ClockSampler:
-    """SM clock and throttle reasons, sampled through NVML every few milliseconds by a
-    separate process while running (reads only; no setting is changed)."""
+    """SM clock and throttle reasons, sampled while running by a separate process that
+    only reads: NVML every few milliseconds, or, if NVML cannot be used there,
+    `nvidia-smi --query-gpu ... -lms 200`. When neither produces a sample, stop() says
+    why instead of returning nothing."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
+    SMI_REASONS = ("hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index: int, period_s: float = 0.005, pci_bus_id: str | None = None):
         self.index = index
         self.period = period_s
         self.pci_bus_id = pci_bus_id
         self.proc = None
+        self.kind = None
+        self.errors = []
+        self.max_mhz = float("nan")
 
     def start(self):
-        """Starts the sampler and returns once it is producing samples."""
+        """Starts the sampler and returns once it is producing samples (or has failed)."""
         try:
             self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER, self.pci_bus_id or "-", str(self.index),
-                                          str(self.period)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                          str(self.period)], stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
                                          text=True)
             first = self.proc.stdout.readline().split()
-            self.max_mhz = float(first[1]) if len(first) == 2 and first[0] == "max" else float("nan")
-            self.proc.stdout.readline()             # one sample taken: the sampler is live
-        except Exception:  # pragma: no cover - no NVML on this host
+            if len(first) == 2 and first[0] == "max":
+                self.max_mhz = float(first[1])
+                self.kind = "nvml"
+                self.proc.stdout.readline()         # one sample taken: the sampler is live
+                return
+            self.errors.append("NVML sampler: " + (" ".join(first) or f"exited with {self.proc.wait()}"))
+            self.proc.wait()
+        except Exception as exc:  # pragma: no cover - no NVML on this host
+            self.errors.append(f"NVML sampler: {type(exc).__name__}: {exc}")
+        self.proc = None
+        target = self.pci_bus_id or str(self.index)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", target, f"--query-gpu={_SMI_QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
+            self.kind = "nvidia-smi"
+            time.sleep(0.3)
+        except Exception as exc:
+            self.errors.append(f"nvidia-smi: {type(exc).__name__}: {exc}")
             self.proc = None
 
     def stop(self):
         if self.proc is None:
-            return None
+            return {"unavailable": "; ".join(self.errors) or "no sampler started"}
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        mhz, reasons = [], set()
+        mhz, reasons, other = [], set(), []
         for line in out.splitlines():
-            parts = line.split()
-            if len(parts) != 2:
-                continue
-            try:
-                m, r = float(parts[0]), int(parts[1])
-            except ValueError:
-                continue
-            mhz.append(m)
-            reasons |= {n for n, bit in self.REASONS.items() if r & bit}
+            if self.kind == "nvml":
+                parts = line.split()
+                try:
+                    m, r = float(parts[0]), int(parts[1])
+                except (ValueError, IndexError):
+                    other.append(line.strip())
+                    continue
+                mhz.append(m)
+                reasons |= {n for n, bit in self.REASONS.items() if r & bit}
+            else:
+                parts = [p.strip() for p in line.split(",")]
+                try:
+                    m, mx = float(parts[0]), float(parts[1])
+                except (ValueError, IndexError):
+                    other.append(line.strip())
+                    continue
+                mhz.append(m)
+                self.max_mhz = mx
+                reasons |= {n for n, v in zip(self.SMI_REASONS, parts[2:]) if v.lower() == "active"}
         if not mhz:
-            return None
-        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "sm_min_mhz": float(min(mhz)),
-                "reasons": sorted(reasons), "samples": len(mhz),
-                "source": "NVML in a separate process, sampled inside the timed region"}
+            why = "; ".join(self.errors + [f"{self.kind}: " + (" | ".join(o for o in other if o)[:300]
+                                                                or "no output in the timed region")])
+            return {"unavailable": why}
+        res = {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "sm_min_mhz": float(min(mhz)),
+               "reasons": sorted(reasons), "samples": len(mhz),
+               "source": f"{self.kind} in a separate process, sampled inside the timed region"}
+        if self.errors:
+            res["note"] = "; ".join(self.errors)
+        return res
+
+
+def tensor_peak(peaks, region_s: float):
+    """The tensor-core peak a kernel is compared with: the burst figure for a timed region
+    shorter than a second (the GPU has not yet settled at its power cap), the sustained
+    figure for a seconds-long loop. Returns (TFLOP/s, the MEASURED_PEAKS key used)."""
+    if region_s >= 1.0 and "bf16_tflops_sustained" in peaks:
+        return peaks["bf16_tflops_sustained"], "bf16_tflops_sustained"
+    return peaks["bf16_tflops"], "bf16_tflops"
+
+
+def host_cpu(threads_used: int) -> dict:
+    """The host the CPU baseline ran on: its logical core count and CPU model, and how
+    the oracle used it (numpy's BLAS threads for the matmuls, one thread elsewhere)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu": model,
+            "threads": f"{threads_used} BLAS thread(s) for the projection and gate matmuls; the sequence map, "
+                       f"hash, row gather and conv run as Python loops on one thread"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs
@@ -218,7 +289,11 @@ def run_reference(args, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": prefill_config(args, w, 1),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "timed_tokens_per_step": args.ref_tokens,
+        "timed_sample": f"each step times the first {args.ref_tokens} of the config's {16384} tokens, as a packed "
+                        f"batch of their own; value is those tokens per second",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample,
+                         **host_cpu(threads)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -368,14 +443,13 @@ def main():
     gemm_s = gemm_ms / 1e3 / max(gemm_n, 1)
     flops = 2.0 * D * H * T
     achieved_tf = flops / gemm_s / 1e12
-    # the GEMM runs back to back in a loop long enough to reach the power cap: compare it with
-    # the sustained bf16 figure (fp16 and bf16 share the nominal dense rate, ratio 1)
-    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_tf, peak_name = tensor_peak(peaks, ms / 1e3)
     roofline = {"kernel": "gemm_kernel (tcgen05 projection + fused gate/conv/residual)", "bound": "tensor",
                 "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
-                "peak_source": f"{peak_kind} bf16_tflops_sustained (timed right after a loop of {args.steps} steps, under the power "
-                               f"cap); fp16 nominal ratio 1.0",
+                "peak_source": f"{peak_kind} {peak_name}: the timed region lasted {ms / 1e3:.3f} s "
+                               f"({'under' if peak_name == 'bf16_tflops' else 'over'} 1 s); fp16 nominal ratio 1.0",
                 "frac_of_burst_peak": achieved_tf / peaks["bf16_tflops"],
+                "frac_of_sustained_peak": achieved_tf / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "traffic": load_traffic("gemm", "prefill", source_hash(GEMM_SOURCES)),
                 "algorithmic_flops_per_launch": flops, "launch_ms": gemm_s * 1e3}
     roofline["library_same_shape"] = library_gemm_same_shape(torch, T, D, H)
@@ -390,6 +464,7 @@ def main():
              "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
              "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"], "launch_ms": e_s * 1e3,
              "algorithmic_bytes_per_launch": embed_bytes,
+             "gathered_row_gbs": (0 if args.path == 4 else T * 2 * D) / e_s / 1e9,
              "traffic": load_traffic("embed", "prefill", source_hash(GATHER_SOURCES))}
     if args.path != 4:
         embed["library_same_bytes"] = library_stream_same_bytes(torch, T, D, peaks["hbm_gbs"])
@@ -406,9 +481,14 @@ def main():
                        "between); per-kernel durations from a following pass of min(K, 300) steps with the "
                        "library's stage events",
     }
-    if clk:
-        line["clocks"] = clk
+    line["clocks"] = clk
     line["gather_roofline"] = gather_bench(ctx, layer, sets, stream, peaks)
+    # the HBM-bound stages beside the projection, in the line's top-level roofline
+    for key, src in (("embed", embed), ("gather", line["gather_roofline"])):
+        roofline[key] = {k: src[k] for k in ("kernel", "bound", "achieved", "peak", "unit", "frac",
+                                             "gathered_row_gbs", "launch_ms", "algorithmic_bytes_per_launch",
+                                             "traffic") if k in src}
+        roofline[key]["gathered_row_frac"] = src["gathered_row_gbs"] / peaks["hbm_gbs"]
 
     if not args.no_extras:
         want = set(args.extras.split(","))
@@ -441,7 +521,7 @@ def main():
             total += s2
         n_runs = min(reps, 20)
         line["cpu_baseline"] = {"value": n_tok * n_runs / total, "unit": "tokens/s", "cores": threads,
-                                "kind": "oracle",
+                                "kind": "oracle", **host_cpu(threads),
                                 "sample": f"first {n_tok} tokens of the prefill batch, {n_runs} run(s), "
                                           f"rows materialised before timing"}
     if rank == 0:
@@ -665,11 +745,11 @@ def gather_fused_bench(ctx, layer, sets, stream, peaks, steps=300):
     T = sets[0]["T"]
     gemm_ms = st["gemm"][0] / max(st["gemm"][1], 1)
     tf = 2.0 * D * H * T / (gemm_ms / 1e3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak, peak_name = tensor_peak(peaks, ms * steps / 1e3)
     return {"workload": "full-scale prefill batches, forward path 4 (gather fused into the projection)",
             "value": T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "stage_ms_per_launch": {k: v[0] / max(v[1], 1) for k, v in st.items() if v[1]},
-            "gemm_tflops": tf, "gemm_frac_of_sustained_peak": tf / peak, "device_status": int(status)}
+            "gemm_tflops": tf, "gemm_frac_of_peak": tf / peak, "peak": peak_name, "device_status": int(status)}
 
 
 def prepared_bench(ctx, layer, sets, stream, steps=200):

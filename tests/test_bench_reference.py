@@ -24,8 +24,10 @@ def test_reference_arm_line():
     assert d["steps"] == 1 and d["warmup"] == 0 and d["n_gpus"] == 1
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["config"]["workload"] and d["config"]["global_batch"] == 16384
+    assert d["timed_tokens_per_step"] == 512 and "512" in d["timed_sample"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert cb["host_cores"] == os.cpu_count() and cb["cpu"] and cb["threads"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0

@@ -77,3 +77,14 @@ def test_the_check_finds_a_planted_name(tmp_path):
     src = tmp_path / "m.py"
     src.write_text("import os\n\ndef f(a):\n    b = a + 1\n    return roofline[b], os.sep\n")
     assert unbound_names(str(src)) == ["m.py:5 f: roofline"]
+
+
+def test_clock_sampler_says_why_it_is_silent():
+    """Without a GPU (or without NVML and nvidia-smi) the sampler reports the reason
+    instead of dropping the clocks key."""
+    import bench
+    c = bench.ClockSampler(0, period_s=0.01)
+    c.start()
+    res = c.stop()
+    assert isinstance(res, dict)
+    assert ("unavailable" in res and res["unavailable"]) or res.get("samples", 0) > 0
