@@ -931,9 +931,37 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
             "decode_us_per_step": 1e3 * d_ms / n_dec, "device_status": int(status)}
 
 
+def timed_each(ctx, stream, fn, n, flush=None):
+    """Mean device time (ms) of fn(i) over n calls, each bracketed by its own CUDA
+    events on `stream`. With `flush`, a write of a buffer larger than L2 runs
+    before every call, outside the events, so each call starts with cold L2 (the
+    state a layer sees after the rest of a model has run)."""
+    torch = ctx["torch"]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    ctx["barrier"]()
+    torch.cuda.synchronize()
+    for i in range(n):
+        if flush is not None:
+            flush.add_(1)
+        ev[i][0].record(stream)
+        fn(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ctx["barrier"]()
+    return ctx["max_over_ranks"](sum(a.elapsed_time(b) for a, b in ev) / n)
+
+
+def l2_flush_buffer(torch):
+    """256 MB, twice the B200's 126 MB L2."""
+    return torch.zeros(64 << 20, dtype=torch.int32, device="cuda")
+
+
 def decode_bench(ctx, layer, stream):
     """Full-scale decode: 8 sequences x 1 new token per step with carried history and
-    conv state; timed eagerly and as a replayed CUDA graph of one ple_decode_step."""
+    conv state. Warm (steps back to back on one batch, W_proj and rows in L2),
+    replayed from CUDA graphs of one and of ten steps, and cold (L2 flushed before
+    every step); the two-call form split into its tokens-only and hidden-dependent
+    halves."""
     torch, ple, pi, bf16_tensor = ctx["torch"], ctx["ple"], ctx["pi"], ctx["bf16_tensor"]
     wd = pi.workload("decode")
     tokens, hidden, hist, conv = pi.decode_batch(wd)
@@ -960,23 +988,89 @@ def decode_bench(ctx, layer, stream):
     stage = ple.ple_get_stage_times(h)
     ple.ple_set_profiling(h, False)
 
-    graph = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream()
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        for i in range(3):
-            eager(i, side)
-    stream.wait_stream(side)
+    graphs = {}
+    for per_graph in (1, 10):
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(3):
+                eager(i, side)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            for i in range(per_graph):
+                eager(i, torch.cuda.current_stream())
+        graphs[per_graph] = timed(ctx, stream, lambda i: graph.replay(), n // per_graph) / (n // per_graph * per_graph)
+        del graph
+
+    flush = l2_flush_buffer(torch)
+    n_cold = 200
+    ms_cold = timed_each(ctx, stream, eager, n_cold, flush)
+
+    def prep(i):
+        ple.ple_decode_prepare(h, tk, B, q, hs, stream)
+
+    def rest(i):
+        ple.ple_decode_step_prepared(h, hd, out, ple.PLE_OUT_BF16, hs, cs, None, stream)
+
+    # the hidden-dependent half after its prepare, both cold: flush, prepare, flush, step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_cold)]
     torch.cuda.synchronize()
-    with torch.cuda.graph(graph):
-        eager(0, torch.cuda.current_stream())
-    ms_graph = timed(ctx, stream, lambda i: graph.replay(), n)
+    for i in range(n_cold):
+        flush.add_(1)
+        ev[i][0].record(stream)
+        prep(i)
+        ev[i][1].record(stream)
+        flush.add_(1)
+        ev[i][2].record(stream)
+        rest(i)
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    prep_cold = sum(e[0].elapsed_time(e[1]) for e in ev) / n_cold
+    rest_cold = sum(e[2].elapsed_time(e[3]) for e in ev) / n_cold
+    for i in range(5):
+        prep(i)
+        rest(i)
+    warm = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_cold)]
+    torch.cuda.synchronize()
+    for i in range(n_cold):
+        warm[i][0].record(stream)
+        prep(i)
+        warm[i][1].record(stream)
+        rest(i)
+        warm[i][2].record(stream)
+    torch.cuda.synchronize()
+    prep_warm = sum(e[0].elapsed_time(e[1]) for e in warm) / n_cold
+    rest_warm = sum(e[1].elapsed_time(e[2]) for e in warm) / n_cold
+    del flush
+    torch.cuda.empty_cache()
+    status = ple.ple_get_error(h)
+
+    peaks, _ = load_peaks()
+    D, H = wd.row_dim, wd.hidden
+    # algorithmic bytes of a step: W_proj fp16, both rows and scales per token, hidden in and
+    # out, conv state in and out, tokens and history
+    step_bytes = D * H * 2 + B * q * (2 * D + 8 + 2 * H + 2 * H + 8) + B * (2 * 3 * H * 4 + 16)
     world = ctx["world"]
+    us = lambda ms: 1e3 * ms  # noqa: E731
     return {"workload": "full-scale decode: 8 sequences x 1 token, 2-token history + 3x2560 conv state",
-            "value": B * q * world * n / (ms_eager / 1e3), "unit": "tokens/s", "us_per_step": 1e3 * ms_eager / n,
-            "graph_value": B * q * world * n / (ms_graph / 1e3), "graph_us_per_step": 1e3 * ms_graph / n,
+            "value": B * q * world * n / (ms_eager / 1e3), "unit": "tokens/s", "us_per_step": us(ms_eager) / n,
+            "graph_us_per_step": us(graphs[1]), "graph10_us_per_step": us(graphs[10]),
+            "cold_us_per_step": us(ms_cold),
+            "cold_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
+                              "achieved_gbs": step_bytes / (ms_cold / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                              "frac": step_bytes / (ms_cold / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            "prepared": {"prepare_us_cold": us(prep_cold), "step_prepared_us_cold": us(rest_cold),
+                         "prepare_us_warm": us(prep_warm), "step_prepared_us_warm": us(rest_warm),
+                         "note": "ple_decode_prepare needs only the tokens and history; ple_decode_step_prepared "
+                                 "(gate, projection, conv, residual, state) is the part that waits for hidden"},
             "stage_us_per_launch": {k: 1e3 * v[0] / max(v[1], 1) for k, v in stage.items() if v[1]},
-            "note": "one batch reused; the graph replays one captured ple_decode_step on static buffers"}
+            "device_status": int(status),
+            "note": "warm: one batch reused, steps back to back (W_proj and rows stay in L2, each step's W_proj "
+                    "copies overlap the previous step under programmatic dependent launch); graph: one or ten "
+                    "captured steps per replay (no overlap across replays); cold: 256 MB written between steps, "
+                    "outside the events"}
 
 
 def mtp_bench(ctx, layer, stream):
@@ -1007,15 +1101,27 @@ def mtp_bench(ctx, layer, stream):
         tk, hd, nc = steps[i % len(steps)]
         ple.ple_decode_step(h, tk, B, q, hd, out, ple.PLE_OUT_BF16, hist, conv, nc, stream)
 
+    hist0, conv0 = hist.clone(), conv.clone()
     for i in range(3):
         step(i)
     n = len(steps)
+    hist.copy_(hist0)
+    conv.copy_(conv0)
     ms = timed(ctx, stream, step, n)
+    # the same 100 steps again from the same state, each after an L2 flush
+    hist.copy_(hist0)
+    conv.copy_(conv0)
+    flush = l2_flush_buffer(torch)
+    ms_cold = timed_each(ctx, stream, step, n, flush)
+    del flush
+    torch.cuda.empty_cache()
+    status = ple.ple_get_error(h)
     committed = int(sum(int(nc.sum()) for _, _, nc in sess["steps"]))
     world = ctx["world"]
     return {"workload": "MTP decode: 64 sequences x 3 tokens/step, 100 steps, 30% shared prefix",
             "value": B * q * world * n / (ms / 1e3), "unit": "tokens/s (processed)",
-            "committed_tokens_per_s": committed * world / (ms / 1e3), "us_per_step": 1e3 * ms / n}
+            "committed_tokens_per_s": committed * world / (ms / 1e3), "us_per_step": 1e3 * ms / n,
+            "cold_us_per_step": 1e3 * ms_cold, "device_status": int(status)}
 
 
 def long_bench(ctx, layer, stream):

@@ -15,6 +15,7 @@ import os
 __all__ = [
     "PleError", "PleConfig", "PleWeights", "PleState", "lib", "ple_create", "ple_destroy",
     "ple_ngram_ids", "ple_gather_rows", "ple_forward", "ple_prepare", "ple_forward_prepared", "ple_decode_step",
+    "ple_decode_prepare", "ple_decode_step_prepared",
     "ple_get_error",
     "ple_status_string", "ple_set_profiling", "ple_get_stage_times", "ple_set_forward_path",
     "ple_launch_count", "ple_wait_selftest", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32",
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
             "ple_decode_step": ([_VP, _VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP, _VP, _VP], _I32),
             "ple_prepare": ([_VP, _VP, _I32, _VP, _I32, _VP, _VP], _I32),
             "ple_forward_prepared": ([_VP, _VP, _VP, _I32, ctypes.POINTER(PleState), _VP], _I32),
+            "ple_decode_prepare": ([_VP, _VP, _I32, _I32, _VP, _VP], _I32),
+            "ple_decode_step_prepared": ([_VP, _VP, _VP, _I32, _VP, _VP, _VP, _VP], _I32),
             "ple_get_error": ([_VP], _I32),
             "ple_status_string": ([_I32], ctypes.c_char_p),
             "ple_set_profiling": ([_VP, _I32], _I32),
@@ -174,6 +177,15 @@ def ple_decode_step(handle, tokens, B, q, hidden, out, out_dtype, hist, conv_sta
                     stream=None) -> None:
     _check(lib().ple_decode_step(handle, _ptr(tokens), B, q, _ptr(hidden), _ptr(out), out_dtype, _ptr(hist),
                                  _ptr(conv_state), _ptr(n_commit), _stream(stream)), "ple_decode_step")
+
+
+def ple_decode_prepare(handle, tokens, B, q, hist, stream=None) -> None:
+    _check(lib().ple_decode_prepare(handle, _ptr(tokens), B, q, _ptr(hist), _stream(stream)), "ple_decode_prepare")
+
+
+def ple_decode_step_prepared(handle, hidden, out, out_dtype, hist, conv_state, n_commit=None, stream=None) -> None:
+    _check(lib().ple_decode_step_prepared(handle, _ptr(hidden), _ptr(out), out_dtype, _ptr(hist), _ptr(conv_state),
+                                          _ptr(n_commit), _stream(stream)), "ple_decode_step_prepared")
 
 
 def ple_get_error(handle) -> int:

@@ -48,20 +48,23 @@ struct ple_handle {
   int64_t partial_elems = 0;
   float* conv0 = nullptr;
   int32_t* hist_new = nullptr;
-  int32_t* status = nullptr;     // [0]: sticky status; [1]: tiles completed by the decode kernel
-  bool decode_small = false;     // the single-kernel decode step fits this shape and device
-  ple::DecodePlan decode_plan{};
-  float* decode_partial = nullptr;
-  int32_t* tile_count = nullptr;
+  int32_t* status = nullptr;     // [0]: sticky status
+  bool decode_proj = false;      // the channel-split decode projection fits this shape and device
+  ple::DecodeProjPlan decode_plan{};
   EncodeTiledFn encode = nullptr;
   CUtensorMap tmap_w{};
-  CUtensorMap tmap_wd{};         // fp16 W_proj, 64 x 16 boxes for the decode kernel
   int32_t forward_path = 0;
   struct Prepared {        // the batch ple_prepare left in the scratch (ids, e, meta, hist_new)
     bool valid = false;
     int32_t T = 0, S = 0;
     bool with_hist = false;
   } prepared;
+  struct PreparedDecode {  // the step ple_decode_prepare left in the scratch (e, meta)
+    bool valid = false;
+    int32_t B = 0, q = 0;
+    const int32_t* tokens = nullptr;
+    const int32_t* hist = nullptr;
+  } prepared_decode;
   bool profiling = false;
   struct Rec { int stage; cudaEvent_t a, b; };
   std::vector<Rec> pending;
@@ -184,8 +187,6 @@ void free_all(ple_handle* h) {
   cudaFree(h->conv0);
   cudaFree(h->hist_new);
   cudaFree(h->status);
-  cudaFree(h->decode_partial);
-  cudaFree(h->tile_count);
   for (auto& r : h->pending) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
@@ -199,19 +200,14 @@ ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q
 
 // Runs prepare + gather + projection (+ combine) for a packed batch.
 ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
-                     int32_t uniform_q, const void* hidden, void* out, ple_out_dtype dtype,
-                     const ple_state* state, int32_t* dec_hist, float* dec_conv, const int32_t* n_commit,
-                     cudaStream_t stream) {
+                     const void* hidden, void* out, ple_out_dtype dtype, const ple_state* state, cudaStream_t stream) {
   const ple_config& c = h->cfg;
-  const bool decode = uniform_q > 0;
-
   ple::PrepareArgs pa{};
   pa.tokens = tokens;
   pa.T = T;
   pa.offsets = offsets;
   pa.S = S;
-  pa.uniform_q = uniform_q;
-  pa.hist = decode ? dec_hist : (state ? state->hist : nullptr);
+  pa.hist = state ? state->hist : nullptr;
   pa.vocab = c.vocab;
   pa.rows0 = c.rows[0];
   pa.rows1 = c.rows[1];
@@ -220,7 +216,7 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   pa.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
   pa.H = c.hidden;
   pa.meta = h->meta;
-  if (!decode && state != nullptr) {
+  if (state != nullptr) {
     pa.conv_in = state->conv;
     pa.conv_copy = h->conv0;
     pa.hist_new = h->hist_new;
@@ -228,14 +224,14 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
   pa.status = h->status;
   // row IDs, gate and the gathered, dequantised rows in one kernel; for the
   // gather-fused projection, IDs and gate only
-  const bool gather = !decode && gather_fused(h, T);
+  const bool gather = gather_fused(h, T);
   h->prepared.valid = false;            // the scratch now holds this call's batch
+  h->prepared_decode.valid = false;
   const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] {
     return launch_embed_for(h, pa, gather ? nullptr : h->e, stream);
   });
   if (st != PLE_OK) return st;
-  return run_projection(h, T, S, uniform_q, hidden, out, dtype, state, dec_hist, dec_conv, tokens, n_commit, gather,
-                        stream);
+  return run_projection(h, T, S, 0, hidden, out, dtype, state, nullptr, nullptr, nullptr, nullptr, gather, stream);
 }
 
 // The projection and everything after it, on the rows, IDs and metadata in the
@@ -338,6 +334,96 @@ ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q
   return run_stage(h, PLE_STAGE_COMBINE, stream, [&] { return ple::launch_combine_forward(ca, stream); });
 }
 
+// The tokens-only half of a decode step: rows into h->e, metadata into h->meta,
+// and the gates when hidden is given.
+ple_status run_decode_embed(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const int32_t* hist,
+                            const void* hidden, cudaStream_t stream) {
+  const ple_config& c = h->cfg;
+  ple::DecodeEmbedArgs a{};
+  a.tokens = tokens;
+  a.B = B;
+  a.q = q;
+  a.hist = hist;
+  a.vocab = c.vocab;
+  a.rows0 = c.rows[0];
+  a.rows1 = c.rows[1];
+  a.magic0 = ple::barrett_magic(c.rows[0]);
+  a.magic1 = ple::barrett_magic(c.rows[1]);
+  a.table = h->w.table;
+  a.blocks = c.table_format == PLE_TABLE_NVFP4 ? h->w.block_scales : nullptr;
+  a.scales = h->w.scales;
+  a.format = c.table_format;
+  a.D = c.row_dim;
+  a.H = c.hidden;
+  a.hidden = static_cast<const __nv_bfloat16*>(hidden);
+  a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
+  a.e = h->e;
+  a.meta = h->meta;
+  a.status = h->status;
+  return run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_decode_embed(a, stream); });
+}
+
+// The hidden-dependent half of a decode step whose rows and metadata are in the
+// scratch: the channel-split projection kernel for steps of up to 16 tokens
+// (unless path 2 forces split-K), else the split-K projection and the decode
+// combine. Without gates in the metadata, a gate kernel writes them first when
+// the kernels after it cannot compute them (split-K, or out aliasing hidden).
+ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const void* hidden, void* out,
+                           ple_out_dtype dtype, int32_t* hist, float* conv_state, const int32_t* n_commit,
+                           bool gate_ready, cudaStream_t stream) {
+  const ple_config& c = h->cfg;
+  const int32_t T = B * q;
+  const bool small = h->forward_path != 2 && h->decode_proj && ple::decode_proj_supported(B, q);
+  if (!gate_ready && (!small || out == hidden)) {
+    ple::PrepareArgs ga{};
+    ga.T = T;
+    ga.S = B;
+    ga.hidden = static_cast<const __nv_bfloat16*>(hidden);
+    ga.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
+    ga.H = c.hidden;
+    ga.meta = h->meta;
+    const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_gate(ga, stream); });
+    if (st != PLE_OK) return st;
+    gate_ready = true;
+  }
+  if (!small)
+    return run_projection(h, T, B, q, hidden, out, dtype, nullptr, hist, conv_state, tokens, n_commit, false, stream);
+  ple::DecodeProjArgs a{};
+  a.tokens = tokens;
+  a.B = B;
+  a.q = q;
+  a.hist = hist;
+  a.conv_state = conv_state;
+  a.n_commit = n_commit;
+  a.w16 = h->w16;
+  a.e = h->e;
+  a.meta = h->meta;
+  a.gate_ready = gate_ready ? 1 : 0;
+  a.hidden = static_cast<const __nv_bfloat16*>(hidden);
+  a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
+  a.conv_w = h->w.conv_w;
+  a.out = out;
+  a.out_f32 = dtype == PLE_OUT_F32 ? 1 : 0;
+  a.H = c.hidden;
+  a.D = c.row_dim;
+  a.status = h->status;
+  return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_decode_proj(a, h->decode_plan, stream); });
+}
+
+// Host checks shared by the decode entry points.
+ple_status check_decode_step(const ple_handle* h, int32_t B, int32_t q, const void* hidden, void* out,
+                             ple_out_dtype out_dtype, const int32_t* hist, const float* conv_state,
+                             const int32_t* n_commit) {
+  if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
+  if (B < 1 || q < 1 || B > h->cfg.max_seqs || static_cast<int64_t>(B) * q > h->cfg.max_tokens) return PLE_ERR_SHAPE;
+  if (hidden == nullptr || out == nullptr || hist == nullptr || conv_state == nullptr) return PLE_ERR_INVALID_ARG;
+  if (out == hidden && out_dtype != PLE_OUT_BF16) return PLE_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(out, 16) || !aligned(hist, 4) || !aligned(conv_state, 16) ||
+      (n_commit && !aligned(n_commit, 4)))
+    return PLE_ERR_ALIGN;
+  return PLE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -417,13 +503,7 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
             cudaMalloc(&h->conv0, static_cast<size_t>(c.max_seqs) * 3 * c.hidden * 4) == cudaSuccess &&
             cudaMalloc(&h->hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess &&
             cudaMalloc(&h->status, 8) == cudaSuccess;
-  h->decode_small = ok && ple::decode_small_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
-  if (h->decode_small) {
-    ok = cudaMalloc(&h->decode_partial,
-                    static_cast<size_t>(ple::decode_small_partial_elems(h->decode_plan, c.hidden)) * 4) == cudaSuccess &&
-         cudaMalloc(&h->tile_count, static_cast<size_t>(c.hidden / 16) * 4) == cudaSuccess &&
-         cudaMemsetAsync(h->tile_count, 0, static_cast<size_t>(c.hidden / 16) * 4, stream) == cudaSuccess;
-  }
+  h->decode_proj = ple::decode_proj_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
   if (!ok) {
     cudaGetLastError();
     free_all(h);
@@ -452,9 +532,6 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   if (cudaMemsetAsync(h->status, 0, 4, stream) != cudaSuccess ||
       !encode_2d(h, &h->tmap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->w16, c.row_dim, c.hidden,
                  static_cast<uint64_t>(c.row_dim) * 2, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      (h->decode_small &&
-       !encode_2d(h, &h->tmap_wd, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->w16, c.row_dim, c.hidden,
-                  static_cast<uint64_t>(c.row_dim) * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) ||
       cudaStreamSynchronize(stream) != cudaSuccess) {
     free_all(h);
     delete h;
@@ -529,7 +606,7 @@ ple_status ple_forward(ple_handle* h, const int32_t* tokens, int32_t T, const in
   if (!aligned(tokens, 4) || !aligned(offsets, 4) || !aligned(hidden, 16) || !aligned(out, 16) ||
       (state && (!aligned(state->hist, 4) || !aligned(state->conv, 16))))
     return PLE_ERR_ALIGN;
-  return run_layer(h, tokens, T, offsets, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, stream);
+  return run_layer(h, tokens, T, offsets, S, hidden, out, out_dtype, state, stream);
 }
 
 ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
@@ -538,6 +615,7 @@ ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const in
   if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
   h->prepared.valid = false;
+  h->prepared_decode.valid = false;
   if (T > 0) {
     if (tokens == nullptr || offsets == nullptr) return PLE_ERR_INVALID_ARG;
     if (!aligned(tokens, 4) || !aligned(offsets, 4) || (hist && !aligned(hist, 4))) return PLE_ERR_ALIGN;
@@ -603,52 +681,43 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
                            cudaStream_t stream) {
   if (h == nullptr) return PLE_ERR_INVALID_ARG;
   if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
-  if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
-  if (B < 1 || q < 1 || B > h->cfg.max_seqs || static_cast<int64_t>(B) * q > h->cfg.max_tokens) return PLE_ERR_SHAPE;
-  if (tokens == nullptr || hidden == nullptr || out == nullptr || hist == nullptr || conv_state == nullptr)
-    return PLE_ERR_INVALID_ARG;
-  if (out == hidden && out_dtype != PLE_OUT_BF16) return PLE_ERR_INVALID_ARG;
-  if (!aligned(tokens, 4) || !aligned(hidden, 16) || !aligned(out, 16) || !aligned(hist, 4) ||
-      !aligned(conv_state, 16) || (n_commit && !aligned(n_commit, 4)))
-    return PLE_ERR_ALIGN;
-  const ple_config& c = h->cfg;
+  const ple_status chk = check_decode_step(h, B, q, hidden, out, out_dtype, hist, conv_state, n_commit);
+  if (chk != PLE_OK) return chk;
+  if (tokens == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(tokens, 4)) return PLE_ERR_ALIGN;
   h->prepared.valid = false;
-  if (h->forward_path != 2 && h->decode_small && out != hidden && ple::decode_small_supported(B, q)) {
-    ple::DecodeSmallArgs a{};
-    a.tokens = tokens;
-    a.B = B;
-    a.q = q;
-    a.hist = hist;
-    a.conv_state = conv_state;
-    a.n_commit = n_commit;
-    a.vocab = c.vocab;
-    a.rows0 = c.rows[0];
-    a.rows1 = c.rows[1];
-    a.magic0 = ple::barrett_magic(c.rows[0]);
-    a.magic1 = ple::barrett_magic(c.rows[1]);
-    a.table = h->w.table;
-    a.blocks = h->w.block_scales;
-    a.scales = h->w.scales;
-    a.nvfp4 = c.table_format == PLE_TABLE_NVFP4 ? 1 : 0;
-    a.heads = c.table_format == PLE_TABLE_E4M3_HEADS ? 1 : 0;
-    a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
-    a.conv_w = h->w.conv_w;
-    a.hidden = static_cast<const __nv_bfloat16*>(hidden);
-    a.out = out;
-    a.out_f32 = out_dtype == PLE_OUT_F32 ? 1 : 0;
-    a.H = c.hidden;
-    a.D = c.row_dim;
-    a.units_max = h->decode_plan.units_max;
-    a.slots = h->decode_plan.slots;
-    a.partial = h->decode_partial;
-    a.tile_count = h->tile_count;
-    a.tiles_done = h->status + 1;
-    a.status = h->status;
-    return run_stage(h, PLE_STAGE_GEMM, stream,
-                     [&] { return ple::launch_decode_small(h->tmap_wd, a, h->decode_plan.grid, stream); });
-  }
-  return run_layer(h, tokens, B * q, nullptr, B, q, hidden, out, out_dtype, nullptr, hist, conv_state, n_commit,
-                   stream);
+  h->prepared_decode.valid = false;
+  const ple_status st = run_decode_embed(h, tokens, B, q, hist, hidden, stream);
+  if (st != PLE_OK) return st;
+  return run_decode_rest(h, tokens, B, q, hidden, out, out_dtype, hist, conv_state, n_commit, true, stream);
+}
+
+ple_status ple_decode_prepare(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const int32_t* hist,
+                              cudaStream_t stream) {
+  if (h == nullptr) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
+  if (B < 1 || q < 1 || B > h->cfg.max_seqs || static_cast<int64_t>(B) * q > h->cfg.max_tokens) return PLE_ERR_SHAPE;
+  if (tokens == nullptr || hist == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(tokens, 4) || !aligned(hist, 4)) return PLE_ERR_ALIGN;
+  h->prepared.valid = false;
+  h->prepared_decode.valid = false;
+  const ple_status st = run_decode_embed(h, tokens, B, q, hist, nullptr, stream);
+  if (st != PLE_OK) return st;
+  h->prepared_decode = {true, B, q, tokens, hist};
+  return PLE_OK;
+}
+
+ple_status ple_decode_step_prepared(ple_handle* h, const void* hidden, void* out, ple_out_dtype out_dtype,
+                                    int32_t* hist, float* conv_state, const int32_t* n_commit, cudaStream_t stream) {
+  if (h == nullptr || !h->prepared_decode.valid) return PLE_ERR_INVALID_ARG;
+  if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
+  const ple_handle::PreparedDecode pd = h->prepared_decode;
+  if (hist != pd.hist) return PLE_ERR_INVALID_ARG;
+  const ple_status chk = check_decode_step(h, pd.B, pd.q, hidden, out, out_dtype, hist, conv_state, n_commit);
+  if (chk != PLE_OK) return chk;
+  h->prepared_decode.valid = false;     // the state advances: the rows belong to this step only
+  return run_decode_rest(h, pd.tokens, pd.B, pd.q, hidden, out, out_dtype, hist, conv_state, n_commit, false,
+                         stream);
 }
 
 ple_status ple_get_error(ple_handle* h) {

@@ -484,4 +484,86 @@ __device__ __forceinline__ void deq_chunk(const RowChunk<NV>& a, const RowChunk<
   else deq16(a.c, b.c, s0, s1, o0, o1);
 }
 
+// ------------------------------------------------------------------ the gate
+constexpr int kEmbedH4 = 10;    // uint4 of h per lane held in registers (hidden <= 2560)
+
+// g = sigmoid(w_gate . h_t) for one token, by one warp, in fp32: lane l adds
+// up the 8-element groups j = l, l + 32, l + 64, ... in that order (the first
+// kEmbedH4 of them already loaded into hv), then a butterfly reduction across
+// the lanes. Every kernel that computes a gate (prefill embed, gate, decode)
+// goes through these functions, which all take the sums in this order, so all
+// paths give the same bits for a token.
+__device__ __forceinline__ void gate_dot8(float& acc, const uint4& hq, const uint4& wq) {
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
+  const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 hf = __bfloat1622float2(h2[q]);
+    const float2 wf = __bfloat1622float2(w2[q]);
+    acc = fmaf(hf.x, wf.x, acc);
+    acc = fmaf(hf.y, wf.y, acc);
+  }
+}
+
+__device__ __forceinline__ float gate_finish(float acc) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return 1.0f / (1.0f + expf(-acc));
+}
+
+__device__ __forceinline__ float gate_warp(const uint4 (&hv)[kEmbedH4], const uint4* hrow, const uint4* wg, int H8,
+                                           int lane) {
+  float acc = 0.f;
+#pragma unroll
+  for (int r = 0; r < kEmbedH4; ++r) {
+    const int j = lane + 32 * r;
+    if (j < H8) gate_dot8(acc, hv[r], __ldg(wg + j));
+  }
+  for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) gate_dot8(acc, ld_stream_v4(hrow + j), __ldg(wg + j));
+  return gate_finish(acc);
+}
+
+// The same gate with the row loaded in two halves of kEmbedH4 / 2 (fewer
+// registers held at once); the sums are taken in the same order.
+__device__ __forceinline__ float gate_warp_halves(const uint4* hrow, const uint4* wg, int H8, int lane) {
+  constexpr int kHalf = kEmbedH4 / 2;
+  float acc = 0.f;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint4 hv[kHalf];
+#pragma unroll
+    for (int r = 0; r < kHalf; ++r) {
+      const int j = lane + 32 * (half * kHalf + r);
+      if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+    }
+#pragma unroll
+    for (int r = 0; r < kHalf; ++r) {
+      const int j = lane + 32 * (half * kHalf + r);
+      if (j < H8) gate_dot8(acc, hv[r], __ldg(wg + j));
+    }
+  }
+  for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) gate_dot8(acc, ld_stream_v4(hrow + j), __ldg(wg + j));
+  return gate_finish(acc);
+}
+
+// The gate of token row hrow (H8 = hidden / 8 groups of 8), loads included.
+__device__ __forceinline__ float gate_warp_row(const uint4* hrow, const uint4* wg, int H8, int lane) {
+  uint4 hv[kEmbedH4];
+#pragma unroll
+  for (int r = 0; r < kEmbedH4; ++r) {
+    const int j = lane + 32 * r;
+    if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+  }
+  return gate_warp(hv, hrow, wg, H8, lane);
+}
+
+// ------------------------------------------------------------------ bulk copies global -> shared
+// One contiguous copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned), completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 }  // namespace ple

@@ -174,47 +174,63 @@ struct DecodeCombineArgs {
 };
 cudaError_t launch_combine_decode(const DecodeCombineArgs& a, cudaStream_t stream);
 
-// A whole decode step in one kernel for B * q <= 16 tokens, one CTA per SM.
-struct DecodeSmallArgs {
+// Decode / speculative-verify steps: B sequences of q tokens (token t = b*q + i).
+//
+// decode_embed_kernel needs only the tokens and the token history: one block
+// per token computes the token's n-gram rows and writes the dequantised rows to
+// e[t] (fp16 [T][D]) and the token's metadata (sequence b, position i, last
+// flag); with hidden set it also writes the gate meta[t].g (through gate_warp).
+struct DecodeEmbedArgs {
   const int32_t* tokens;   // [B][q]
+  int32_t B, q;
+  const int32_t* hist;     // [B][2]: token t-2, t-1 before the step; < 0 = absent
+  int32_t vocab;
+  int64_t rows0, rows1;    // rows per sub-table (E4M3_HEADS: rows0 per head)
+  uint64_t magic0, magic1; // barrett_magic(rows0), barrett_magic(rows1)
+  const uint8_t* table;
+  const uint8_t* blocks;   // NVFP4 block scales (null otherwise)
+  const float* scales;
+  int32_t format;          // ple_table_format
+  int32_t D, H;
+  const __nv_bfloat16* hidden;   // [T][H], or null: the gate is computed later
+  const __nv_bfloat16* w_gate;
+  __half* e;               // [T][D]
+  TokMeta* meta;           // [T]
+  int32_t* status;
+};
+cudaError_t launch_decode_embed(const DecodeEmbedArgs& a, cudaStream_t stream);
+uint64_t barrett_magic(int64_t m);
+
+// decode_proj_kernel, for steps of B * q <= 16 tokens: the projection, gate,
+// conv against the carried state, residual and state commit, one CTA per SM.
+// CTA b owns a contiguous range of 8-channel groups with the whole K, so no
+// partial sums cross CTAs and no CTA waits for another.
+struct DecodeProjArgs {
+  const int32_t* tokens;   // [B][q] (for the new token history)
   int32_t B, q;
   int32_t* hist;           // [B][2] in/out
   float* conv_state;       // [B][3][H] in/out
   const int32_t* n_commit; // [B] or null
-  int32_t vocab;
-  int64_t rows0, rows1;
-  uint64_t magic0, magic1; // barrett_magic(rows0), barrett_magic(rows1)
-  const uint8_t* table;
-  const uint8_t* blocks;   // NVFP4 block scales (null for E4M3)
-  const float* scales;
-  int32_t nvfp4;
-  int32_t heads;           // 1: PLE_TABLE_E4M3_HEADS (rows0 = rows per head sub-table)
+  const __half* w16;       // fp16 W_proj [H][D] (K-major)
+  const __half* e;         // [T][D] from decode_embed_kernel
+  const TokMeta* meta;     // [T]
+  int32_t gate_ready;      // 1: meta[t].g holds the gate; 0: each CTA computes it from hidden
+  const __nv_bfloat16* hidden;
   const __nv_bfloat16* w_gate;
   const float* conv_w;
-  const __nv_bfloat16* hidden;
   void* out;
   int32_t out_f32;
   int32_t H, D;
-  int32_t units_max;       // DecodePlan::units_max
-  int32_t slots;           // DecodePlan::slots
-  float* partial;          // [H / 16][slots][16 * 16] per-CTA tile sums
-  int32_t* tile_count;     // [H / 16], zero between launches
-  int32_t* tiles_done;     // zero between launches
+  int32_t max_groups;      // DecodeProjPlan::max_groups
   int32_t* status;
 };
-// Work split of the single-kernel decode step for a layer shape and SM count.
-struct DecodePlan {
-  int32_t grid;            // CTAs (one per SM)
-  int32_t units_max;       // most 16 x 64 W_proj units one CTA owns
-  int32_t slots;           // most CTAs that share one 16-channel tile
+struct DecodeProjPlan {
+  int32_t grid;            // CTAs (at most one per SM)
+  int32_t max_groups;      // most 8-channel groups one CTA owns
 };
-// False when the shape does not fit the kernel (the step then runs split-K).
-bool decode_small_plan(int32_t H, int32_t D, int32_t num_sms, DecodePlan* plan);
-bool decode_small_supported(int32_t B, int32_t q);
-int64_t decode_small_partial_elems(const DecodePlan& plan, int32_t H);
-uint64_t barrett_magic(int64_t m);
-// tmap_w: fp16 W_proj [H][D], box 64 x 16, 128-byte swizzle.
-cudaError_t launch_decode_small(const CUtensorMap& tmap_w, const DecodeSmallArgs& a, int32_t grid,
-                                cudaStream_t stream);
+// False when the layer shape does not fit the kernel (steps then run split-K).
+bool decode_proj_plan(int32_t H, int32_t D, int32_t num_sms, DecodeProjPlan* plan);
+bool decode_proj_supported(int32_t B, int32_t q);
+cudaError_t launch_decode_proj(const DecodeProjArgs& a, const DecodeProjPlan& plan, cudaStream_t stream);
 
 }  // namespace ple

@@ -224,39 +224,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ id
 }
 
 // ------------------------------------------------------------------ embed (prepare + gather)
-constexpr int kEmbedH4 = 10;    // uint4 of h per lane held in registers (hidden <= 2560)
 constexpr int kEmbedD16 = 5;    // 16-code chunks per lane and row held in registers (rows <= 2560 codes)
-
-// g = sigmoid(w_gate . h_t) for one token, by one warp, in fp32: lane l adds
-// up the 8-element groups j = l, l + 32, l + 64, ... in that order (the first
-// kEmbedH4 of them already loaded into hv), then a butterfly reduction across
-// the lanes. The embed and gate kernels both compute the gate through this
-// function, so ple_forward and ple_prepare + ple_forward_prepared agree bit
-// for bit.
-__device__ __forceinline__ float gate_warp(const uint4 (&hv)[kEmbedH4], const uint4* hrow, const uint4* wg, int H8,
-                                           int lane) {
-  float acc = 0.f;
-  auto dot8 = [&](const uint4& hq, const uint4& wq) {
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hq);
-    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wq);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 hf = __bfloat1622float2(h2[q]);
-      const float2 wf = __bfloat1622float2(w2[q]);
-      acc = fmaf(hf.x, wf.x, acc);
-      acc = fmaf(hf.y, wf.y, acc);
-    }
-  };
-#pragma unroll
-  for (int r = 0; r < kEmbedH4; ++r) {
-    const int j = lane + 32 * r;
-    if (j < H8) dot8(hv[r], __ldg(wg + j));
-  }
-  for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) dot8(ld_stream_v4(hrow + j), __ldg(wg + j));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  return 1.0f / (1.0f + expf(-acc));
-}
 
 // ------------------------------------------------------------------ gate (after ple_prepare)
 // The gate of a batch whose IDs, rows and metadata ple_prepare left in the
@@ -576,7 +544,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 // gate blocks come first, a warp per token; they stream h and write g with no
 // wait, since h does not depend on the IDs, and so cover the IDs kernel's
 // latency. The gather blocks follow: each waits for the IDs, then a thread
-// dequantises two 16-code chunks of both rows into e. They walk the tokens from
+// dequantises one 16-code chunk of both rows into e. Both kinds of block hold
+// at most 40 registers per thread (the gate loads h in two halves), so six
+// blocks fit on an SM. They walk the tokens from
 // the end, so the first tokens' rows are the last written and still in L2 when
 // the projection starts on them. A gather block waiting for the IDs grid means
 // this grid completes only after that one, which the projection relies on; a
@@ -584,7 +554,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 constexpr int kIdsThreads = 256;
 constexpr int kSplitThreads = 256;
 constexpr int kSplitGateTokens = kSplitThreads / 32;          // tokens per gate block
-constexpr int kSplitGatherChunks = 2 * kSplitThreads;         // 16-code chunks per gather block
+constexpr int kSplitGatherChunks = kSplitThreads;             // 16-code chunks per gather block
+constexpr int kSplitBlocksPerSm = 6;                          // 40 registers per thread
 constexpr int kSplitMinTokens = 4096;                        // below this the one-kernel form is faster
 
 __global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs a, int token_blocks) {
@@ -618,7 +589,7 @@ __global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs
 }
 
 template <bool NV>
-__global__ void __launch_bounds__(kSplitThreads, 4)
+__global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
     embed_split_kernel(const PrepareArgs a, const TableRef tab, int32_t D, __half* __restrict__ e, int32_t n_gate,
                        int32_t n_blocks) {
   pdl_launch_dependents();
@@ -627,15 +598,8 @@ __global__ void __launch_bounds__(kSplitThreads, 4)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = static_cast<int>(b) * kSplitGateTokens + warp;
     if (t < a.T) {
-      const int H8 = a.H / 8;
       const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
-      uint4 hv[kEmbedH4];
-#pragma unroll
-      for (int r = 0; r < kEmbedH4; ++r) {
-        const int j = lane + 32 * r;
-        if (j < H8) hv[r] = ld_stream_v4(hrow + j);
-      }
-      const float g = gate_warp(hv, hrow, reinterpret_cast<const uint4*>(a.w_gate), H8, lane);
+      const float g = gate_warp_halves(hrow, reinterpret_cast<const uint4*>(a.w_gate), a.H / 8, lane);
       if (lane == 0) a.meta[t].g = g;
     }
     if (n_blocks == n_gate) pdl_wait();                          // no gather block waits for the IDs grid
@@ -643,36 +607,21 @@ __global__ void __launch_bounds__(kSplitThreads, 4)
   }
   pdl_wait();                                                    // the row IDs
   const int D16 = D / 16;
-  const int64_t n_chunks = static_cast<int64_t>(a.T) * D16;
-  const int64_t base = (n_blocks - 1 - b) * kSplitGatherChunks + threadIdx.x;
-  RowChunk<NV> ca[2], cb[2];
-  float sa[2], sb[2];
-  int64_t idx[2];
-  // both chunks' loads first, then both dequantisations
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    idx[u] = base + u * kSplitThreads;
-    if (idx[u] < n_chunks) {
-      const int32_t t = static_cast<int32_t>(idx[u] / D16);
-      const int c = static_cast<int>(idx[u] - static_cast<int64_t>(t) * D16);
-      const int2 id = reinterpret_cast<const int2*>(a.ids)[t];
-      const int64_t row0 = id.x, row1 = a.rows0 + id.y;
-      ca[u] = load_chunk<NV>(tab.codes, tab.blocks, row0, D, c);
-      cb[u] = load_chunk<NV>(tab.codes, tab.blocks, row1, D, c);
-      sa[u] = __ldg(tab.scales + row0);
-      sb[u] = __ldg(tab.scales + row1);
-    }
-  }
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    if (idx[u] < n_chunks) {
-      uint4 o0, o1;
-      deq_chunk<NV>(ca[u], cb[u], sa[u], sb[u], o0, o1);
-      uint4* dst = reinterpret_cast<uint4*>(e + idx[u] * 16);
-      dst[0] = o0;
-      dst[1] = o1;
-    }
-  }
+  const int64_t idx = (n_blocks - 1 - b) * kSplitGatherChunks + threadIdx.x;
+  if (idx >= static_cast<int64_t>(a.T) * D16) return;
+  const int32_t t = static_cast<int32_t>(idx / D16);
+  const int c = static_cast<int>(idx - static_cast<int64_t>(t) * D16);
+  const int2 id = reinterpret_cast<const int2*>(a.ids)[t];
+  const int64_t row0 = id.x, row1 = a.rows0 + id.y;
+  const RowChunk<NV> ca = load_chunk<NV>(tab.codes, tab.blocks, row0, D, c);
+  const RowChunk<NV> cb = load_chunk<NV>(tab.codes, tab.blocks, row1, D, c);
+  const float sa = __ldg(tab.scales + row0);
+  const float sb = __ldg(tab.scales + row1);
+  uint4 o0, o1;
+  deq_chunk<NV>(ca, cb, sa, sb, o0, o1);
+  uint4* dst = reinterpret_cast<uint4*>(e + idx * 16);
+  dst[0] = o0;
+  dst[1] = o1;
 }
 
 // ------------------------------------------------------------------ bounded-wait self-test

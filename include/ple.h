@@ -210,6 +210,32 @@ ple_status ple_decode_step(ple_handle* handle, const int32_t* tokens, int32_t B,
                            int32_t* hist, float* conv_state, const int32_t* n_commit,
                            cudaStream_t stream);
 
+/* The decode step in two calls, for callers that know a step's tokens before
+ * its hidden states. The n-gram IDs and the row lookup need no hidden state
+ * (DGX Spark report, section "n-gram embedding 是一条附加的条件记忆路径"), and
+ * the SSD-stream model card ("Qwen3.8 Flash-Next NVFP4 - SSD Stream", section
+ * "技术细节") fetches the rows before the model reaches the block that uses
+ * them. ple_decode_prepare takes the tokens [B][q] and the token history
+ * hist [B][2] that ple_decode_step would take, and leaves the step's
+ * dequantised rows and per-token metadata in the handle's scratch.
+ * ple_decode_step_prepared then takes the rest of ple_decode_step's arguments
+ * and runs the gate, the projection, the conv, the residual and the state
+ * update. Together they give ple_decode_step's result bit for bit.
+ *   - hist must be the buffer ple_decode_prepare read, unchanged in between;
+ *     ple_decode_step_prepared updates it. Another pointer gives
+ *     PLE_ERR_INVALID_ARG.
+ *   - tokens must stay valid and unchanged until ple_decode_step_prepared has
+ *     run: it reads them for the new token history.
+ *   - ple_decode_step_prepared consumes the prepared step. ple_forward,
+ *     ple_prepare, ple_decode_step and another ple_decode_prepare discard it.
+ *     Without a prepared step the call returns PLE_ERR_INVALID_ARG.
+ *   - The two calls may use different streams; ordering them (an event) is the
+ *     caller's job. */
+ple_status ple_decode_prepare(ple_handle* handle, const int32_t* tokens, int32_t B, int32_t q, const int32_t* hist,
+                              cudaStream_t stream);
+ple_status ple_decode_step_prepared(ple_handle* handle, const void* hidden, void* out, ple_out_dtype out_dtype,
+                                    int32_t* hist, float* conv_state, const int32_t* n_commit, cudaStream_t stream);
+
 /* ---- lookup without allocation ------------------------------------------
  * The pages have no counterpart of this entry point; it exists for callers of
  * this library that cannot allocate device memory where they run the layer:
@@ -258,10 +284,13 @@ const char* ple_status_string(ple_status status);
 /* Kernel stages of the library, in launch order within a call. In
  * ple_forward and ple_decode_step the PREPARE stage also gathers and
  * dequantises the rows, except on the gather-fused path, where the GEMM stage
- * does. PREPARE is one fused kernel, or, for a batch of 4,096 tokens or more,
- * a row-ID kernel followed by the gate-and-gather kernel. ple_prepare and the
- * gate kernel of ple_forward_prepared count as PREPARE too. GATHER counts
- * ple_gather_rows. */
+ * does. In ple_forward, PREPARE is one fused kernel, or, for a batch of 4,096
+ * tokens or more, a row-ID kernel followed by the gate-and-gather kernel. In
+ * a decode step it is the kernel of the step's tokens (rows, metadata, gates),
+ * and for a step of up to 16 tokens GEMM is one kernel that also does the
+ * gate, conv, residual and state (no COMBINE). ple_prepare, ple_decode_prepare
+ * and the gate kernels of the prepared forms count as PREPARE too. GATHER
+ * counts ple_gather_rows. */
 enum { PLE_STAGE_PREPARE = 0, PLE_STAGE_GATHER = 1, PLE_STAGE_GEMM = 2, PLE_STAGE_COMBINE = 3,
        PLE_NUM_STAGES = 4 };
 
@@ -286,9 +315,10 @@ ple_status ple_get_stage_times(ple_handle* handle, float* ms, int64_t* launches)
  * tables, SM-pair tiles, row_dim >= 128; elsewhere path 4 runs as
  * path 1). Paths 1 and 4 give identical bits; path 4 is never chosen
  * automatically, because on B200 it is slower (each token's rows are
- * dequantised once per 256-channel tile inside the tensor-bound kernel). For ple_decode_step: steps of B * q <= 16 tokens with
- * out != hidden run as one kernel unless path is 2, which forces the split-K
- * path. */
+ * dequantised once per 256-channel tile inside the tensor-bound kernel). For ple_decode_step: steps of B * q <= 16 tokens
+ * run the channel-split projection kernel (every CTA owns whole output
+ * channels, no partial sums cross CTAs) unless path is 2, which forces the
+ * split-K projection and its combine kernel. */
 ple_status ple_set_forward_path(ple_handle* handle, int32_t path);
 
 /* Total number of kernels the handle has launched since creation. */

@@ -3,11 +3,11 @@ graphs) replays to the same bits as eager launches.
 
 Every call is stream-ordered and does its host work (argument checks, tensor
 maps, launch planning) at capture time; the kernels keep no state between
-launches that a replay could see stale (the single-kernel decode step resets
-its tile counters itself). Four forms are captured: a decode step (one
-kernel under programmatic dependent launch), an MTP-style decode step on the
-split-K path, a prefill on SM-pair tiles and a small forward on the split-K
-path (projection then combine).
+launches that a replay could see stale. Four forms are captured: a decode step
+(the tokens kernel, then the channel-split projection under programmatic
+dependent launch), an MTP-style decode step on the split-K path, a prefill on
+SM-pair tiles and a small forward on the split-K path (projection then
+combine).
 """
 import numpy as np
 import pytest

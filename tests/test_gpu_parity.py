@@ -685,10 +685,10 @@ def test_forward_mid_in_place(mid_layer):
 
 
 def test_decode_mid_in_place(mid_layer):
-    """out == hidden: every CTA of the single-kernel step reads whole hidden rows
-    for the gates, so an in-place step runs the split-K kernels; it must equal
-    the out-of-place split-K step bit for bit and stay within tolerance of the
-    single-kernel one."""
+    """out == hidden: the tokens kernel computes the gates before the projection
+    writes anything, and each CTA of the projection reads hidden only at its own
+    channels, so an in-place step equals the out-of-place step bit for bit (on
+    the channel-split kernel and on the split-K path alike)."""
     from tests.gpu_common import MID
     B, q = 8, 1
     rng = np.random.default_rng(77)
@@ -696,31 +696,32 @@ def test_decode_mid_in_place(mid_layer):
     hid = pi.hidden_bf16(rng, B * q, MID.hidden)
     hist = rng.integers(-1, MID.vocab, (B, 2)).astype(np.int32)
     conv = rng.standard_normal((B, 3, MID.hidden)).astype(np.float32)
-    single, h_s, c_s = gpu_decode(mid_layer, toks, hid, hist, conv, out_dtype=0)      # bf16 bits
-    ple.ple_set_forward_path(mid_layer.handle, 2)
-    split, _, _ = gpu_decode(mid_layer, toks, hid, hist, conv, out_dtype=0)
-    ple.ple_set_forward_path(mid_layer.handle, 0)
-    h = dev_bf16(hid)
-    hs = dev_i32(hist)
-    cs = torch.from_numpy(np.ascontiguousarray(conv, np.float32)).cuda()
-    ple.ple_decode_step(mid_layer.handle, dev_i32(toks), B, q, h, h, 0, hs, cs)
-    torch.cuda.synchronize()
-    assert ple.ple_get_error(mid_layer.handle) == 0
-    assert np.array_equal(to_bits(h), split)
-    assert np.array_equal(hs.cpu().numpy(), h_s)
-    assert_close(cs.cpu().numpy(), c_s, "in-place decode state")
     W = mid_layer.host_weights
     ref = O.ple_decode_step(toks, hid, W.w_proj, W.w_gate, W.conv_w, mid_layer.host_table, MID.rows_per_order,
                             hist, conv)
-    assert_bf16_close(to_bits(h), ref["out"])
-    assert_bf16_close(single, ref["out"])
+    for path in (0, 2):
+        ple.ple_set_forward_path(mid_layer.handle, path)
+        try:
+            apart, h_a, c_a = gpu_decode(mid_layer, toks, hid, hist, conv, out_dtype=0)      # bf16 bits
+            h = dev_bf16(hid)
+            hs = dev_i32(hist)
+            cs = torch.from_numpy(np.ascontiguousarray(conv, np.float32)).cuda()
+            ple.ple_decode_step(mid_layer.handle, dev_i32(toks), B, q, h, h, 0, hs, cs)
+            torch.cuda.synchronize()
+        finally:
+            ple.ple_set_forward_path(mid_layer.handle, 0)
+        assert ple.ple_get_error(mid_layer.handle) == 0
+        assert np.array_equal(to_bits(h), apart), path
+        assert np.array_equal(hs.cpu().numpy(), h_a)
+        assert np.array_equal(cs.cpu().numpy(), c_a)
+        assert_bf16_close(apart, ref["out"])
 
 
-# ----------------------------------------------------------------------------- decode: single-kernel path
+# ----------------------------------------------------------------------------- decode: channel-split projection
 @pytest.mark.parametrize("shape", [(1, 1), (8, 1), (5, 3), (16, 1), (2, 8), (6, 3), (3, 7)])
 def test_decode_paths_tiny(tiny_layer, shape):
-    """B * q <= 16 runs the single-kernel step, larger steps the split-K path; both
-    match the oracle and each other (path 2 forces split-K)."""
+    """B * q <= 16 runs the channel-split projection kernel, larger steps the split-K
+    path; both match the oracle and each other (path 2 forces split-K)."""
     w = tiny_layer.w
     B, q = shape
     rng = np.random.default_rng(B * 100 + q)
