@@ -47,7 +47,7 @@ def parse_args():
     ap.add_argument("--sets", type=int, default=3, help="rotating input sets")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the e2e, decode and clocks measurements")
-    ap.add_argument("--extras", default="e2e,decode,mtp,long,nvfp4,heads,prepared,gather_fused",
+    ap.add_argument("--extras", default="e2e,decode,mtp,long,nvfp4,heads,prepared,pipelined,gather_fused",
                     help="comma-separated extra lines to measure (for profiling one of them alone)")
     ap.add_argument("--ref-tokens", type=int, default=512, help="tokens per reference-arm step")
     ap.add_argument("--path", type=int, default=0,
@@ -376,7 +376,7 @@ def main():
     w0 = pi.workload("prefill")
     w = w0 if args.table_rows <= 0 else pi.Workload("prefill", w0.vocab, args.table_rows, w0.row_dim, w0.hidden,
                                                       w0.table_seed, w0.seed, w0.extra)
-    layer = DeviceLayer(w, max_tokens=16384, max_seqs=64)
+    layer = DeviceLayer(w, max_tokens=16384, max_seqs=64, prepare_slots=2)
     h = layer.handle
     H, D = w.hidden, w.row_dim
 
@@ -506,6 +506,8 @@ def main():
             line["heads"] = heads_bench(ctx, sets, stream, peaks)
         if "prepared" in want:
             line["prepared"] = prepared_bench(ctx, layer, sets, stream)
+        if "pipelined" in want:
+            line["pipelined"] = pipelined_bench(ctx, layer, sets, stream)
         if "gather_fused" in want:
             line["gather_fused"] = gather_fused_bench(ctx, layer, sets, stream, peaks)
 
@@ -798,6 +800,50 @@ def prepared_bench(ctx, layer, sets, stream, steps=200):
                     "is the part that waits for the hidden states"}
 
 
+def pipelined_bench(ctx, layer, sets, stream, steps=300):
+    """The headline batches as a stream with two in flight (ple_prepare_slot /
+    ple_forward_prepared_slot): batch i + 1's IDs and rows are prepared into the
+    other slot on a side stream while batch i's gate, projection and epilogue run
+    on the main stream. Each batch is fresh sequences, so a prepare waits only
+    for its slot to be free. Device time from the main stream's events around the
+    whole stream of batches, max over ranks."""
+    torch, ple = ctx["torch"], ctx["ple"]
+    h = layer.handle
+    side = torch.cuda.Stream()
+
+    def run(n):
+        prepared = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event() for _ in range(n)]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        side.wait_event(start)
+        for i in range(n):
+            s = sets[i % len(sets)]
+            slot = i % 2
+            if i >= 2:
+                side.wait_event(done[i - 2])
+            ple.ple_prepare_slot(h, slot, s["tokens"], s["T"], s["offsets"], s["S"], None, side)
+            prepared[i].record(side)
+            stream.wait_event(prepared[i])
+            ple.ple_forward_prepared_slot(h, slot, s["hidden"], s["out"], ple.PLE_OUT_BF16, None, stream)
+            done[i].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    run(6)
+    ctx["barrier"]()
+    ms = ctx["max_over_ranks"](run(steps))
+    ctx["barrier"]()
+    status = ple.ple_get_error(h)
+    T = sets[0]["T"]
+    world = ctx["world"]
+    return {"workload": "full-scale prefill batches, two in flight (prepare of the next batch on a side stream)",
+            "value": T * world * steps / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms / steps,
+            "device_status": int(status)}
+
+
 def heads_bench(ctx, sets, stream, peaks, steps=300):
     """The multi-head row layout (PLE_TABLE_E4M3_HEADS: 16 lookups of 160-byte rows
     per token, 16 sub-tables of 20,000,096 rows, the same 51.2 GB): the headline
@@ -1029,6 +1075,18 @@ def decode_bench(ctx, layer, stream):
     torch.cuda.synchronize()
     prep_cold = sum(e[0].elapsed_time(e[1]) for e in ev) / n_cold
     rest_cold = sum(e[2].elapsed_time(e[3]) for e in ev) / n_cold
+    # the hidden-dependent half right after its prepare, from a cold L2: flush, prepare, step
+    # (the prepare also pulls W_proj into L2, as it would ahead of the hidden states)
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_cold)]
+    torch.cuda.synchronize()
+    for i in range(n_cold):
+        flush.add_(1)
+        prep(i)
+        ev2[i][0].record(stream)
+        rest(i)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    rest_after_prep = sum(e[0].elapsed_time(e[1]) for e in ev2) / n_cold
     for i in range(5):
         prep(i)
         rest(i)
@@ -1062,6 +1120,7 @@ def decode_bench(ctx, layer, stream):
                               "achieved_gbs": step_bytes / (ms_cold / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                               "frac": step_bytes / (ms_cold / 1e3) / 1e9 / peaks["hbm_gbs"]},
             "prepared": {"prepare_us_cold": us(prep_cold), "step_prepared_us_cold": us(rest_cold),
+                         "step_prepared_us_after_cold_prepare": us(rest_after_prep),
                          "prepare_us_warm": us(prep_warm), "step_prepared_us_warm": us(rest_warm),
                          "note": "ple_decode_prepare needs only the tokens and history; ple_decode_step_prepared "
                                  "(gate, projection, conv, residual, state) is the part that waits for hidden"},

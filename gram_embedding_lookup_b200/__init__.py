@@ -15,7 +15,7 @@ import os
 __all__ = [
     "PleError", "PleConfig", "PleWeights", "PleState", "lib", "ple_create", "ple_destroy",
     "ple_ngram_ids", "ple_gather_rows", "ple_forward", "ple_prepare", "ple_forward_prepared", "ple_decode_step",
-    "ple_decode_prepare", "ple_decode_step_prepared",
+    "ple_decode_prepare", "ple_decode_step_prepared", "ple_prepare_slot", "ple_forward_prepared_slot",
     "ple_get_error",
     "ple_status_string", "ple_set_profiling", "ple_get_stage_times", "ple_set_forward_path",
     "ple_launch_count", "ple_wait_selftest", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32",
@@ -46,7 +46,7 @@ class PleError(RuntimeError):
 class PleConfig(ctypes.Structure):
     _fields_ = [("vocab", ctypes.c_int32), ("hidden", ctypes.c_int32), ("row_dim", ctypes.c_int32),
                 ("max_tokens", ctypes.c_int32), ("max_seqs", ctypes.c_int32), ("table_format", ctypes.c_int32),
-                ("rows", ctypes.c_int64 * 2)]
+                ("prepare_slots", ctypes.c_int32), ("rows", ctypes.c_int64 * 2)]
 
 
 class PleWeights(ctypes.Structure):
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "ple_prepare": ([_VP, _VP, _I32, _VP, _I32, _VP, _VP], _I32),
             "ple_forward_prepared": ([_VP, _VP, _VP, _I32, ctypes.POINTER(PleState), _VP], _I32),
             "ple_decode_prepare": ([_VP, _VP, _I32, _I32, _VP, _VP], _I32),
+            "ple_prepare_slot": ([_VP, _I32, _VP, _I32, _VP, _I32, _VP, _VP], _I32),
+            "ple_forward_prepared_slot": ([_VP, _I32, _VP, _VP, _I32, ctypes.POINTER(PleState), _VP], _I32),
             "ple_decode_step_prepared": ([_VP, _VP, _VP, _I32, _VP, _VP, _VP, _VP], _I32),
             "ple_get_error": ([_VP], _I32),
             "ple_status_string": ([_I32], ctypes.c_char_p),
@@ -177,6 +179,20 @@ def ple_decode_step(handle, tokens, B, q, hidden, out, out_dtype, hist, conv_sta
                     stream=None) -> None:
     _check(lib().ple_decode_step(handle, _ptr(tokens), B, q, _ptr(hidden), _ptr(out), out_dtype, _ptr(hist),
                                  _ptr(conv_state), _ptr(n_commit), _stream(stream)), "ple_decode_step")
+
+
+def ple_prepare_slot(handle, slot, tokens, T, offsets, S, hist=None, stream=None) -> None:
+    _check(lib().ple_prepare_slot(handle, slot, _ptr(tokens), T, _ptr(offsets), S, _ptr(hist), _stream(stream)),
+           "ple_prepare_slot")
+
+
+def ple_forward_prepared_slot(handle, slot, hidden, out, out_dtype, state=None, stream=None) -> None:
+    st = None
+    if state is not None:
+        hist, conv = state
+        st = ctypes.byref(PleState(_ptr(hist), _ptr(conv)))
+    _check(lib().ple_forward_prepared_slot(handle, slot, _ptr(hidden), _ptr(out), out_dtype, st, _stream(stream)),
+           "ple_forward_prepared_slot")
 
 
 def ple_decode_prepare(handle, tokens, B, q, hist, stream=None) -> None:

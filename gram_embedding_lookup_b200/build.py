@@ -19,7 +19,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
           "-Xptxas", "-v"]
 
-LIBPLE_SOURCES = ["ple_api.cu", "ple_kernels.cu", "ple_gemm.cu", "ple_decode.cu", "ple_static.cu"]
+LIBPLE_SOURCES = ["ple_api.cu", "ple_kernels.cu", "ple_gemm.cu", "ple_decode.cu", "ple_mtp.cu", "ple_static.cu"]
 LIBPLE = os.path.join(PKG, "libple.so")
 LIBSYNTH = os.path.join(ROOT, "ple_inputs", "libple_synth.so")
 SYNTH_SOURCES = [os.path.join(ROOT, "ple_inputs", "csrc", "ple_synth.cu")]

@@ -41,24 +41,38 @@ struct ple_handle {
   int device = 0;
   int num_sms = 148;
   __half* w16 = nullptr;
-  __half* e = nullptr;
-  int32_t* ids = nullptr;
-  ple::TokMeta* meta = nullptr;
+  // the batch scratch (rows, IDs, metadata, new history): set 0 serves
+  // ple_forward, the decode steps and prepare slot 0; set 1 (with
+  // prepare_slots == 2) only prepare slot 1
+  struct Scratch {
+    __half* e = nullptr;
+    int32_t* ids = nullptr;
+    ple::TokMeta* meta = nullptr;
+    int32_t* hist_new = nullptr;
+  } scratch[2];
+  __half*& e = scratch[0].e;
+  int32_t*& ids = scratch[0].ids;
+  ple::TokMeta*& meta = scratch[0].meta;
+  int32_t*& hist_new = scratch[0].hist_new;
   float* partial = nullptr;
   int64_t partial_elems = 0;
   float* conv0 = nullptr;
-  int32_t* hist_new = nullptr;
   int32_t* status = nullptr;     // [0]: sticky status
   bool decode_proj = false;      // the channel-split decode projection fits this shape and device
   ple::DecodeProjPlan decode_plan{};
+  bool mtp = false;              // the split-K decode projection with in-kernel sums fits
+  ple::MtpPlan mtp_plan{};
+  float* mtp_partial = nullptr;  // its split sums
+  int32_t* mtp_counts = nullptr; // its per-tile counters [2][m_tiles], zero between launches
   EncodeTiledFn encode = nullptr;
   CUtensorMap tmap_w{};
   int32_t forward_path = 0;
-  struct Prepared {        // the batch ple_prepare left in the scratch (ids, e, meta, hist_new)
+  struct Prepared {        // the batch ple_prepare left in a scratch set (ids, e, meta, hist_new)
     bool valid = false;
     int32_t T = 0, S = 0;
     bool with_hist = false;
-  } prepared;
+  } prepared_slot[2];
+  Prepared& prepared = prepared_slot[0];
   struct PreparedDecode {  // the step ple_decode_prepare left in the scratch (e, meta)
     bool valid = false;
     int32_t B = 0, q = 0;
@@ -171,22 +185,27 @@ ple::TableRef table_ref(const ple_handle* h) {
 }
 
 cudaError_t launch_embed_for(ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream) {
-  if (heads_layout(h)) return ple::launch_embed_heads(pa, table_ref(h), h->cfg.row_dim, e, stream);
   int kernels = 1;
-  const cudaError_t r = ple::launch_embed(pa, table_ref(h), h->cfg.row_dim, e, h->num_sms, stream, &kernels);
+  const cudaError_t r = heads_layout(h)
+                            ? ple::launch_embed_heads(pa, table_ref(h), h->cfg.row_dim, e, stream, &kernels)
+                            : ple::launch_embed(pa, table_ref(h), h->cfg.row_dim, e, h->num_sms, stream, &kernels);
   h->launches += kernels - 1;           // the stage counts one launch; large batches take two kernels
   return r;
 }
 
 void free_all(ple_handle* h) {
   cudaFree(h->w16);
-  cudaFree(h->e);
-  cudaFree(h->ids);
-  cudaFree(h->meta);
+  for (auto& sc : h->scratch) {
+    cudaFree(sc.e);
+    cudaFree(sc.ids);
+    cudaFree(sc.meta);
+    cudaFree(sc.hist_new);
+  }
   cudaFree(h->partial);
   cudaFree(h->conv0);
-  cudaFree(h->hist_new);
   cudaFree(h->status);
+  cudaFree(h->mtp_partial);
+  cudaFree(h->mtp_counts);
   for (auto& r : h->pending) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
@@ -194,9 +213,10 @@ void free_all(ple_handle* h) {
   for (auto e : h->free_events) cudaEventDestroy(e);
 }
 
-ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q, const void* hidden, void* out,
-                          ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist, float* dec_conv,
-                          const int32_t* tokens, const int32_t* n_commit, bool gather, cudaStream_t stream);
+ple_status run_projection(ple_handle* h, const ple_handle::Scratch& sc, int32_t T, int32_t S, int32_t uniform_q,
+                          const void* hidden, void* out, ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist,
+                          float* dec_conv, const int32_t* tokens, const int32_t* n_commit, bool gather,
+                          cudaStream_t stream);
 
 // Runs prepare + gather + projection (+ combine) for a packed batch.
 ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
@@ -231,23 +251,25 @@ ple_status run_layer(ple_handle* h, const int32_t* tokens, int32_t T, const int3
     return launch_embed_for(h, pa, gather ? nullptr : h->e, stream);
   });
   if (st != PLE_OK) return st;
-  return run_projection(h, T, S, 0, hidden, out, dtype, state, nullptr, nullptr, nullptr, nullptr, gather, stream);
+  return run_projection(h, h->scratch[0], T, S, 0, hidden, out, dtype, state, nullptr, nullptr, nullptr, nullptr, gather,
+                        stream);
 }
 
 // The projection and everything after it, on the rows, IDs and metadata in the
 // handle's scratch (written by the embed kernel, or by ple_prepare plus the gate
 // kernel). gather: the rows are not in the scratch; the projection gathers them
 // from the table by the IDs.
-ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q, const void* hidden, void* out,
-                          ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist, float* dec_conv,
-                          const int32_t* tokens, const int32_t* n_commit, bool gather, cudaStream_t stream) {
+ple_status run_projection(ple_handle* h, const ple_handle::Scratch& sc, int32_t T, int32_t S, int32_t uniform_q,
+                          const void* hidden, void* out, ple_out_dtype dtype, const ple_state* state, int32_t* dec_hist,
+                          float* dec_conv, const int32_t* tokens, const int32_t* n_commit, bool gather,
+                          cudaStream_t stream) {
   const ple_config& c = h->cfg;
   const bool decode = uniform_q > 0;
   const Plan pl = plan_projection(h, T, decode ? 2 : (gather ? 4 : h->forward_path), h->partial_elems);
   if (gather && !(pl.fused && pl.ctas == 2)) return PLE_ERR_UNSUPPORTED;
   ple_status st = PLE_OK;
   CUtensorMap tmap_e{}, tmap_h{}, tmap_o{}, tmap_o_head{};
-  if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->e, c.row_dim, T, static_cast<uint64_t>(c.row_dim) * 2,
+  if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, sc.e, c.row_dim, T, static_cast<uint64_t>(c.row_dim) * 2,
                  kTileK, pl.n_tok / pl.ctas, CU_TENSOR_MAP_SWIZZLE_128B))
     return PLE_ERR_CUDA;
   if (!encode_2d(h, &tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, c.hidden, T,
@@ -275,18 +297,18 @@ ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q
   gp.k_splits = pl.k_splits;
   gp.num_kb = c.row_dim / kTileK;
   gp.fused = pl.fused ? 1 : 0;
-  gp.meta = h->meta;
+  gp.meta = sc.meta;
   gp.conv_w = h->w.conv_w;
   gp.conv0 = (!decode && state) ? h->conv0 : nullptr;
   gp.conv_state = (!decode && state) ? state->conv : nullptr;
   gp.hist_state = (!decode && state) ? state->hist : nullptr;
-  gp.hist_new = h->hist_new;
+  gp.hist_new = sc.hist_new;
   gp.out = out;
   gp.out_f32 = dtype == PLE_OUT_F32 ? 1 : 0;
   gp.partial = h->partial;
   gp.status = h->status;
   if (gather) {
-    gp.ids = reinterpret_cast<const int2*>(h->ids);
+    gp.ids = reinterpret_cast<const int2*>(sc.ids);
     gp.codes = h->w.table;
     gp.scales = h->w.scales;
     gp.rows0 = c.rows[0];
@@ -305,7 +327,7 @@ ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q
     da.H = c.hidden;
     da.k_splits = pl.k_splits;
     da.partial = h->partial;
-    da.meta = h->meta;
+    da.meta = sc.meta;
     da.hidden = static_cast<const __nv_bfloat16*>(hidden);
     da.conv_w = h->w.conv_w;
     da.tokens = tokens;
@@ -322,13 +344,13 @@ ple_status run_projection(ple_handle* h, int32_t T, int32_t S, int32_t uniform_q
   ca.H = c.hidden;
   ca.k_splits = pl.k_splits;
   ca.partial = h->partial;
-  ca.meta = h->meta;
+  ca.meta = sc.meta;
   ca.hidden = static_cast<const __nv_bfloat16*>(hidden);
   ca.conv_w = h->w.conv_w;
   ca.conv0 = gp.conv0;
   ca.conv_state = gp.conv_state;
   ca.hist_state = gp.hist_state;
-  ca.hist_new = h->hist_new;
+  ca.hist_new = sc.hist_new;
   ca.out = out;
   ca.out_f32 = gp.out_f32;
   return run_stage(h, PLE_STAGE_COMBINE, stream, [&] { return ple::launch_combine_forward(ca, stream); });
@@ -359,9 +381,16 @@ ple_status run_decode_embed(ple_handle* h, const int32_t* tokens, int32_t B, int
   a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
   a.e = h->e;
   a.meta = h->meta;
+  a.w16 = h->w16;
+  a.w16_bytes = static_cast<int64_t>(c.hidden) * c.row_dim * 2;
+  a.prefetch_blocks = h->num_sms;
   a.status = h->status;
   return run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_decode_embed(a, stream); });
 }
+
+ple::DecodeProjArgs decode_proj_args(const ple_handle* h, const int32_t* tokens, int32_t B, int32_t q,
+                                     const void* hidden, void* out, ple_out_dtype dtype, int32_t* hist,
+                                     float* conv_state, const int32_t* n_commit);
 
 // The hidden-dependent half of a decode step whose rows and metadata are in the
 // scratch: the channel-split projection kernel for steps of up to 16 tokens
@@ -386,8 +415,50 @@ ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int3
     if (st != PLE_OK) return st;
     gate_ready = true;
   }
+  if (!small && h->forward_path != 2 && h->mtp && T <= ple::kMtpMaxTokens && q <= ple::kMtpMaxQ) {
+    const int n_pad = (T + 15) / 16 * 16;
+    CUtensorMap tmap_e{};
+    if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->e, c.row_dim, T,
+                   static_cast<uint64_t>(c.row_dim) * 2, kTileK, n_pad, CU_TENSOR_MAP_SWIZZLE_128B))
+      return PLE_ERR_CUDA;
+    ple::MtpProjArgs a{};
+    a.tokens = tokens;
+    a.B = B;
+    a.q = q;
+    a.hist = hist;
+    a.conv_state = conv_state;
+    a.n_commit = n_commit;
+    a.meta = h->meta;
+    a.hidden = static_cast<const __nv_bfloat16*>(hidden);
+    a.conv_w = h->w.conv_w;
+    a.out = out;
+    a.out_f32 = dtype == PLE_OUT_F32 ? 1 : 0;
+    a.H = c.hidden;
+    a.m_tiles = h->mtp_plan.m_tiles;
+    a.k_splits = h->mtp_plan.k_splits;
+    a.num_kb = h->mtp_plan.num_kb;
+    a.n_pad = n_pad;
+    a.partial = h->mtp_partial;
+    a.tile_count = h->mtp_counts;
+    a.tile_done = h->mtp_counts + h->mtp_plan.m_tiles;
+    a.status = h->status;
+    return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_mtp_proj(h->tmap_w, tmap_e, a, stream); });
+  }
   if (!small)
-    return run_projection(h, T, B, q, hidden, out, dtype, nullptr, hist, conv_state, tokens, n_commit, false, stream);
+    return run_projection(h, h->scratch[0], T, B, q, hidden, out, dtype, nullptr, hist, conv_state, tokens, n_commit,
+                          false, stream);
+  ple::DecodeProjArgs a = decode_proj_args(h, tokens, B, q, hidden, out, dtype, hist, conv_state, n_commit);
+  a.e = h->e;
+  a.meta = h->meta;
+  a.gate_ready = gate_ready ? 1 : 0;
+  return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_decode_proj(a, h->decode_plan, stream); });
+}
+
+// The arguments of the channel-split decode kernel common to its two forms.
+ple::DecodeProjArgs decode_proj_args(const ple_handle* h, const int32_t* tokens, int32_t B, int32_t q,
+                                     const void* hidden, void* out, ple_out_dtype dtype, int32_t* hist,
+                                     float* conv_state, const int32_t* n_commit) {
+  const ple_config& c = h->cfg;
   ple::DecodeProjArgs a{};
   a.tokens = tokens;
   a.B = B;
@@ -396,9 +467,6 @@ ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int3
   a.conv_state = conv_state;
   a.n_commit = n_commit;
   a.w16 = h->w16;
-  a.e = h->e;
-  a.meta = h->meta;
-  a.gate_ready = gate_ready ? 1 : 0;
   a.hidden = static_cast<const __nv_bfloat16*>(hidden);
   a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
   a.conv_w = h->w.conv_w;
@@ -406,8 +474,18 @@ ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int3
   a.out_f32 = dtype == PLE_OUT_F32 ? 1 : 0;
   a.H = c.hidden;
   a.D = c.row_dim;
+  a.vocab = c.vocab;
+  a.rows0 = c.rows[0];
+  a.rows1 = c.rows[1];
+  a.magic0 = ple::barrett_magic(c.rows[0]);
+  a.magic1 = ple::barrett_magic(c.rows[1]);
+  a.table = h->w.table;
+  a.blocks = c.table_format == PLE_TABLE_NVFP4 ? h->w.block_scales : nullptr;
+  a.scales = h->w.scales;
+  a.format = c.table_format;
+  a.step_count = h->status + 1;
   a.status = h->status;
-  return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_decode_proj(a, h->decode_plan, stream); });
+  return a;
 }
 
 // Host checks shared by the decode entry points.
@@ -451,6 +529,7 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
        c.table_format != PLE_TABLE_E4M3_HEADS) ||
       c.vocab <= 0 || c.hidden <= 0 || c.row_dim <= 0 || c.max_tokens <= 0 || c.max_seqs <= 0)
     return PLE_ERR_INVALID_ARG;
+  if (c.prepare_slots < 0 || c.prepare_slots > 2) return PLE_ERR_INVALID_ARG;
   if (c.hidden % 128 != 0 || c.row_dim % 64 != 0) return PLE_ERR_UNSUPPORTED;
   if (c.table_format == PLE_TABLE_E4M3_HEADS) {
     // 16 head rows of row_dim / 16 codes, a whole number of 16-byte chunks each
@@ -496,14 +575,24 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
 
   const int64_t e_rows = std::max<int64_t>(c.max_tokens, 256);
   bool ok = cudaMalloc(&h->w16, static_cast<size_t>(c.row_dim) * c.hidden * 2) == cudaSuccess &&
-            cudaMalloc(&h->e, static_cast<size_t>(e_rows) * c.row_dim * 2) == cudaSuccess &&
-            cudaMalloc(&h->ids, static_cast<size_t>(c.max_tokens) * ids_per_token(c) * 4) == cudaSuccess &&
-            cudaMalloc(&h->meta, static_cast<size_t>(c.max_tokens) * sizeof(ple::TokMeta)) == cudaSuccess &&
             cudaMalloc(&h->partial, static_cast<size_t>(cap) * 4) == cudaSuccess &&
             cudaMalloc(&h->conv0, static_cast<size_t>(c.max_seqs) * 3 * c.hidden * 4) == cudaSuccess &&
-            cudaMalloc(&h->hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess &&
             cudaMalloc(&h->status, 8) == cudaSuccess;
+  for (int k = 0; k < (c.prepare_slots == 2 ? 2 : 1) && ok; ++k) {
+    ple_handle::Scratch& sc = h->scratch[k];
+    ok = cudaMalloc(&sc.e, static_cast<size_t>(e_rows) * c.row_dim * 2) == cudaSuccess &&
+         cudaMalloc(&sc.ids, static_cast<size_t>(c.max_tokens) * ids_per_token(c) * 4) == cudaSuccess &&
+         cudaMalloc(&sc.meta, static_cast<size_t>(c.max_tokens) * sizeof(ple::TokMeta)) == cudaSuccess &&
+         cudaMalloc(&sc.hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess;
+  }
   h->decode_proj = ple::decode_proj_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
+  h->mtp = ok && c.max_tokens > 16 && ple::mtp_proj_plan(c.hidden, c.row_dim, h->num_sms, &h->mtp_plan);
+  if (h->mtp) {
+    const size_t counts = static_cast<size_t>(2 * h->mtp_plan.m_tiles) * 4;
+    ok = cudaMalloc(&h->mtp_partial, static_cast<size_t>(ple::mtp_partial_elems(h->mtp_plan)) * 4) == cudaSuccess &&
+         cudaMalloc(&h->mtp_counts, counts) == cudaSuccess &&
+         cudaMemsetAsync(h->mtp_counts, 0, counts, stream) == cudaSuccess;
+  }
   if (!ok) {
     cudaGetLastError();
     free_all(h);
@@ -609,17 +698,19 @@ ple_status ple_forward(ple_handle* h, const int32_t* tokens, int32_t T, const in
   return run_layer(h, tokens, T, offsets, S, hidden, out, out_dtype, state, stream);
 }
 
-ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
-                       const int32_t* hist, cudaStream_t stream) {
-  if (h == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+ple_status ple_prepare_slot(ple_handle* h, int32_t slot, const int32_t* tokens, int32_t T, const int32_t* offsets,
+                            int32_t S, const int32_t* hist, cudaStream_t stream) {
+  if (h == nullptr || T < 0 || slot < 0 || slot > 1) return PLE_ERR_INVALID_ARG;
   if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
+  if (h->scratch[slot].e == nullptr) return PLE_ERR_INVALID_ARG;      // slot 1 needs prepare_slots == 2
   if (S < 1 || S > h->cfg.max_seqs || T > h->cfg.max_tokens) return PLE_ERR_SHAPE;
-  h->prepared.valid = false;
-  h->prepared_decode.valid = false;
+  h->prepared_slot[slot].valid = false;
+  if (slot == 0) h->prepared_decode.valid = false;
   if (T > 0) {
     if (tokens == nullptr || offsets == nullptr) return PLE_ERR_INVALID_ARG;
     if (!aligned(tokens, 4) || !aligned(offsets, 4) || (hist && !aligned(hist, 4))) return PLE_ERR_ALIGN;
     const ple_config& c = h->cfg;
+    const ple_handle::Scratch& sc = h->scratch[slot];
     ple::PrepareArgs pa{};
     pa.tokens = tokens;
     pa.T = T;
@@ -629,30 +720,37 @@ ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const in
     pa.vocab = c.vocab;
     pa.rows0 = c.rows[0];
     pa.rows1 = c.rows[1];
-    pa.ids = h->ids;
+    pa.ids = sc.ids;
     pa.hidden = nullptr;                 // the gate waits for ple_forward_prepared
     pa.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
     pa.H = c.hidden;
-    pa.meta = h->meta;
-    pa.hist_new = h->hist_new;
+    pa.meta = sc.meta;
+    pa.hist_new = sc.hist_new;
     pa.status = h->status;
-    const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return launch_embed_for(h, pa, h->e, stream); });
+    const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return launch_embed_for(h, pa, sc.e, stream); });
     if (st != PLE_OK) return st;
   }
-  h->prepared.valid = true;
-  h->prepared.T = T;
-  h->prepared.S = S;
-  h->prepared.with_hist = hist != nullptr;
+  ple_handle::Prepared& pr = h->prepared_slot[slot];
+  pr.valid = true;
+  pr.T = T;
+  pr.S = S;
+  pr.with_hist = hist != nullptr;
   return PLE_OK;
 }
 
-ple_status ple_forward_prepared(ple_handle* h, const void* hidden, void* out, ple_out_dtype out_dtype,
-                                const ple_state* state, cudaStream_t stream) {
-  if (h == nullptr || !h->prepared.valid) return PLE_ERR_INVALID_ARG;
+ple_status ple_prepare(ple_handle* h, const int32_t* tokens, int32_t T, const int32_t* offsets, int32_t S,
+                       const int32_t* hist, cudaStream_t stream) {
+  return ple_prepare_slot(h, 0, tokens, T, offsets, S, hist, stream);
+}
+
+ple_status ple_forward_prepared_slot(ple_handle* h, int32_t slot, const void* hidden, void* out,
+                                     ple_out_dtype out_dtype, const ple_state* state, cudaStream_t stream) {
+  if (h == nullptr || slot < 0 || slot > 1 || !h->prepared_slot[slot].valid) return PLE_ERR_INVALID_ARG;
   if (wrong_device(h)) return PLE_ERR_INVALID_ARG;
   if (out_dtype != PLE_OUT_BF16 && out_dtype != PLE_OUT_F32) return PLE_ERR_INVALID_ARG;
-  if ((state != nullptr) != h->prepared.with_hist) return PLE_ERR_INVALID_ARG;
-  const int32_t T = h->prepared.T, S = h->prepared.S;
+  const ple_handle::Prepared& pr = h->prepared_slot[slot];
+  if ((state != nullptr) != pr.with_hist) return PLE_ERR_INVALID_ARG;
+  const int32_t T = pr.T, S = pr.S;
   if (T == 0) return PLE_OK;
   if (hidden == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
   if (out == hidden && out_dtype != PLE_OUT_BF16) return PLE_ERR_INVALID_ARG;
@@ -660,20 +758,27 @@ ple_status ple_forward_prepared(ple_handle* h, const void* hidden, void* out, pl
   if (!aligned(hidden, 16) || !aligned(out, 16) || (state && (!aligned(state->hist, 4) || !aligned(state->conv, 16))))
     return PLE_ERR_ALIGN;
   const ple_config& c = h->cfg;
+  const ple_handle::Scratch& sc = h->scratch[slot];
   ple::PrepareArgs ga{};
   ga.T = T;
   ga.S = S;
   ga.hidden = static_cast<const __nv_bfloat16*>(hidden);
   ga.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
   ga.H = c.hidden;
-  ga.meta = h->meta;
+  ga.meta = sc.meta;
   if (state != nullptr) {
     ga.conv_in = state->conv;
     ga.conv_copy = h->conv0;
   }
   const ple_status st = run_stage(h, PLE_STAGE_PREPARE, stream, [&] { return ple::launch_gate(ga, stream); });
   if (st != PLE_OK) return st;
-  return run_projection(h, T, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, nullptr, false, stream);
+  return run_projection(h, sc, T, S, 0, hidden, out, out_dtype, state, nullptr, nullptr, nullptr, nullptr, false,
+                        stream);
+}
+
+ple_status ple_forward_prepared(ple_handle* h, const void* hidden, void* out, ple_out_dtype out_dtype,
+                                const ple_state* state, cudaStream_t stream) {
+  return ple_forward_prepared_slot(h, 0, hidden, out, out_dtype, state, stream);
 }
 
 ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const void* hidden, void* out,
@@ -687,6 +792,15 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
   if (!aligned(tokens, 4)) return PLE_ERR_ALIGN;
   h->prepared.valid = false;
   h->prepared_decode.valid = false;
+  if (h->forward_path != 2 && h->decode_proj && ple::decode_proj_supported(B, q) && out != hidden) {
+    // the whole step in one kernel: each CTA hashes the tokens and gathers the
+    // K range of the rows it multiplies, and computes the gates
+    ple::DecodeProjArgs a = decode_proj_args(h, tokens, B, q, hidden, out, out_dtype, hist, conv_state, n_commit);
+    a.e = nullptr;
+    a.meta = nullptr;
+    a.gate_ready = 0;
+    return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_decode_proj(a, h->decode_plan, stream); });
+  }
   const ple_status st = run_decode_embed(h, tokens, B, q, hist, hidden, stream);
   if (st != PLE_OK) return st;
   return run_decode_rest(h, tokens, B, q, hidden, out, out_dtype, hist, conv_state, n_commit, true, stream);

@@ -16,9 +16,11 @@
 //
 //   decode_proj_kernel (T <= 16): one CTA per SM owns a contiguous range of
 //     8-channel groups with the whole K. Its share of W_proj (at most 24 rows
-//     of fp16, 123 KB at D = 2560) is requested by bulk copies before it waits
-//     for the embed kernel (programmatic dependent launch), so the W_proj
-//     stream runs under the embed kernel. After the wait it copies e, takes
+//     of fp16, 123 KB at D = 2560) is requested by 16-byte cp.async from every
+//     lane (each warp copies the K range it multiplies; bulk copies of such
+//     short pieces measured slower) before it waits for the embed kernel
+//     (programmatic dependent launch), so the W_proj stream runs under the
+//     embed kernel. After the wait it copies e the same way, takes
 //     the gates, runs the products on mma.sync m16n8k16 (tokens x channels,
 //     fp16 inputs, fp32 accumulation; eight warps split K and add their sums
 //     in warp order in shared memory), then the conv against the carried
@@ -70,12 +72,36 @@ template <int FMT>
 __global__ void __launch_bounds__(512) decode_embed_kernel(const DecodeEmbedArgs a) {
   constexpr bool NV = FMT == 1;
   pdl_launch_dependents();             // the projection's prologue (its W_proj copies) may start now
-  pdl_wait();                          // tokens, history and hidden may come from the previous kernel
+  if (a.w16 != nullptr && threadIdx.x < 32) {
+    // this block's share of W_proj into L2 (16 KB pieces, one lane each), spread
+    // over every block of the grid, which has a block per SM at least: the
+    // projection after this kernel then reads it from L2, and when the step is
+    // prepared ahead of its hidden states the stream is off the step's path
+    const int64_t pieces = (a.w16_bytes + 16383) / 16384;
+    const int64_t p0 = pieces * blockIdx.x / gridDim.x, p1 = pieces * (blockIdx.x + 1) / gridDim.x;
+    const uint8_t* wb = reinterpret_cast<const uint8_t*>(a.w16);
+    for (int64_t pc = p0 + threadIdx.x; pc < p1; pc += 32) {
+      const int64_t off = pc * 16384;
+      const int64_t left = a.w16_bytes - off;
+      bulk_prefetch_l2(wb + off, static_cast<uint32_t>(left < 16384 ? left : 16384));
+    }
+  }
+  if (static_cast<int>(blockIdx.x) >= a.B * a.q) return;    // a prefetch-only block
   const int t = blockIdx.x;
   const int b = t / a.q, i = t - b * a.q;
   const int lane = threadIdx.x & 31;
   const bool gate_warp0 = a.hidden != nullptr && threadIdx.x < 32;
   const int H8 = a.H / 8;
+  const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+  uint4 wv[kEmbedH4];
+  if (gate_warp0) {                    // w_gate is a weight: load it before the wait
+#pragma unroll
+    for (int r = 0; r < kEmbedH4; ++r) {
+      const int j = lane + 32 * r;
+      if (j < H8) wv[r] = __ldg(wg + j);
+    }
+  }
+  pdl_wait();                          // tokens, history and hidden may come from the previous kernel
   const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
   uint4 hv[kEmbedH4];
   if (gate_warp0) {                    // the gate's loads go out first: they need no row ID
@@ -125,7 +151,7 @@ __global__ void __launch_bounds__(512) decode_embed_kernel(const DecodeEmbedArgs
     }
   }
   if (threadIdx.x < 32) {
-    const float g = gate_warp0 ? gate_warp(hv, hrow, reinterpret_cast<const uint4*>(a.w_gate), H8, lane) : 0.f;
+    const float g = gate_warp0 ? gate_warp_pre(hv, wv, hrow, wg, H8, lane) : 0.f;
     if (lane == 0) {
       TokMeta m;
       m.g = g;
@@ -148,11 +174,15 @@ constexpr int kSmemLimit = 227 * 1024;
 
 struct __align__(16) ProjSmem {
   float red[kPjWarps][kPjMaxGroups][kPjMaxTok][kPjGroup];   // per-warp sums over the warp's K range
-  float res[kPjMaxTok][kPjMaxChan];                         // hidden at this CTA's channels
   float cst[kPjMaxTok][3][kPjMaxChan];                      // carried conv state at this CTA's channels
+  __nv_bfloat16 res[kPjMaxTok][kPjMaxChan];                 // hidden at this CTA's channels
+  TokMeta meta[kPjMaxTok];                                  // gates (prepared steps)
   float g[kPjMaxTok];                                       // gates
-  uint64_t bar_w[kPjWarps];                                 // W_proj pieces of warp w's K range
-  uint64_t bar_e[kPjWarps];                                 // e pieces of warp w's K range
+  int32_t tok[kPjMaxTok];                                   // the step's tokens
+  int32_t hist[kPjMaxTok][2];                               // the token history before the step
+  int32_t nc[kPjMaxTok];                                    // n_commit
+  int64_t rid[kPjMaxTok][2];                                // fused steps: global rows of the two orders
+  int32_t rid16[kPjMaxTok][kHeads];                         // fused steps, multi-head layout
 };
 
 // K-steps (16 values of K) of warp w: [ks_begin(w), ks_begin(w + 1)).
@@ -184,7 +214,11 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// FMT < 0: the rows come from e (decode_embed_kernel); FMT = 0, 1, 2: the
+// kernel gathers them from an E4M3, NVFP4 or multi-head table.
+template <int FMT>
 __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const DecodeProjArgs a) {
+  constexpr bool FUSED = FMT >= 0;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw_s + 127u) & ~127u) - raw_s);
@@ -200,74 +234,179 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
   const int ng = g1 - g0, c0 = g0 * kPjGroup, nch = ng * kPjGroup;
   const int KS = a.D / 16;
   const int kb = ks_begin(warp, KS), ke = ks_begin(warp + 1, KS);
-  const uint32_t piece = static_cast<uint32_t>(ke - kb) * 32u;   // bytes of one row in this warp's K range
-
-  if (tid == 0) {
-    for (int w = 0; w < kPjWarps; ++w) {
-      mbar_init(smem_u32(&sm->bar_w[w]), 1);
-      mbar_init(smem_u32(&sm->bar_e[w]), 1);
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
 
   // ---- 1. before the wait: this warp's K range of the CTA's W_proj rows (constant
-  //         since ple_create), and the conv taps of this thread's items
-  if (piece > 0) {
-    const uint32_t bw = smem_u32(&sm->bar_w[warp]);
-    if (lane == 0) mbar_arrive_expect_tx(bw, piece * nch);
-    __syncwarp();
-    for (int r = lane; r < nch; r += 32)
-      bulk_load(smem_u32(ws + r * ldr + kb * 16), a.w16 + static_cast<int64_t>(c0 + r) * a.D + kb * 16, piece, bw);
+  //         since ple_create), 16-byte cp.async (lane l copies chunks l and l + 32
+  //         of the range of every row), the conv taps of this lane's channel and,
+  //         when the gates are computed here, w_gate. Each warp reads back only the
+  //         W_proj and e it copied.
+  const int kchunks = (ke - kb) * 2;                         // 16-byte chunks of one row in this warp's K range
+  const bool second = lane + 32 < kchunks;
+  {
+    const __half* src = a.w16 + static_cast<int64_t>(c0) * a.D + kb * 16 + lane * 8;
+    uint32_t dst = smem_u32(ws + kb * 16 + lane * 8);
+    if (lane < kchunks) {
+      for (int r = 0; r < nch; ++r, src += a.D, dst += ldr * 2) {
+        cp_async_16(dst, src);
+        if (second) cp_async_16(dst + 512, src + 256);
+      }
+    }
   }
-  const int n_items = a.B * nch;                             // (sequence b, channel c) pairs
-  float4 cw[2];
+  cp_async_commit();
+  // items: (sequence b, channel c), warp w takes sequences w, w + 8, ..., lane c
+  float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane < nch) cw = __ldg(reinterpret_cast<const float4*>(a.conv_w) + c0 + lane);
+  const int H8 = a.H / 8;
+  const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+  uint4 wv[kEmbedH4];
+  if (!a.gate_ready) {
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int it = tid + k * kPjThreads;
-    if (it < n_items) cw[k] = __ldg(reinterpret_cast<const float4*>(a.conv_w) + c0 + it % nch);
+    for (int r = 0; r < kEmbedH4; ++r) {
+      const int j = lane + 32 * r;
+      if (j < H8) wv[r] = __ldg(wg + j);
+    }
   }
   pdl_launch_dependents();
-  pdl_wait();                                                // e, meta, hidden and the state are ready
+  pdl_wait();                                                // tokens, e, meta, hidden and the state are ready
 
-  // ---- 2. e pieces; gates; residual and state at this CTA's channels
-  if (piece > 0) {
-    const uint32_t be = smem_u32(&sm->bar_e[warp]);
-    if (lane == 0) mbar_arrive_expect_tx(be, piece * T);
-    __syncwarp();
-    for (int r = lane; r < T; r += 32)
-      bulk_load(smem_u32(es + r * ldr + kb * 16), a.e + static_cast<int64_t>(r) * a.D + kb * 16, piece, be);
+  // ---- 2. everything the step reads, in one round trip: e (this warp's K range)
+  //         or the row IDs; residual, state, gates, tokens, history and n_commit
+  //         into shared memory by cp.async
+  if constexpr (!FUSED) {
+    if (lane < kchunks) {
+      const __half* src = a.e + kb * 16 + lane * 8;
+      uint32_t dst = smem_u32(es + kb * 16 + lane * 8);
+      for (int r = 0; r < T; ++r, src += a.D, dst += ldr * 2) {
+        cp_async_16(dst, src);
+        if (second) cp_async_16(dst + 512, src + 256);
+      }
+    }
   }
-  for (int it = tid; it < T * nch; it += kPjThreads) {
-    const int t = it / nch, c = it - (it / nch) * nch;
-    sm->res[t][c] = __bfloat162float(a.hidden[static_cast<int64_t>(t) * a.H + c0 + c]);
+  {
+    // hidden at this CTA's channels: ng 16-byte pieces per token
+    for (int x = tid; x < T * ng; x += kPjThreads) {
+      const int t = x / ng, p = x - t * ng;
+      cp_async_16(smem_u32(&sm->res[t][p * 8]), a.hidden + static_cast<int64_t>(t) * a.H + c0 + p * 8);
+    }
+    // carried conv state: 2 ng 16-byte pieces per (sequence, tap)
+    const int pc = 2 * ng;
+    for (int x = tid; x < a.B * 3 * pc; x += kPjThreads) {
+      const int bk = x / pc, p = x - bk * pc;
+      cp_async_16(smem_u32(&sm->cst[bk / 3][bk % 3][p * 4]), a.conv_state + static_cast<int64_t>(bk) * a.H + c0 + p * 4);
+    }
+    if (tid < T) {
+      if (a.gate_ready) cp_async_16(smem_u32(&sm->meta[tid]), a.meta + tid);
+      cp_async_4(smem_u32(&sm->tok[tid]), a.tokens + tid);
+    }
+    if (tid < a.B) {
+      cp_async_4(smem_u32(&sm->hist[tid][0]), a.hist + 2 * tid);
+      cp_async_4(smem_u32(&sm->hist[tid][1]), a.hist + 2 * tid + 1);
+      if (a.n_commit) cp_async_4(smem_u32(&sm->nc[tid]), a.n_commit + tid);
+    }
   }
-  for (int it = tid; it < a.B * 3 * nch; it += kPjThreads) {
-    const int bk = it / nch, c = it - bk * nch;
-    sm->cst[bk / 3][bk % 3][c] = a.conv_state[static_cast<int64_t>(bk) * a.H + c0 + c];
+  cp_async_commit();
+  uint4 hv[kEmbedH4];
+  if (!a.gate_ready && warp < T) {                           // the gate loads need no row ID
+#pragma unroll
+    for (int r = 0; r < kEmbedH4; ++r) {
+      const int j = lane + 32 * r;
+      if (j < H8) hv[r] = ld_stream_v4(reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(warp) * a.H) + j);
+    }
   }
-  if (a.gate_ready) {
-    if (tid < T) sm->g[tid] = a.meta[tid].g;
-  } else {
-    const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+  int32_t ticket = -1;
+  if constexpr (FUSED) {
+    // row IDs: thread t hashes token t (for the multi-head layout, thread (t, head))
+    constexpr int kIdsPerTok = FMT == 2 ? kHeads : 1;
+    if (tid < T * kIdsPerTok) {
+      const int t = tid / kIdsPerTok, hh = tid - t * kIdsPerTok;
+      const int b = t / a.q, i = t - b * a.q;
+      const int32_t tok = a.tokens[t];
+      if (blockIdx.x == 0 && hh == 0 && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
+      auto carried = [](int32_t h) -> uint64_t { return h < 0 ? 0ull : ctx_of(h); };
+      const uint64_t x0 = ctx_of(tok);
+      const uint64_t x1 = i >= 1 ? ctx_of(a.tokens[t - 1]) : carried(a.hist[2 * b + 1]);
+      const uint64_t x2 = i >= 2 ? ctx_of(a.tokens[t - 2]) : (i == 1 ? carried(a.hist[2 * b + 1]) : carried(a.hist[2 * b]));
+      const uint64_t k2 = (x0 * kQ0) ^ (x1 * kQ1);
+      const uint64_t k3 = k2 ^ (x2 * kQ2);
+      if constexpr (FMT == 2) {
+        const uint64_t k = ((hh >> 3) ? k3 : k2) ^ (static_cast<uint64_t>(hh & 7) * kHeadMix);
+        sm->rid16[t][hh] = static_cast<int32_t>(mod_barrett(k ^ (k >> 32), a.rows0, a.magic0));
+      } else {
+        sm->rid[t][0] = static_cast<int64_t>(mod_barrett(k2 ^ (k2 >> 32), a.rows0, a.magic0));
+        sm->rid[t][1] = a.rows0 + static_cast<int64_t>(mod_barrett(k3 ^ (k3 >> 32), a.rows1, a.magic1));
+      }
+    }
+    __syncthreads();                                         // row IDs ready: this CTA has read the history
+    // count this CTA in; the last CTA to arrive writes the new history at the end,
+    // when no CTA of the grid can still read the old one (the ticket is used only then)
+    if (tid == 0) ticket = atomicAdd(a.step_count, 1);
+    // this warp's K range (chunks of 16 codes) of every token's rows, dequantised
+    // into e rows in shared memory: lane l takes tasks l, l + 32, ... of
+    // (token, chunk), all of a batch's loads in flight before any is used
+    constexpr int kBatch = 5;
+    const int nck = ke - kb;
+    const int tasks = T * nck;
+    for (int x0 = 0; x0 < tasks; x0 += 32 * kBatch) {
+      RowChunk<FMT == 1> ra[kBatch], rb[kBatch];
+      float sa[kBatch], sb[kBatch];
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int x = x0 + lane + 32 * r;
+        if (x < tasks) {
+          const int t = x / nck, j = kb + (x - t * nck);
+          if constexpr (FMT == 2) {
+            const int hd = a.D / kHeads, cph = hd / 16, hh = j / cph;
+            const int64_t row = static_cast<int64_t>(hh) * a.rows0 + sm->rid16[t][hh];
+            ra[r].c = ld_stream_v4(a.table + row * hd + (j - hh * cph) * 16);
+            sa[r] = __ldg(a.scales + row);
+          } else {
+            const int64_t r0 = sm->rid[t][0], r1 = sm->rid[t][1];
+            ra[r] = load_chunk<FMT == 1>(a.table, a.blocks, r0, a.D, j);
+            rb[r] = load_chunk<FMT == 1>(a.table, a.blocks, r1, a.D, j);
+            sa[r] = __ldg(a.scales + r0);
+            sb[r] = __ldg(a.scales + r1);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int x = x0 + lane + 32 * r;
+        if (x < tasks) {
+          const int t = x / nck, j = kb + (x - t * nck);
+          uint4 o0, o1;
+          if constexpr (FMT == 2) deq16_one(ra[r].c, sa[r], o0, o1);
+          else deq_chunk<FMT == 1>(ra[r], rb[r], sa[r], sb[r], o0, o1);
+          uint4* dst = reinterpret_cast<uint4*>(es + t * ldr + j * 16);
+          dst[0] = o0;
+          dst[1] = o1;
+        }
+      }
+    }
+  }
+  if (!a.gate_ready) {
     for (int t = warp; t < T; t += kPjWarps) {
-      const float g = gate_warp_row(reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H), wg,
-                                    a.H / 8, lane);
+      const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+      if (t != warp) {
+#pragma unroll
+        for (int r = 0; r < kEmbedH4; ++r) {
+          const int j = lane + 32 * r;
+          if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+        }
+      }
+      const float g = gate_warp_pre(hv, wv, hrow, wg, H8, lane);
       if (lane == 0) sm->g[t] = g;
     }
   }
+  cp_async_wait_all();
+  __syncthreads();                                           // every copy and every e row has landed
+  if (a.gate_ready && tid < T) sm->g[tid] = sm->meta[tid].g;
 
   // ---- 3. products over this warp's K range: tokens (A, rows of e) x channels
   //         (B, rows of W_proj), one accumulator per 8-channel group
   float acc[kPjMaxGroups][4];
 #pragma unroll
   for (int g = 0; g < kPjMaxGroups; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
-  bool ok = true;
-  if (piece > 0) {
-    ok = mbar_wait(smem_u32(&sm->bar_w[warp]), 0) && mbar_wait(smem_u32(&sm->bar_e[warp]), 0);
-    if (!ok && lane == 0) set_status(a.status, PLE_ERR_TIMEOUT);
-  }
-  if (ok) {
+  {
     // ldmatrix.x4 for A: matrix m = lane / 8 covers token rows (m & 1) * 8 + 0..7 and
     // K offset (m >> 1) * 8; rows past T repeat the last token (their sums are unused)
     const int am = lane >> 3;
@@ -276,6 +415,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
     // ldmatrix.x2 for B: lanes 0..15 address channel rows 0..7 at K offsets 0 and 8
     const uint32_t b_addr = smem_u32(ws + (lane & 7) * ldr + kb * 16 + (((lane >> 3) & 1) << 3));
     const uint32_t group_bytes = kPjGroup * ldr * 2;
+#pragma unroll 4
     for (int ks = 0; ks < ke - kb; ++ks) {
       uint32_t a0, a1, a2, a3;
       ldmatrix_x4(a_addr + ks * 32, a0, a1, a2, a3);
@@ -305,56 +445,55 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
 
   // ---- 4. per (sequence b, channel c): sum over the warps in order, gate, conv
   //         against the carried state, residual, state after n_commit[b] tokens
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int it = tid + k * kPjThreads;
-    if (it >= n_items) break;
-    const int b = it / nch, c = it - (it / nch) * nch;
-    const int g = c >> 3, cc = c & 7;
+  if (lane < nch) {
+    const int c = lane, g = c >> 3, cc = c & 7;
     const int ch = c0 + c;
-    int32_t ncb = a.n_commit ? a.n_commit[b] : a.q;
-    if (ncb < 1 || ncb > a.q) {
-      if (c == 0 && blockIdx.x == 0) set_status(a.status, PLE_ERR_RANGE);
-      ncb = max(1, min(ncb, a.q));
-    }
-    float w0 = sm->cst[b][0][c], w1 = sm->cst[b][1][c], w2 = sm->cst[b][2][c];
-    float k0 = w0, k1 = w1, k2 = w2;
-    const float4 cwt = cw[k];
-    for (int i = 0; i < a.q; ++i) {
-      const int t = b * a.q + i;
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < kPjWarps; ++w) v += sm->red[w][g][t][cc];
-      const float u = sm->g[t] * v;
-      const float y = cwt.x * w0 + cwt.y * w1 + cwt.z * w2 + cwt.w * u;
-      w0 = w1;
-      w1 = w2;
-      w2 = u;
-      const int64_t idx = static_cast<int64_t>(t) * a.H + ch;
-      const float o = sm->res[t][c] + y;
-      if (a.out_f32) reinterpret_cast<float*>(a.out)[idx] = o;
-      else reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(o);
-      if (i == ncb - 1) {
-        k0 = w0;
-        k1 = w1;
-        k2 = w2;
+    for (int b = warp; b < a.B; b += kPjWarps) {
+      int32_t ncb = a.n_commit ? sm->nc[b] : a.q;
+      if (ncb < 1 || ncb > a.q) {
+        if (c == 0 && blockIdx.x == 0) set_status(a.status, PLE_ERR_RANGE);
+        ncb = max(1, min(ncb, a.q));
       }
+      float w0 = sm->cst[b][0][c], w1 = sm->cst[b][1][c], w2 = sm->cst[b][2][c];
+      float k0 = w0, k1 = w1, k2 = w2;
+      for (int i = 0; i < a.q; ++i) {
+        const int t = b * a.q + i;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kPjWarps; ++w) v += sm->red[w][g][t][cc];
+        const float u = sm->g[t] * v;
+        const float y = cw.x * w0 + cw.y * w1 + cw.z * w2 + cw.w * u;
+        w0 = w1;
+        w1 = w2;
+        w2 = u;
+        const int64_t idx = static_cast<int64_t>(t) * a.H + ch;
+        const float o = __bfloat162float(sm->res[t][c]) + y;
+        if (a.out_f32) reinterpret_cast<float*>(a.out)[idx] = o;
+        else reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(o);
+        if (i == ncb - 1) {
+          k0 = w0;
+          k1 = w1;
+          k2 = w2;
+        }
+      }
+      float* cs = a.conv_state + static_cast<int64_t>(b) * 3 * a.H + ch;
+      cs[0] = k0;
+      cs[a.H] = k1;
+      cs[2 * a.H] = k2;
     }
-    float* cs = a.conv_state + static_cast<int64_t>(b) * 3 * a.H + ch;
-    cs[0] = k0;
-    cs[a.H] = k1;
-    cs[2 * a.H] = k2;
   }
-  // ---- 5. the new token history: the last two committed tokens (the embed
-  //         kernel, the only reader of the old one, has completed)
-  if (blockIdx.x == 0 && tid < a.B) {
-    const int b = tid;
-    const int32_t ncb = max(1, min(a.n_commit ? a.n_commit[b] : a.q, a.q));
-    const int32_t* tkp = a.tokens + static_cast<int64_t>(b) * a.q;
-    const int32_t n1 = tkp[ncb - 1];
-    const int32_t n0 = ncb >= 2 ? tkp[ncb - 2] : a.hist[2 * b + 1];
-    a.hist[2 * b] = n0;
-    a.hist[2 * b + 1] = n1;
+  // ---- 5. the new token history: the last two committed tokens, written by one
+  //         thread once every reader of the old one is done with it (fused: the
+  //         last CTA past its hashing; otherwise the embed kernel read it)
+  if (tid == 0 && (FUSED ? ticket == static_cast<int32_t>(gridDim.x) - 1 : blockIdx.x == 0)) {
+    for (int b = 0; b < a.B; ++b) {
+      const int32_t ncb = max(1, min(a.n_commit ? sm->nc[b] : a.q, a.q));
+      const int32_t n1 = sm->tok[b * a.q + ncb - 1];
+      const int32_t n0 = ncb >= 2 ? sm->tok[b * a.q + ncb - 2] : sm->hist[b][1];
+      a.hist[2 * b] = n0;
+      a.hist[2 * b + 1] = n1;
+    }
+    if (FUSED) *a.step_count = 0;                            // ready for the next step
   }
 }
 
@@ -378,10 +517,18 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, const 
 uint64_t barrett_magic(int64_t m) { return ~0ull / static_cast<uint64_t>(m); }
 
 cudaError_t launch_decode_embed(const DecodeEmbedArgs& a, cudaStream_t stream) {
+  static PerDeviceOnce configured;
+  const cudaError_t r = configured.run([] {
+    cudaError_t x = prefer_max_shared(decode_embed_kernel<0>);
+    if (x == cudaSuccess) x = prefer_max_shared(decode_embed_kernel<1>);
+    if (x == cudaSuccess) x = prefer_max_shared(decode_embed_kernel<2>);
+    return x;
+  });
+  if (r != cudaSuccess) return r;
   const int T = a.B * a.q;
   const int nch = a.D / 16;
   const int threads = std::min(512, std::max(32, (nch + 31) / 32 * 32));
-  const dim3 grid(T), block(threads);
+  const dim3 grid(a.w16 != nullptr ? std::max(T, a.prefetch_blocks) : T), block(threads);
   if (a.format == PLE_TABLE_E4M3_HEADS) return launch_pdl(decode_embed_kernel<2>, grid, block, 0, a, stream);
   if (a.format == PLE_TABLE_NVFP4) return launch_pdl(decode_embed_kernel<1>, grid, block, 0, a, stream);
   return launch_pdl(decode_embed_kernel<0>, grid, block, 0, a, stream);
@@ -404,13 +551,27 @@ bool decode_proj_supported(int32_t B, int32_t q) { return static_cast<int64_t>(B
 cudaError_t launch_decode_proj(const DecodeProjArgs& a, const DecodeProjPlan& plan, cudaStream_t stream) {
   static PerDeviceOnce configured;
   const cudaError_t e = configured.run([] {
-    return cudaFuncSetAttribute(decode_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    cudaError_t x = cudaSuccess;
+    auto set = [&x](auto kernel) {
+      if (x == cudaSuccess)
+        x = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+      if (x == cudaSuccess) x = prefer_max_shared(kernel);
+    };
+    set(decode_proj_kernel<-1>);
+    set(decode_proj_kernel<0>);
+    set(decode_proj_kernel<1>);
+    set(decode_proj_kernel<2>);
+    return x;
   });
   if (e != cudaSuccess) return e;
   DecodeProjArgs b = a;
   b.max_groups = plan.max_groups;
-  return launch_pdl(decode_proj_kernel, dim3(plan.grid), dim3(kPjThreads),
-                    proj_smem_bytes(plan.max_groups, a.D, a.B * a.q), b, stream);
+  const size_t smem = proj_smem_bytes(plan.max_groups, a.D, a.B * a.q);
+  const dim3 grid(plan.grid), block(kPjThreads);
+  if (a.e != nullptr) return launch_pdl(decode_proj_kernel<-1>, grid, block, smem, b, stream);
+  if (a.format == PLE_TABLE_E4M3_HEADS) return launch_pdl(decode_proj_kernel<2>, grid, block, smem, b, stream);
+  if (a.format == PLE_TABLE_NVFP4) return launch_pdl(decode_proj_kernel<1>, grid, block, smem, b, stream);
+  return launch_pdl(decode_proj_kernel<0>, grid, block, smem, b, stream);
 }
 
 }  // namespace ple

@@ -323,6 +323,8 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
 // ------------------------------------------------------------------ shared-memory loads and stores
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -449,6 +451,12 @@ __device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t ld_stream_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t ld_stream_u8(const void* p) {
   uint16_t v;
   asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(v) : "l"(p));
@@ -523,6 +531,20 @@ __device__ __forceinline__ float gate_warp(const uint4 (&hv)[kEmbedH4], const ui
   return gate_finish(acc);
 }
 
+// The same gate with the first kEmbedH4 groups of w_gate loaded as well (wv):
+// a caller can load the weights before it waits for the previous kernel.
+__device__ __forceinline__ float gate_warp_pre(const uint4 (&hv)[kEmbedH4], const uint4 (&wv)[kEmbedH4],
+                                               const uint4* hrow, const uint4* wg, int H8, int lane) {
+  float acc = 0.f;
+#pragma unroll
+  for (int r = 0; r < kEmbedH4; ++r) {
+    const int j = lane + 32 * r;
+    if (j < H8) gate_dot8(acc, hv[r], wv[r]);
+  }
+  for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) gate_dot8(acc, ld_stream_v4(hrow + j), __ldg(wg + j));
+  return gate_finish(acc);
+}
+
 // The same gate with the row loaded in two halves of kEmbedH4 / 2 (fewer
 // registers held at once); the sums are taken in the same order.
 __device__ __forceinline__ float gate_warp_halves(const uint4* hrow, const uint4* wg, int H8, int lane) {
@@ -555,6 +577,14 @@ __device__ __forceinline__ float gate_warp_row(const uint4* hrow, const uint4* w
     if (j < H8) hv[r] = ld_stream_v4(hrow + j);
   }
   return gate_warp(hv, hrow, wg, H8, lane);
+}
+
+// ------------------------------------------------------------------ L2 prefetch
+// Asks for `bytes` (a multiple of 16, 16-byte aligned address) to be brought
+// into L2; no completion is tracked.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
 }
 
 // ------------------------------------------------------------------ bulk copies global -> shared

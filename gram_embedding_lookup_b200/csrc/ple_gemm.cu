@@ -739,13 +739,18 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmap_w, const CUtensorMap& tmap_
                              cudaStream_t stream) {
   static PerDeviceOnce configured;
   const cudaError_t e = configured.run([] {
-    return cudaFuncSetAttribute(gemm_kernel<CTAS, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+    const cudaError_t x = cudaFuncSetAttribute(gemm_kernel<CTAS, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               kGemmSmemBytes);
+    return x == cudaSuccess ? prefer_max_shared(gemm_kernel<CTAS, GATHER>) : x;
   });
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(Roles<GATHER>::THREADS);
-  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  // what the layout uses (plus the alignment slack), not the per-block maximum:
+  // the few KB left let small kernels of another stream (the next batch's
+  // ple_prepare_slot) share the SMs
+  cfg.dynamicSmemBytes = Cfg<CTAS, GATHER>::SMEM_USED + 1024;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;

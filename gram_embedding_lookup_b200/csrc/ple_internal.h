@@ -36,6 +36,16 @@ class PerDeviceOnce {
   std::atomic<uint64_t> done_{0};
 };
 
+// Every kernel of the library asks for the largest shared-memory carveout, so
+// that a kernel and its programmatic dependent (the projections take up to
+// 227 KB of shared memory) can share an SM: an SM changes its L1/shared split
+// only once it has drained.
+template <typename Kernel>
+cudaError_t prefer_max_shared(Kernel kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              static_cast<int>(cudaSharedmemCarveoutMaxShared));
+}
+
 // The table as the kernels see it (ple_table_format in ple.h).
 struct TableRef {
   const uint8_t* codes;        // E4M3: one byte per element; NVFP4: two E2M1 codes per byte
@@ -79,7 +89,7 @@ cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D,
 // e[t] (the 16 dequantised rows side by side) when e is set; extra blocks do
 // the offsets check and the state work. a.rows0 is the rows per head sub-table.
 cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
-                               cudaStream_t stream);
+                               cudaStream_t stream, int* kernels = nullptr);
 
 // Gather stage of the multi-head layout: ids [T][16] -> e [T][D].
 cudaError_t launch_gather_heads(const int32_t* ids, int32_t T, const TableRef& table, int64_t rows, int32_t D,
@@ -196,6 +206,9 @@ struct DecodeEmbedArgs {
   const __nv_bfloat16* w_gate;
   __half* e;               // [T][D]
   TokMeta* meta;           // [T]
+  const __half* w16;       // fp16 W_proj, prefetched into L2 for the kernel after this one (null: none)
+  int64_t w16_bytes;
+  int32_t prefetch_blocks; // the grid has at least this many blocks (past T: prefetch only)
   int32_t* status;
 };
 cudaError_t launch_decode_embed(const DecodeEmbedArgs& a, cudaStream_t stream);
@@ -204,17 +217,29 @@ uint64_t barrett_magic(int64_t m);
 // decode_proj_kernel, for steps of B * q <= 16 tokens: the projection, gate,
 // conv against the carried state, residual and state commit, one CTA per SM.
 // CTA b owns a contiguous range of 8-channel groups with the whole K, so no
-// partial sums cross CTAs and no CTA waits for another.
+// partial sums cross CTAs and no CTA waits for another. With e null the
+// kernel also computes the row IDs and gathers and dequantises, in each warp,
+// the K range of every token's rows that the warp multiplies (the whole step
+// in one kernel); otherwise it reads the rows decode_embed_kernel wrote.
 struct DecodeProjArgs {
-  const int32_t* tokens;   // [B][q] (for the new token history)
+  const int32_t* tokens;   // [B][q] (the rows of a fused step, and the new token history)
   int32_t B, q;
   int32_t* hist;           // [B][2] in/out
   float* conv_state;       // [B][3][H] in/out
   const int32_t* n_commit; // [B] or null
   const __half* w16;       // fp16 W_proj [H][D] (K-major)
-  const __half* e;         // [T][D] from decode_embed_kernel
+  const __half* e;         // [T][D] from decode_embed_kernel, or null: the kernel gathers the rows itself
   const TokMeta* meta;     // [T]
   int32_t gate_ready;      // 1: meta[t].g holds the gate; 0: each CTA computes it from hidden
+  // the table, for a step whose rows the kernel gathers itself (e null)
+  int32_t vocab;
+  int64_t rows0, rows1;
+  uint64_t magic0, magic1;
+  const uint8_t* table;
+  const uint8_t* blocks;
+  const float* scales;
+  int32_t format;          // ple_table_format
+  int32_t* step_count;     // fused steps: CTAs past their hashing, zero between launches
   const __nv_bfloat16* hidden;
   const __nv_bfloat16* w_gate;
   const float* conv_w;
@@ -232,5 +257,46 @@ struct DecodeProjPlan {
 bool decode_proj_plan(int32_t H, int32_t D, int32_t num_sms, DecodeProjPlan* plan);
 bool decode_proj_supported(int32_t B, int32_t q);
 cudaError_t launch_decode_proj(const DecodeProjArgs& a, const DecodeProjPlan& plan, cudaStream_t stream);
+
+// mtp_proj_kernel, for steps of 17..kMtpMaxTokens tokens after
+// decode_embed_kernel (gates in meta): a split-K tcgen05 projection whose
+// K-split CTAs meet at a per-tile counter, then each adds the splits' sums in
+// order for its share of the sequences and runs gate, conv, residual and state
+// commit. Its CTAs wait for one another, so the grid (m_tiles * k_splits) never
+// exceeds the SM count.
+constexpr int kMtpMaxTokens = 256;
+constexpr int kMtpMaxQ = 16;       // tokens per sequence: a chunk of whole sequences fits the staging area
+constexpr int kMtpMaxSplits = 8;
+struct MtpPlan {
+  int32_t m_tiles;         // hidden / 128
+  int32_t k_splits;        // CTAs per channel tile
+  int32_t num_kb;          // row_dim / 64
+};
+struct MtpProjArgs {
+  const int32_t* tokens;   // [B][q]
+  int32_t B, q;
+  int32_t* hist;           // [B][2] in/out
+  float* conv_state;       // [B][3][H] in/out
+  const int32_t* n_commit; // [B] or null
+  const TokMeta* meta;     // [T]: gates
+  const __nv_bfloat16* hidden;
+  const float* conv_w;
+  void* out;
+  int32_t out_f32;
+  int32_t H;
+  int32_t m_tiles, k_splits, num_kb;
+  int32_t n_pad;           // T rounded up to 16 (the MMA's N)
+  int32_t stages;          // set by the launcher
+  float* partial;          // [m_tiles][k_splits][kMtpMaxTokens][128]
+  int32_t* tile_count;     // [m_tiles], zero between launches
+  int32_t* tile_done;      // [m_tiles], zero between launches
+  int32_t* status;
+};
+bool mtp_proj_plan(int32_t H, int32_t D, int32_t num_sms, MtpPlan* plan);
+int64_t mtp_partial_elems(const MtpPlan& plan);
+// tmap_w: fp16 W_proj [H][D], box 64 x 128, 128-byte swizzle; tmap_e: fp16 e
+// [T][D], box 64 x n_pad, 128-byte swizzle.
+cudaError_t launch_mtp_proj(const CUtensorMap& tmap_w, const CUtensorMap& tmap_e, const MtpProjArgs& a,
+                            cudaStream_t stream);
 
 }  // namespace ple

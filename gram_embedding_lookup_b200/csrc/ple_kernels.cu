@@ -554,10 +554,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 constexpr int kIdsThreads = 256;
 constexpr int kSplitThreads = 256;
 constexpr int kSplitGateTokens = kSplitThreads / 32;          // tokens per gate block
-constexpr int kSplitGatherChunks = kSplitThreads;             // 16-code chunks per gather block
 constexpr int kSplitBlocksPerSm = 6;                          // 40 registers per thread
 constexpr int kSplitMinTokens = 4096;                        // below this the one-kernel form is faster
 
+// FMT: 0 = E4M3 rows (two orders, ids [T][2]), 1 = NVFP4 (the same IDs), 2 = the
+// multi-head layout (ids [T][16], a.rows0 rows per head sub-table).
+template <int FMT>
 __global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs a, int token_blocks) {
   pdl_launch_dependents();
   if (static_cast<int>(blockIdx.x) >= token_blocks) {
@@ -566,13 +568,25 @@ __global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs
   }
   const int t = blockIdx.x * kIdsThreads + threadIdx.x;
   if (t >= a.T) return;
-  int32_t s, pos, last, r0, r1;
+  int32_t s, pos, last;
   sequence_of(a, t, true, s, pos, last);
   uint64_t k2, k3;
   keys_of(a, t, s, pos, true, k2, k3);
-  r0 = static_cast<int32_t>(mod_barrett(fold64(k2), static_cast<uint64_t>(a.rows0), a.magic0));
-  r1 = static_cast<int32_t>(mod_barrett(fold64(k3), static_cast<uint64_t>(a.rows1), a.magic1));
-  reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
+  if constexpr (FMT == 2) {
+    int32_t r[kHeads];
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh) {
+      const uint64_t k = ((hh >> 3) ? k3 : k2) ^ (static_cast<uint64_t>(hh & 7) * kHeadMix);
+      r[hh] = static_cast<int32_t>(mod_barrett(fold64(k), static_cast<uint64_t>(a.rows0), a.magic0));
+    }
+    int4* dst = reinterpret_cast<int4*>(a.ids + static_cast<int64_t>(t) * kHeads);
+#pragma unroll
+    for (int q4 = 0; q4 < kHeads / 4; ++q4) dst[q4] = make_int4(r[4 * q4], r[4 * q4 + 1], r[4 * q4 + 2], r[4 * q4 + 3]);
+  } else {
+    const int32_t r0 = static_cast<int32_t>(mod_barrett(fold64(k2), static_cast<uint64_t>(a.rows0), a.magic0));
+    const int32_t r1 = static_cast<int32_t>(mod_barrett(fold64(k3), static_cast<uint64_t>(a.rows1), a.magic1));
+    reinterpret_cast<int2*>(a.ids)[t] = make_int2(r0, r1);
+  }
   if (a.meta == nullptr) return;
   if (a.hidden == nullptr) {                  // no gate blocks: the gate field is written later, by the gate kernel
     TokMeta m;
@@ -588,7 +602,12 @@ __global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs
   }
 }
 
-template <bool NV>
+// Gather units of a token: E4M3 and the multi-head layout one 16-code chunk per
+// thread; NVFP4 two chunks (16 bytes of packed codes and 2 block-scale bytes
+// per row), so that each load is as wide as an E4M3 thread's.
+template <int FMT> constexpr int kSplitChunksPerThread = FMT == 1 ? 2 : 1;
+
+template <int FMT>
 __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
     embed_split_kernel(const PrepareArgs a, const TableRef tab, int32_t D, __half* __restrict__ e, int32_t n_gate,
                        int32_t n_blocks) {
@@ -606,22 +625,48 @@ __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
     return;
   }
   pdl_wait();                                                    // the row IDs
-  const int D16 = D / 16;
-  const int64_t idx = (n_blocks - 1 - b) * kSplitGatherChunks + threadIdx.x;
-  if (idx >= static_cast<int64_t>(a.T) * D16) return;
-  const int32_t t = static_cast<int32_t>(idx / D16);
-  const int c = static_cast<int>(idx - static_cast<int64_t>(t) * D16);
-  const int2 id = reinterpret_cast<const int2*>(a.ids)[t];
-  const int64_t row0 = id.x, row1 = a.rows0 + id.y;
-  const RowChunk<NV> ca = load_chunk<NV>(tab.codes, tab.blocks, row0, D, c);
-  const RowChunk<NV> cb = load_chunk<NV>(tab.codes, tab.blocks, row1, D, c);
-  const float sa = __ldg(tab.scales + row0);
-  const float sb = __ldg(tab.scales + row1);
-  uint4 o0, o1;
-  deq_chunk<NV>(ca, cb, sa, sb, o0, o1);
-  uint4* dst = reinterpret_cast<uint4*>(e + idx * 16);
-  dst[0] = o0;
-  dst[1] = o1;
+  constexpr int CPT = kSplitChunksPerThread<FMT>;
+  const int units = D / (16 * CPT);                              // per token
+  const int64_t idx = (n_blocks - 1 - b) * kSplitThreads + threadIdx.x;
+  if (idx >= static_cast<int64_t>(a.T) * units) return;
+  const int32_t t = static_cast<int32_t>(idx / units);
+  const int c = static_cast<int>(idx - static_cast<int64_t>(t) * units);
+  uint4* dst = reinterpret_cast<uint4*>(e + idx * 16 * CPT);
+  if constexpr (FMT == 2) {
+    const int hd = D / kHeads, cph = hd / 16, hh = c / cph;
+    const int64_t row = static_cast<int64_t>(hh) * a.rows0 + a.ids[static_cast<int64_t>(t) * kHeads + hh];
+    const uint4 v = ld_stream_v4(tab.codes + row * hd + (c - hh * cph) * 16);
+    uint4 o0, o1;
+    deq16_one(v, __ldg(tab.scales + row), o0, o1);
+    dst[0] = o0;
+    dst[1] = o1;
+  } else {
+    const int2 id = reinterpret_cast<const int2*>(a.ids)[t];
+    const int64_t row0 = id.x, row1 = a.rows0 + id.y;
+    const float sa = __ldg(tab.scales + row0);
+    const float sb = __ldg(tab.scales + row1);
+    if constexpr (FMT == 1) {
+      // elements [32c, 32c + 32): 16 bytes of codes and 2 block-scale bytes per row
+      const uint4 xa = ld_stream_v4(tab.codes + row0 * (D / 2) + 16 * c);
+      const uint4 xb = ld_stream_v4(tab.codes + row1 * (D / 2) + 16 * c);
+      const uint32_t ba = ld_stream_u16(tab.blocks + row0 * (D / 16) + 2 * c);
+      const uint32_t bb = ld_stream_u16(tab.blocks + row1 * (D / 16) + 2 * c);
+      uint4 o0, o1, o2, o3;
+      deq16_nv(make_uint2(xa.x, xa.y), make_uint2(xb.x, xb.y), ba & 0xFFu, bb & 0xFFu, sa, sb, o0, o1);
+      deq16_nv(make_uint2(xa.z, xa.w), make_uint2(xb.z, xb.w), ba >> 8, bb >> 8, sa, sb, o2, o3);
+      dst[0] = o0;
+      dst[1] = o1;
+      dst[2] = o2;
+      dst[3] = o3;
+    } else {
+      const RowChunk<false> ca = load_chunk<false>(tab.codes, tab.blocks, row0, D, c);
+      const RowChunk<false> cb = load_chunk<false>(tab.codes, tab.blocks, row1, D, c);
+      uint4 o0, o1;
+      deq_chunk<false>(ca, cb, sa, sb, o0, o1);
+      dst[0] = o0;
+      dst[1] = o1;
+    }
+  }
 }
 
 // ------------------------------------------------------------------ bounded-wait self-test
@@ -741,6 +786,31 @@ __global__ void __launch_bounds__(128) combine_decode_kernel(const DecodeCombine
   }
 }
 
+// The kernels that run in a chain with a projection or under programmatic
+// dependent launch take the largest shared-memory carveout (prefer_max_shared).
+cudaError_t configure_chain_kernels() {
+  static PerDeviceOnce configured;
+  return configured.run([] {
+    cudaError_t r = cudaSuccess;
+    auto set = [&r](auto kernel) {
+      if (r == cudaSuccess) r = prefer_max_shared(kernel);
+    };
+    set(ids_meta_kernel<0>);
+    set(ids_meta_kernel<1>);
+    set(ids_meta_kernel<2>);
+    set(embed_split_kernel<0>);
+    set(embed_split_kernel<1>);
+    set(embed_split_kernel<2>);
+    set(embed_pipe_kernel<false>);
+    set(embed_pipe_kernel<true>);
+    set(embed_heads_kernel);
+    set(gate_kernel);
+    set(combine_forward_kernel);
+    set(combine_decode_kernel);
+    return r;
+  });
+}
+
 }  // namespace
 
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
@@ -755,37 +825,47 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// The embed of a batch of kSplitMinTokens or more as two launches (all table
+// formats): the IDs kernel, then the gate and gather blocks as its dependent.
+template <int FMT>
+cudaError_t launch_embed_split(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
+                               cudaStream_t stream, int* kernels) {
+  const PrepareArgs am = with_magic(a);
+  const int token_blocks = (a.T + kIdsThreads - 1) / kIdsThreads;
+  int sblocks = 1;
+  if (a.conv_in != nullptr) {
+    const int64_t want = (static_cast<int64_t>(a.S) * 3 * a.H / 4 + kIdsThreads - 1) / kIdsThreads;
+    sblocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
+  }
+  ids_meta_kernel<FMT><<<token_blocks + sblocks, kIdsThreads, 0, stream>>>(am, token_blocks);
+  cudaError_t r = cudaGetLastError();
+  if (r != cudaSuccess) return r;
+  const int64_t units = static_cast<int64_t>(a.T) * (D / (16 * kSplitChunksPerThread<FMT>));
+  const int64_t n_gate = a.hidden != nullptr && a.meta != nullptr ? (a.T + kSplitGateTokens - 1) / kSplitGateTokens : 0;
+  const int64_t n_gather = e != nullptr ? (units + kSplitThreads - 1) / kSplitThreads : 0;
+  if (n_gate + n_gather == 0) return cudaSuccess;
+  if (kernels != nullptr) *kernels = 2;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_gate + n_gather));
+  cfg.blockDim = dim3(kSplitThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int32_t ng = static_cast<int32_t>(n_gate), nblk = static_cast<int32_t>(n_gate + n_gather);
+  return cudaLaunchKernelEx(&cfg, embed_split_kernel<FMT>, am, table, D, e, ng, nblk);
+}
+
 cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
                          cudaStream_t stream, int* kernels) {
   if (kernels != nullptr) *kernels = 1;
+  const cudaError_t cfg_err = configure_chain_kernels();
+  if (cfg_err != cudaSuccess) return cfg_err;
   if (a.T >= kSplitMinTokens) {
-    // large batches: IDs kernel, then gate and gather blocks as its dependent
-    const PrepareArgs am = with_magic(a);
-    const int token_blocks = (a.T + kIdsThreads - 1) / kIdsThreads;
-    int sblocks = 1;
-    if (a.conv_in != nullptr) {
-      const int64_t want = (static_cast<int64_t>(a.S) * 3 * a.H / 4 + kIdsThreads - 1) / kIdsThreads;
-      sblocks = static_cast<int>(want < 1 ? 1 : (want > 148 ? 148 : want));
-    }
-    ids_meta_kernel<<<token_blocks + sblocks, kIdsThreads, 0, stream>>>(am, token_blocks);
-    cudaError_t r = cudaGetLastError();
-    if (r != cudaSuccess) return r;
-    const int64_t n_gate = a.hidden != nullptr && a.meta != nullptr ? (a.T + kSplitGateTokens - 1) / kSplitGateTokens : 0;
-    const int64_t n_gather = e != nullptr ? (static_cast<int64_t>(a.T) * (D / 16) + kSplitGatherChunks - 1) / kSplitGatherChunks : 0;
-    if (n_gate + n_gather == 0) return cudaSuccess;
-    if (kernels != nullptr) *kernels = 2;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(n_gate + n_gather));
-    cfg.blockDim = dim3(kSplitThreads);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const int32_t ng = static_cast<int32_t>(n_gate), nblk = static_cast<int32_t>(n_gate + n_gather);
-    if (table.nvfp4) return cudaLaunchKernelEx(&cfg, embed_split_kernel<true>, am, table, D, e, ng, nblk);
-    return cudaLaunchKernelEx(&cfg, embed_split_kernel<false>, am, table, D, e, ng, nblk);
+    if (table.nvfp4) return launch_embed_split<1>(a, table, D, e, stream, kernels);
+    return launch_embed_split<0>(a, table, D, e, stream, kernels);
   }
   const bool state = a.conv_in != nullptr || a.hist_new != nullptr;
   // small batches spread over the SMs: a few tokens per CTA, no warp taking two in turn
@@ -798,7 +878,11 @@ cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D,
 }
 
 cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, int* kernels) {
+  if (kernels != nullptr) *kernels = 1;
+  const cudaError_t cfg_err = configure_chain_kernels();
+  if (cfg_err != cudaSuccess) return cfg_err;
+  if (a.T >= kSplitMinTokens && a.ids != nullptr) return launch_embed_split<2>(a, table, D, e, stream, kernels);
   const int token_blocks = (a.T + 7) / 8;
   int sblocks = 1;
   if (a.conv_in != nullptr) {
@@ -822,6 +906,8 @@ cudaError_t launch_wait_selftest(int32_t* status, long long limit_cycles, cudaSt
 }
 
 cudaError_t launch_gate(const PrepareArgs& a, cudaStream_t stream) {
+  const cudaError_t cfg_err = configure_chain_kernels();
+  if (cfg_err != cudaSuccess) return cfg_err;
   const int token_blocks = (a.T + 7) / 8;
   int state_blocks = 0;
   if (a.conv_in != nullptr) {
@@ -855,6 +941,8 @@ cudaError_t launch_convert_w(const __nv_bfloat16* w, int32_t D, int32_t H, __hal
 // for the projection before they read anything it writes.
 template <typename Kernel, typename Args>
 cudaError_t launch_after_projection(Kernel kernel, dim3 grid, const Args& a, cudaStream_t stream) {
+  const cudaError_t cfg_err = configure_chain_kernels();
+  if (cfg_err != cudaSuccess) return cfg_err;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(128);

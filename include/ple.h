@@ -95,7 +95,9 @@ typedef enum { PLE_TABLE_E4M3 = 0, PLE_TABLE_NVFP4 = 1, PLE_TABLE_E4M3_HEADS = 2
 
 /* Sizes fixed at creation. hidden % 128 == 0, row_dim % 64 == 0,
  * 0 < rows[n] < 2^31. max_tokens bounds T of every call (and B*q of a decode
- * step); max_seqs bounds S (and B). */
+ * step); max_seqs bounds S (and B). prepare_slots: 0 or 1 = one batch scratch;
+ * 2 = a second one for ple_prepare_slot / ple_forward_prepared_slot slot 1
+ * (max_tokens * row_dim * 2 bytes more). */
 typedef struct {
   int32_t vocab;
   int32_t hidden;
@@ -103,6 +105,7 @@ typedef struct {
   int32_t max_tokens;
   int32_t max_seqs;
   int32_t table_format;      /* ple_table_format */
+  int32_t prepare_slots;     /* 0, 1 or 2 */
   int64_t rows[2];           /* rows of the bigram (0) and trigram (1) sub-tables */
 } ple_config;
 
@@ -197,6 +200,26 @@ ple_status ple_prepare(ple_handle* handle, const int32_t* tokens, int32_t T,
                        const int32_t* offsets, int32_t S, const int32_t* hist, cudaStream_t stream);
 ple_status ple_forward_prepared(ple_handle* handle, const void* hidden, void* out,
                                 ple_out_dtype out_dtype, const ple_state* state, cudaStream_t stream);
+
+/* The same two calls on one of two batch slots, so that the next batch can be
+ * prepared while the current one is projected: the Thor report's SSD tier
+ * ("第四条路：让 47.68 GiB PLE 留在 SSD") and the SSD-stream model card
+ * ("技术细节") fetch rows while earlier work runs and wait only when fetching
+ * is slower. ple_prepare / ple_forward_prepared are slot 0. Slot 1 exists when
+ * the handle was created with prepare_slots == 2 (else PLE_ERR_INVALID_ARG).
+ *   - Each slot holds its own rows, IDs, metadata and new token history; a
+ *     slot's prepared batch stays usable until the next ple_prepare_slot on
+ *     the same slot. ple_forward, ple_prepare and the decode calls use slot
+ *     0's scratch and discard slot 0's batch only.
+ *   - ple_prepare_slot(s) may run on another stream at the same time as
+ *     ple_forward_prepared_slot(1 - s); the caller orders the calls on the
+ *     same slot (events), and runs the hidden-dependent calls (forward,
+ *     forward_prepared, decode steps) on one stream at a time.
+ *   - Results equal ple_forward's bit for bit. */
+ple_status ple_prepare_slot(ple_handle* handle, int32_t slot, const int32_t* tokens, int32_t T,
+                            const int32_t* offsets, int32_t S, const int32_t* hist, cudaStream_t stream);
+ple_status ple_forward_prepared_slot(ple_handle* handle, int32_t slot, const void* hidden, void* out,
+                                     ple_out_dtype out_dtype, const ple_state* state, cudaStream_t stream);
 
 /* One decode / speculative-verify step: B sequences with q new tokens each.
  * tokens int32 [B][q]; hidden bf16 [B*q][hidden]; out [B*q][hidden];

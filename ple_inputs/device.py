@@ -33,7 +33,7 @@ class DeviceLayer:
     rows_per_order rows of row_dim / 16 codes)."""
 
     def __init__(self, w: Workload, max_tokens: int, max_seqs: int, weights=None, stream=None,
-                 table_format: int = 0):
+                 table_format: int = 0, prepare_slots: int = 1):
         self.w = w
         self.table_format = table_format
         R, D, H = w.rows_per_order, w.row_dim, w.hidden
@@ -62,6 +62,7 @@ class DeviceLayer:
         cfg = ple.PleConfig()
         cfg.vocab, cfg.hidden, cfg.row_dim = w.vocab, H, D
         cfg.max_tokens, cfg.max_seqs, cfg.table_format = max_tokens, max_seqs, table_format
+        cfg.prepare_slots = prepare_slots
         cfg.rows[0] = R
         cfg.rows[1] = R
         self.config = cfg

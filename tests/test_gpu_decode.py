@@ -91,8 +91,12 @@ def test_decode_prepared_tiny(tiny_layer, shape):
     _check(tiny_layer, shape, seed=shape[0] * 10 + shape[1])
 
 
-@pytest.mark.parametrize("shape,path", [((8, 1), 0), ((4, 3), 0), ((16, 1), 0), ((8, 1), 2), ((64, 3), 0)])
+@pytest.mark.parametrize("shape,path", [((8, 1), 0), ((4, 3), 0), ((16, 1), 0), ((8, 1), 2), ((64, 3), 0),
+                                        ((6, 3), 0), ((64, 4), 0), ((32, 9), 0), ((64, 3), 2)])
 def test_decode_prepared_mid(mid_layer, shape, path):
+    """Steps of up to 16 tokens run the channel-split kernel, 17 to 256 tokens the
+    split-K kernel with in-kernel sums (256 = its largest N, with fewer stages), more
+    than 256 the split-K projection and combine kernel, as does path 2 for any size."""
     _check(mid_layer, shape, seed=shape[0] * 7 + shape[1] + path, path=path)
 
 
@@ -122,7 +126,7 @@ def test_decode_prepared_full(full_layer):  # noqa: F811
     assert_close(a[2][seqs], ref["conv_out"], "full MTP state")
 
 
-@pytest.mark.parametrize("shape", [(1, 1), (3, 1), (1, 3)])
+@pytest.mark.parametrize("shape", [(1, 1), (3, 1), (1, 3), (64, 3)])
 def test_decode_step_bits_repeat(full_layer, shape):  # noqa: F811
     """Every sum in a decode step is taken in a fixed order: 50 runs of the same step
     (full scale, where one token's gate spans many lanes and warps) give the same bits."""

@@ -105,12 +105,24 @@ def test_forward_graph_replay_matches_eager(mid_layer, lengths, path):  # noqa: 
         ple.ple_set_forward_path(L.handle, 0)
 
 
-def test_split_decode_step_graph_replay_matches_eager(mid_layer):  # noqa: F811
-    """A decode step of more than 16 tokens (an MTP-style step with n_commit) takes
-    the split-K path: embed, projection and combine, three kernels chained by
-    programmatic dependent launch. Captured once, it replays to the same bits."""
+@pytest.mark.parametrize("path,kernels", [(0, 2), (2, 3)])
+def test_split_decode_step_graph_replay_matches_eager(mid_layer, path, kernels):  # noqa: F811
+    """A decode step of more than 16 tokens (an MTP-style step with n_commit): the
+    tokens kernel, then the split-K projection with its sums, gate, conv and state
+    in one kernel (automatic path), or the split-K projection and a combine kernel
+    (path 2), chained by programmatic dependent launch. Captured once, it replays
+    to the same bits."""
     from ple_inputs.device import bf16_tensor
     L = mid_layer
+    ple.ple_set_forward_path(L.handle, path)
+    try:
+        _split_decode_graph(L, kernels)
+    finally:
+        ple.ple_set_forward_path(L.handle, 0)
+
+
+def _split_decode_graph(L, kernels):
+    from ple_inputs.device import bf16_tensor
     B, q = 24, 3
     rng = np.random.default_rng(32)
     tok = rng.integers(0, MID.vocab, (B, q)).astype(np.int32)
@@ -124,7 +136,7 @@ def test_split_decode_step_graph_replay_matches_eager(mid_layer):  # noqa: F811
     ple.ple_decode_step(L.handle, _i32(tok), B, q, bf16_tensor(hid), ref, 1, hs, cs, nc)
     torch.cuda.synchronize()
     assert ple.ple_get_error(L.handle) == 0
-    assert ple.ple_launch_count(L.handle) - n0 == 3
+    assert ple.ple_launch_count(L.handle) - n0 == kernels
     s_tok, s_hid = _i32(tok), bf16_tensor(hid)
     s_hs, s_cs = _i32(hist0), torch.from_numpy(conv0).cuda()
     out = torch.empty_like(ref)

@@ -191,3 +191,108 @@ def test_two_launch_embed_ragged_state_full(full_layer):
     assert np.array_equal(_f32bits(got), _f32bits(out))
     assert np.array_equal(got_st[0], st[0])
     assert np.array_equal(_f32bits(got_st[1]), _f32bits(st[1]))
+
+
+# ----------------------------------------------------------------------------- two prepare slots
+@pytest.fixture(scope="module")
+def mid_two_slots():
+    from ple_inputs.device import DeviceLayer
+    import oracle as O
+    L = DeviceLayer(MID, max_tokens=4096, max_seqs=64, prepare_slots=2)
+    codes, scales = MID.table().full()
+    L.host_table = O.ArrayTable(codes, scales)
+    yield L
+    L.close()
+
+
+def test_two_slots_in_flight(mid_two_slots):
+    """A stream of batches with two in flight: batch i + 1 is prepared into the other
+    slot on a side stream while batch i is projected on the main stream, the state
+    carried from batch to batch. Every output and the final state equal ple_forward's
+    run of the same batches one after the other, bit for bit."""
+    L = mid_two_slots
+    rng = np.random.default_rng(404)
+    H = MID.hidden
+    batches = []
+    for lengths in ([300, 1, 2000], [5, 700, 12], [1500, 3, 1], [64, 64, 64], [1, 1, 900]):
+        T = sum(lengths)
+        batches.append((rng.integers(0, MID.vocab, T).astype(np.int32),
+                        np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32), pi.hidden_bf16(rng, T, H)))
+    hist0, conv0 = _state(rng, 3, H, MID.vocab)
+
+    # one call per batch
+    hs, cs = dev_i32(hist0), torch.from_numpy(conv0).cuda()
+    ref = []
+    for tk, of, hd in batches:
+        out = torch.empty(len(tk), H, dtype=torch.bfloat16, device="cuda")
+        ple.ple_forward(L.handle, dev_i32(tk), len(tk), dev_i32(of), 3, dev_bf16(hd), out, 0, (hs, cs))
+        ref.append(out)
+    torch.cuda.synchronize()
+    ref_state = (hs.cpu().numpy(), cs.cpu().numpy())
+
+    # two slots: the prepare of batch i + 1 reads the history that the projection of
+    # batch i writes, so the side stream waits for it; rows then overlap the projection
+    hs2, cs2 = dev_i32(hist0), torch.from_numpy(conv0).cuda()
+    side, main = torch.cuda.Stream(), torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    main.wait_stream(torch.cuda.current_stream())
+    dev = [(dev_i32(tk), dev_i32(of), dev_bf16(hd)) for tk, of, hd in batches]
+    torch.cuda.synchronize()
+    outs = [torch.empty(len(tk), H, dtype=torch.bfloat16, device="cuda") for tk, _, _ in batches]
+    prepared = [torch.cuda.Event() for _ in batches]
+    done = [torch.cuda.Event() for _ in batches]
+    hist_ready = torch.cuda.Event()
+    hist_ready.record(main)
+    for i, (tk, of, hd) in enumerate(dev):
+        slot = i % 2
+        with torch.cuda.stream(side):
+            side.wait_event(hist_ready)
+            if i >= 2:
+                side.wait_event(done[i - 2])            # the slot's previous batch is projected
+            ple.ple_prepare_slot(L.handle, slot, tk, len(batches[i][0]), of, 3, hs2, side)
+            prepared[i].record(side)
+        with torch.cuda.stream(main):
+            main.wait_event(prepared[i])
+            ple.ple_forward_prepared_slot(L.handle, slot, hd, outs[i], 0, (hs2, cs2), main)
+            done[i].record(main)
+            hist_ready = torch.cuda.Event()
+            hist_ready.record(main)
+    torch.cuda.synchronize()
+    assert ple.ple_get_error(L.handle) == 0
+    for i in range(len(batches)):
+        assert torch.equal(outs[i], ref[i]), i
+    assert np.array_equal(hs2.cpu().numpy(), ref_state[0])
+    assert np.array_equal(cs2.cpu().numpy(), ref_state[1])
+
+
+def test_slot_one_needs_two_slots(tiny_layer):
+    toks, offs, hid = pi.tiny_batch(tiny_layer.w)
+    with pytest.raises(ple.PleError) as ei:
+        ple.ple_prepare_slot(tiny_layer.handle, 1, dev_i32(toks), len(toks), dev_i32(offs), 1)
+    assert ei.value.code == 1
+    with pytest.raises(ple.PleError) as ei:
+        ple.ple_prepare_slot(tiny_layer.handle, 2, dev_i32(toks), len(toks), dev_i32(offs), 1)
+    assert ei.value.code == 1
+    out = torch.empty(len(toks), tiny_layer.w.hidden, dtype=torch.float32, device="cuda")
+    with pytest.raises(ple.PleError) as ei:
+        ple.ple_forward_prepared_slot(tiny_layer.handle, 1, dev_bf16(hid), out, 1)
+    assert ei.value.code == 1
+
+
+def test_slot_batch_survives_forward(mid_two_slots):
+    """ple_forward uses slot 0's scratch: a batch prepared in slot 1 stays valid."""
+    L = mid_two_slots
+    rng = np.random.default_rng(9)
+    T = 700
+    toks = rng.integers(0, MID.vocab, T).astype(np.int32)
+    offs = np.array([0, 200, T], np.int32)
+    hid = pi.hidden_bf16(rng, T, MID.hidden)
+    ref, _ = gpu_forward(L, toks, offs, hid, 0)
+    ple.ple_prepare_slot(L.handle, 1, dev_i32(toks), T, dev_i32(offs), 2)
+    other = rng.integers(0, MID.vocab, 300).astype(np.int32)
+    gpu_forward(L, other, np.array([0, 300], np.int32), pi.hidden_bf16(rng, 300, MID.hidden), 0)
+    out = torch.empty(T, MID.hidden, dtype=torch.bfloat16, device="cuda")
+    ple.ple_forward_prepared_slot(L.handle, 1, dev_bf16(hid), out, 0)
+    torch.cuda.synchronize()
+    assert ple.ple_get_error(L.handle) == 0
+    assert np.array_equal(to_bits(out), ref)
