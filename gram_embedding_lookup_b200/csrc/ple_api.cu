@@ -380,6 +380,7 @@ ple_status run_decode_embed(ple_handle* h, const int32_t* tokens, int32_t B, int
   a.hidden = static_cast<const __nv_bfloat16*>(hidden);
   a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
   a.e = h->e;
+  a.ids = h->ids;
   a.meta = h->meta;
   a.w16 = h->w16;
   a.w16_bytes = static_cast<int64_t>(c.hidden) * c.row_dim * 2;
@@ -449,6 +450,7 @@ ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int3
                           false, stream);
   ple::DecodeProjArgs a = decode_proj_args(h, tokens, B, q, hidden, out, dtype, hist, conv_state, n_commit);
   a.e = h->e;
+  a.ids = h->ids;
   a.meta = h->meta;
   a.gate_ready = gate_ready ? 1 : 0;
   return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_decode_proj(a, h->decode_plan, stream); });

@@ -140,6 +140,8 @@ __global__ void __launch_bounds__(512) decode_embed_kernel(const DecodeEmbedArgs
   } else {
     const int64_t r0 = static_cast<int64_t>(mod_barrett(k2 ^ (k2 >> 32), a.rows0, a.magic0));
     const int64_t r1 = a.rows0 + static_cast<int64_t>(mod_barrett(k3 ^ (k3 >> 32), a.rows1, a.magic1));
+    if (threadIdx.x == 0 && a.ids != nullptr)
+      reinterpret_cast<int2*>(a.ids)[t] = make_int2(static_cast<int32_t>(r0), static_cast<int32_t>(r1 - a.rows0));
     const float s0 = __ldg(a.scales + r0), s1 = __ldg(a.scales + r1);
     for (int j = threadIdx.x; j < nch; j += blockDim.x) {
       const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.D, j);
@@ -170,6 +172,7 @@ constexpr int kPjMaxTok = 16;          // the mma's M: tokens
 constexpr int kPjGroup = 8;            // the mma's N: channels per group
 constexpr int kPjMaxGroups = 3;        // groups per CTA (24 channels)
 constexpr int kPjMaxChan = kPjGroup * kPjMaxGroups;
+constexpr int kTwoOrderMaxTok = 8;     // the two orders of up to 8 tokens fill the mma's 16 rows
 constexpr int kSmemLimit = 227 * 1024;
 
 struct __align__(16) ProjSmem {
@@ -182,6 +185,7 @@ struct __align__(16) ProjSmem {
   int32_t hist[kPjMaxTok][2];                               // the token history before the step
   int32_t nc[kPjMaxTok];                                    // n_commit
   int64_t rid[kPjMaxTok][2];                                // fused steps: global rows of the two orders
+  float sc[kPjMaxTok][2];                                   // two-order steps: the rows' scales
   int32_t rid16[kPjMaxTok][kHeads];                         // fused steps, multi-head layout
 };
 
@@ -214,11 +218,53 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// FMT < 0: the rows come from e (decode_embed_kernel); FMT = 0, 1, 2: the
-// kernel gathers them from an E4M3, NVFP4 or multi-head table.
-template <int FMT>
+// 16 codes of one row as exact fp16 values: E4M3 codes as they are; NVFP4
+// codes times their block scale (an E2M1 value times an E4M3 value has at most
+// 6 significant bits and lies in the fp16 range, so the product is exact).
+template <bool NV>
+__device__ __forceinline__ void codes_to_f16(const RowChunk<NV>& x, uint4& o0, uint4& o1) {
+  uint32_t h[8];
+  if constexpr (NV) {
+    const __half2 bs = __float2half2_rn(e4m3x2_cvt(x.b & 0xFFu).x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t w = k < 4 ? x.c.x : x.c.y;
+      const __half2 v = __hmul2(e2m1x2_cvt(w >> (8 * (k & 3))), bs);
+      h[k] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+  } else {
+    const uint32_t w[4] = {x.c.x, x.c.y, x.c.z, x.c.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu), __NV_E4M3);
+      h[k] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+  }
+  o0 = make_uint4(h[0], h[1], h[2], h[3]);
+  o1 = make_uint4(h[4], h[5], h[6], h[7]);
+}
+
+// How the kernel gets the step's rows:
+//   kRowsE      from e (fp16 e_t, decode_embed_kernel);
+//   kRowsHash   it hashes the tokens and gathers and dequantises e_t itself;
+//   kRowsHash2  it hashes the tokens and gathers the two orders' codes as exact
+//               fp16 A rows (token t's order-0 row in A row t, order-1 row in A
+//               row t + 8, T <= 8), the row scales applied after the products:
+//               v_t = s0 * (codes0 . W) + s1 * (codes1 . W);
+//   kRowsIds2   the same with the row IDs decode_embed_kernel wrote.
+// The two-order forms leave no rounding of e_t to fp16 and cost one
+// conversion per code pair instead of a fused multiply-add and a rounding per
+// element; a step gives the same bits through ple_decode_step and
+// ple_decode_prepare + ple_decode_step_prepared.
+constexpr int kRowsE = 0, kRowsHash = 1, kRowsHash2 = 2, kRowsIds2 = 3;
+
+// FMT = 0, 1, 2: E4M3, NVFP4 or multi-head table (unused with kRowsE).
+template <int FMT, int MODE>
 __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const DecodeProjArgs a) {
-  constexpr bool FUSED = FMT >= 0;
+  constexpr bool FUSED = MODE == kRowsHash || MODE == kRowsHash2;   // the kernel reads the history itself
+  constexpr bool TWO = MODE == kRowsHash2 || MODE == kRowsIds2;
+  static_assert(!TWO || FMT != 2, "the multi-head rows carry a scale per head: no two-order form");
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw_s + 127u) & ~127u) - raw_s);
@@ -226,7 +272,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
   const int ldr = a.D + 8;                                   // fp16 per shared-memory row
   __half* ws = reinterpret_cast<__half*>(base);              // [max_groups * 8][ldr]
   __half* es = ws + static_cast<int64_t>(a.max_groups) * kPjGroup * ldr;   // [T][ldr]
-  ProjSmem* sm = reinterpret_cast<ProjSmem*>(es + static_cast<int64_t>(T) * ldr);
+  ProjSmem* sm = reinterpret_cast<ProjSmem*>(es + static_cast<int64_t>(TWO ? kPjMaxTok : T) * ldr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G8 = a.H / kPjGroup;
   const int g0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * G8 / gridDim.x);
@@ -235,14 +281,16 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
   const int KS = a.D / 16;
   const int kb = ks_begin(warp, KS), ke = ks_begin(warp + 1, KS);
 
-  // ---- 1. before the wait: this warp's K range of the CTA's W_proj rows (constant
-  //         since ple_create), 16-byte cp.async (lane l copies chunks l and l + 32
-  //         of the range of every row), the conv taps of this lane's channel and,
-  //         when the gates are computed here, w_gate. Each warp reads back only the
+  // ---- 1. this warp's K range of the CTA's W_proj rows (constant since
+  //         ple_create), 16-byte cp.async (lane l copies chunks l and l + 32 of the
+  //         range of every row), before the wait, so that under programmatic
+  //         dependent launch they run under the kernel before. Before the wait
+  //         also the conv taps of this lane's channel and, when
+  //         the gates are computed here, w_gate. Each warp reads back only the
   //         W_proj and e it copied.
   const int kchunks = (ke - kb) * 2;                         // 16-byte chunks of one row in this warp's K range
   const bool second = lane + 32 < kchunks;
-  {
+  auto copy_w = [&] {
     const __half* src = a.w16 + static_cast<int64_t>(c0) * a.D + kb * 16 + lane * 8;
     uint32_t dst = smem_u32(ws + kb * 16 + lane * 8);
     if (lane < kchunks) {
@@ -251,8 +299,9 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
         if (second) cp_async_16(dst + 512, src + 256);
       }
     }
-  }
-  cp_async_commit();
+    cp_async_commit();
+  };
+  copy_w();
   // items: (sequence b, channel c), warp w takes sequences w, w + 8, ..., lane c
   float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane < nch) cw = __ldg(reinterpret_cast<const float4*>(a.conv_w) + c0 + lane);
@@ -272,7 +321,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
   // ---- 2. everything the step reads, in one round trip: e (this warp's K range)
   //         or the row IDs; residual, state, gates, tokens, history and n_commit
   //         into shared memory by cp.async
-  if constexpr (!FUSED) {
+  if constexpr (MODE == kRowsE) {
     if (lane < kchunks) {
       const __half* src = a.e + kb * 16 + lane * 8;
       uint32_t dst = smem_u32(es + kb * 16 + lane * 8);
@@ -314,32 +363,86 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
     }
   }
   int32_t ticket = -1;
+  float s_two[2] = {0.f, 0.f};                               // two-order forms: this thread's token's row scales
+  if constexpr (MODE == kRowsIds2) {
+    if (tid < T) {
+      const int2 id = reinterpret_cast<const int2*>(a.ids)[tid];
+      sm->rid[tid][0] = id.x;
+      sm->rid[tid][1] = a.rows0 + id.y;
+      s_two[0] = __ldg(a.scales + id.x);
+      s_two[1] = __ldg(a.scales + a.rows0 + id.y);
+    }
+    __syncthreads();                                         // row IDs ready
+  }
   if constexpr (FUSED) {
     // row IDs: thread t hashes token t (for the multi-head layout, thread (t, head))
     constexpr int kIdsPerTok = FMT == 2 ? kHeads : 1;
-    if (tid < T * kIdsPerTok) {
-      const int t = tid / kIdsPerTok, hh = tid - t * kIdsPerTok;
-      const int b = t / a.q, i = t - b * a.q;
-      const int32_t tok = a.tokens[t];
+    const bool hasher = tid < T * kIdsPerTok;
+    const int t = hasher ? tid / kIdsPerTok : 0, hh = hasher ? tid - t * kIdsPerTok : 0;
+    const int b = t / a.q, i = t - b * a.q;
+    int32_t tok = 0, p1 = -1, p2 = -1;                       // the token, then the one or two before it
+    if (hasher) {
+      tok = a.tokens[t];
+      p1 = i >= 1 ? a.tokens[t - 1] : a.hist[2 * b + 1];
+      p2 = i >= 2 ? a.tokens[t - 2] : (i == 1 ? a.hist[2 * b + 1] : a.hist[2 * b]);
+    }
+    if (hasher) {
       if (blockIdx.x == 0 && hh == 0 && (tok < 0 || tok >= a.vocab)) set_status(a.status, PLE_ERR_RANGE);
-      auto carried = [](int32_t h) -> uint64_t { return h < 0 ? 0ull : ctx_of(h); };
+      // inside the sequence every context is a token (+1); before it, a carried entry < 0 is absent
       const uint64_t x0 = ctx_of(tok);
-      const uint64_t x1 = i >= 1 ? ctx_of(a.tokens[t - 1]) : carried(a.hist[2 * b + 1]);
-      const uint64_t x2 = i >= 2 ? ctx_of(a.tokens[t - 2]) : (i == 1 ? carried(a.hist[2 * b + 1]) : carried(a.hist[2 * b]));
+      const uint64_t x1 = (i >= 1 || p1 >= 0) ? ctx_of(p1) : 0ull;
+      const uint64_t x2 = (i >= 2 || p2 >= 0) ? ctx_of(p2) : 0ull;
       const uint64_t k2 = (x0 * kQ0) ^ (x1 * kQ1);
       const uint64_t k3 = k2 ^ (x2 * kQ2);
       if constexpr (FMT == 2) {
         const uint64_t k = ((hh >> 3) ? k3 : k2) ^ (static_cast<uint64_t>(hh & 7) * kHeadMix);
         sm->rid16[t][hh] = static_cast<int32_t>(mod_barrett(k ^ (k >> 32), a.rows0, a.magic0));
       } else {
-        sm->rid[t][0] = static_cast<int64_t>(mod_barrett(k2 ^ (k2 >> 32), a.rows0, a.magic0));
-        sm->rid[t][1] = a.rows0 + static_cast<int64_t>(mod_barrett(k3 ^ (k3 >> 32), a.rows1, a.magic1));
+        const int64_t r0 = static_cast<int64_t>(mod_barrett(k2 ^ (k2 >> 32), a.rows0, a.magic0));
+        const int64_t r1 = a.rows0 + static_cast<int64_t>(mod_barrett(k3 ^ (k3 >> 32), a.rows1, a.magic1));
+        sm->rid[t][0] = r0;
+        sm->rid[t][1] = r1;
+        if constexpr (TWO) {
+          s_two[0] = __ldg(a.scales + r0);
+          s_two[1] = __ldg(a.scales + r1);
+        }
       }
     }
     __syncthreads();                                         // row IDs ready: this CTA has read the history
     // count this CTA in; the last CTA to arrive writes the new history at the end,
     // when no CTA of the grid can still read the old one (the ticket is used only then)
     if (tid == 0) ticket = atomicAdd(a.step_count, 1);
+  }
+  if constexpr (TWO) {
+    // this warp's K range (chunks of 16 codes, lane l takes chunk kb + l) of A
+    // rows r = 0..15: token r & 7, order r >> 3; two batches of 8 rows, each
+    // batch's loads in flight before any is used
+    const int nck = ke - kb;
+#pragma unroll
+    for (int r0 = 0; r0 < kPjMaxTok; r0 += 8) {
+      RowChunk<FMT == 1> x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = r0 + i, t = rr & 7;
+        if (t < T && lane < nck) x[i] = load_chunk<FMT == 1>(a.table, a.blocks, sm->rid[t][rr >> 3], a.D, kb + lane);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = r0 + i, t = rr & 7;
+        if (t < T && lane < nck) {
+          uint4 o0, o1;
+          codes_to_f16<FMT == 1>(x[i], o0, o1);
+          uint4* dst = reinterpret_cast<uint4*>(es + rr * ldr + (kb + lane) * 16);
+          dst[0] = o0;
+          dst[1] = o1;
+        }
+      }
+    }
+    if (tid < T) {
+      sm->sc[tid][0] = s_two[0];
+      sm->sc[tid][1] = s_two[1];
+    }
+  } else if constexpr (FUSED) {
     // this warp's K range (chunks of 16 codes) of every token's rows, dequantised
     // into e rows in shared memory: lane l takes tasks l, l + 32, ... of
     // (token, chunk), all of a batch's loads in flight before any is used
@@ -410,7 +513,8 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
     // ldmatrix.x4 for A: matrix m = lane / 8 covers token rows (m & 1) * 8 + 0..7 and
     // K offset (m >> 1) * 8; rows past T repeat the last token (their sums are unused)
     const int am = lane >> 3;
-    const int arow = min((lane & 7) + ((am & 1) << 3), T - 1);
+    const int lrow = (lane & 7) + ((am & 1) << 3);
+    const int arow = TWO ? (min(lrow & 7, T - 1) | (lrow & 8)) : min(lrow, T - 1);
     const uint32_t a_addr = smem_u32(es + arow * ldr + kb * 16 + ((am >> 1) << 3));
     // ldmatrix.x2 for B: lanes 0..15 address channel rows 0..7 at K offsets 0 and 8
     const uint32_t b_addr = smem_u32(ws + (lane & 7) * ldr + kb * 16 + (((lane >> 3) & 1) << 3));
@@ -459,8 +563,18 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
       for (int i = 0; i < a.q; ++i) {
         const int t = b * a.q + i;
         float v = 0.f;
+        if constexpr (TWO) {
+          float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-        for (int w = 0; w < kPjWarps; ++w) v += sm->red[w][g][t][cc];
+          for (int w = 0; w < kPjWarps; ++w) {
+            v0 += sm->red[w][g][t][cc];
+            v1 += sm->red[w][g][t + 8][cc];
+          }
+          v = sm->sc[t][0] * v0 + sm->sc[t][1] * v1;
+        } else {
+#pragma unroll
+          for (int w = 0; w < kPjWarps; ++w) v += sm->red[w][g][t][cc];
+        }
         const float u = sm->g[t] * v;
         const float y = cw.x * w0 + cw.y * w1 + cw.z * w2 + cw.w * u;
         w0 = w1;
@@ -557,21 +671,36 @@ cudaError_t launch_decode_proj(const DecodeProjArgs& a, const DecodeProjPlan& pl
         x = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
       if (x == cudaSuccess) x = prefer_max_shared(kernel);
     };
-    set(decode_proj_kernel<-1>);
-    set(decode_proj_kernel<0>);
-    set(decode_proj_kernel<1>);
-    set(decode_proj_kernel<2>);
+    set(decode_proj_kernel<0, kRowsE>);
+    set(decode_proj_kernel<0, kRowsHash>);
+    set(decode_proj_kernel<1, kRowsHash>);
+    set(decode_proj_kernel<2, kRowsHash>);
+    set(decode_proj_kernel<0, kRowsHash2>);
+    set(decode_proj_kernel<1, kRowsHash2>);
+    set(decode_proj_kernel<0, kRowsIds2>);
+    set(decode_proj_kernel<1, kRowsIds2>);
     return x;
   });
   if (e != cudaSuccess) return e;
   DecodeProjArgs b = a;
   b.max_groups = plan.max_groups;
-  const size_t smem = proj_smem_bytes(plan.max_groups, a.D, a.B * a.q);
+  const int T = a.B * a.q;
+  const bool two = a.format != PLE_TABLE_E4M3_HEADS && T <= kTwoOrderMaxTok;
+  const size_t smem = proj_smem_bytes(plan.max_groups, a.D, two ? kPjMaxTok : T);
   const dim3 grid(plan.grid), block(kPjThreads);
-  if (a.e != nullptr) return launch_pdl(decode_proj_kernel<-1>, grid, block, smem, b, stream);
-  if (a.format == PLE_TABLE_E4M3_HEADS) return launch_pdl(decode_proj_kernel<2>, grid, block, smem, b, stream);
-  if (a.format == PLE_TABLE_NVFP4) return launch_pdl(decode_proj_kernel<1>, grid, block, smem, b, stream);
-  return launch_pdl(decode_proj_kernel<0>, grid, block, smem, b, stream);
+  const bool nv = a.format == PLE_TABLE_NVFP4;
+  if (a.e != nullptr) {                                      // rows prepared by decode_embed_kernel
+    if (!two) return launch_pdl(decode_proj_kernel<0, kRowsE>, grid, block, smem, b, stream);
+    if (nv) return launch_pdl(decode_proj_kernel<1, kRowsIds2>, grid, block, smem, b, stream);
+    return launch_pdl(decode_proj_kernel<0, kRowsIds2>, grid, block, smem, b, stream);
+  }
+  if (two) {
+    if (nv) return launch_pdl(decode_proj_kernel<1, kRowsHash2>, grid, block, smem, b, stream);
+    return launch_pdl(decode_proj_kernel<0, kRowsHash2>, grid, block, smem, b, stream);
+  }
+  if (a.format == PLE_TABLE_E4M3_HEADS) return launch_pdl(decode_proj_kernel<2, kRowsHash>, grid, block, smem, b, stream);
+  if (nv) return launch_pdl(decode_proj_kernel<1, kRowsHash>, grid, block, smem, b, stream);
+  return launch_pdl(decode_proj_kernel<0, kRowsHash>, grid, block, smem, b, stream);
 }
 
 }  // namespace ple

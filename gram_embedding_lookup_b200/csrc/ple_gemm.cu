@@ -520,7 +520,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
   constexpr int STAGES = C::STAGES;
   constexpr int HBUFS = C::HBUFS;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, by pointer arithmetic on the shared array (an integer
+  // round trip would hide the address space, and plain loads from it would be
+  // generic ones)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   auto* bars = reinterpret_cast<SmemBars<STAGES, HBUFS>*>(smem + C::OFF_BAR);
   volatile int32_t* abort_flag = &bars->abort_flag;
   const uint32_t sA = smem_u32(smem + C::OFF_A);

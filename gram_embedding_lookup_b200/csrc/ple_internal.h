@@ -205,6 +205,7 @@ struct DecodeEmbedArgs {
   const __nv_bfloat16* hidden;   // [T][H], or null: the gate is computed later
   const __nv_bfloat16* w_gate;
   __half* e;               // [T][D]
+  int32_t* ids;            // [T][2] row IDs (two-order table formats; null: not written)
   TokMeta* meta;           // [T]
   const __half* w16;       // fp16 W_proj, prefetched into L2 for the kernel after this one (null: none)
   int64_t w16_bytes;
@@ -218,9 +219,12 @@ uint64_t barrett_magic(int64_t m);
 // conv against the carried state, residual and state commit, one CTA per SM.
 // CTA b owns a contiguous range of 8-channel groups with the whole K, so no
 // partial sums cross CTAs and no CTA waits for another. With e null the
-// kernel also computes the row IDs and gathers and dequantises, in each warp,
-// the K range of every token's rows that the warp multiplies (the whole step
-// in one kernel); otherwise it reads the rows decode_embed_kernel wrote.
+// kernel also computes the row IDs and gathers, in each warp, the K range of
+// every token's rows that the warp multiplies (the whole step in one kernel);
+// otherwise it reads the rows (or, for steps of up to 8 tokens, the row IDs)
+// decode_embed_kernel wrote. Up to 8 tokens of a two-order table run as 16
+// mma rows of exact codes (order 0 and order 1 of each token) with the row
+// scales applied after the products.
 struct DecodeProjArgs {
   const int32_t* tokens;   // [B][q] (the rows of a fused step, and the new token history)
   int32_t B, q;
@@ -229,6 +233,7 @@ struct DecodeProjArgs {
   const int32_t* n_commit; // [B] or null
   const __half* w16;       // fp16 W_proj [H][D] (K-major)
   const __half* e;         // [T][D] from decode_embed_kernel, or null: the kernel gathers the rows itself
+  const int32_t* ids;      // [T][2] from decode_embed_kernel (with e; read for steps of up to 8 tokens)
   const TokMeta* meta;     // [T]
   int32_t gate_ready;      // 1: meta[t].g holds the gate; 0: each CTA computes it from hidden
   // the table, for a step whose rows the kernel gathers itself (e null)

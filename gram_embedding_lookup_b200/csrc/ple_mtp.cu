@@ -99,7 +99,10 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     mtp_proj_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_e,
                     const MtpProjArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, by pointer arithmetic on the shared array (an integer
+  // round trip would hide the address space, and plain loads from it would be
+  // generic ones)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int S = a.stages;
   const uint32_t b_stage = static_cast<uint32_t>(a.n_pad) * kMtBK * 2;
   const uint32_t sA = smem_u32(smem);
@@ -295,45 +298,72 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         const __nv_bfloat16* Hb = reinterpret_cast<const __nv_bfloat16*>(Hs);
         const TokMeta* Mm = reinterpret_cast<const TokMeta*>(Ms);
         const float* Cf = reinterpret_cast<const float*>(Cs);
+        // Each thread owns its channel's row of every staged array, so the three
+        // passes below need no barrier between them. 1. The gated sums u, every
+        // token independent: the splits' sums are added in split order, four
+        // tokens' loads in flight at once; u overwrites split 0's slot.
+        float* Uf = reinterpret_cast<float*>(P);
+        for (int tq = 0; tq < nt; tq += 4) {
+          float part[4][kMtpMaxSplits];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float* pt = Pf + (tq + j) * kMtM + row;
+#pragma unroll
+            for (int sp = 0; sp < kMtpMaxSplits; ++sp)
+              part[j][sp] = (tq + j < nt && sp < a.k_splits) ? pt[sp * nt * kMtM] : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (tq + j < nt) {
+              float v = 0.f;
+#pragma unroll
+              for (int sp = 0; sp < kMtpMaxSplits; ++sp)
+                if (sp < a.k_splits) v += part[j][sp];
+              Uf[(tq + j) * kMtM + row] = Mm[tq + j].g * v;
+            }
+          }
+        }
+        // 2. the outputs, every token independent: the conv reads the sequence's
+        //    extended stream (three carried entries, then its tokens' u), token i
+        //    taps entries i, i + 1, i + 2 and its own u
+        {
+          int sb = 0, i = 0;
+#pragma unroll 4
+          for (int tc = 0; tc < nt; ++tc) {
+            const float* xc = Cf + sb * 3 * kMtM + row;
+            const float* xu = Uf + (tc - i) * kMtM + row;
+            const float e0 = i >= 3 ? xu[(i - 3) * kMtM] : xc[i * kMtM];
+            const float e1 = i >= 2 ? xu[(i - 2) * kMtM] : xc[(i + 1) * kMtM];
+            const float e2 = i >= 1 ? xu[(i - 1) * kMtM] : xc[(i + 2) * kMtM];
+            const float u = xu[i * kMtM];
+            const float y = cw.x * e0 + cw.y * e1 + cw.z * e2 + cw.w * u;
+            const int64_t idx = static_cast<int64_t>(t0 + tc) * a.H + ch;
+            const float o = __bfloat162float(Hb[tc * kMtM + row]) + y;
+            if (a.out_f32) reinterpret_cast<float*>(a.out)[idx] = o;
+            else reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(o);
+            if (++i == a.q) {
+              i = 0;
+              ++sb;
+            }
+          }
+        }
+        // 3. the carried state: the three entries of the extended stream that end
+        //    at the sequence's last committed token
         for (int sb = 0; sb < ns; ++sb) {
-          const int b = bc + sb;
           int32_t ncb = a.n_commit ? reinterpret_cast<const int32_t*>(Ns)[sb] : a.q;
           if (ncb < 1 || ncb > a.q) {
             if (et == 0 && m == 0) set_status(a.status, PLE_ERR_RANGE);
             ncb = max(1, min(ncb, a.q));
           }
-          float w0 = Cf[(sb * 3) * kMtM + row], w1 = Cf[(sb * 3 + 1) * kMtM + row], w2 = Cf[(sb * 3 + 2) * kMtM + row];
-          float k0 = w0, k1 = w1, k2 = w2;
-          for (int i = 0; i < a.q; ++i) {
-            const int tc = sb * a.q + i;
-            // all of the token's split sums first (independent loads), then their sum in split order
-            const float* pt = Pf + tc * kMtM + row;
-            float part[kMtpMaxSplits];
+          const float* xc = Cf + sb * 3 * kMtM + row;
+          const float* xu = Uf + sb * a.q * kMtM + row;
+          float k[3];
 #pragma unroll
-            for (int sp = 0; sp < kMtpMaxSplits; ++sp) part[sp] = sp < a.k_splits ? pt[sp * nt * kMtM] : 0.f;
-            float v = 0.f;
-#pragma unroll
-            for (int sp = 0; sp < kMtpMaxSplits; ++sp)
-              if (sp < a.k_splits) v += part[sp];
-            const float u = Mm[tc].g * v;
-            const float y = cw.x * w0 + cw.y * w1 + cw.z * w2 + cw.w * u;
-            w0 = w1;
-            w1 = w2;
-            w2 = u;
-            const int64_t idx = static_cast<int64_t>(t0 + tc) * a.H + ch;
-            const float o = __bfloat162float(Hb[tc * kMtM + row]) + y;
-            if (a.out_f32) reinterpret_cast<float*>(a.out)[idx] = o;
-            else reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(o);
-            if (i == ncb - 1) {
-              k0 = w0;
-              k1 = w1;
-              k2 = w2;
-            }
-          }
-          float* cs = a.conv_state + static_cast<int64_t>(b) * 3 * a.H + ch;
-          cs[0] = k0;
-          cs[a.H] = k1;
-          cs[2 * a.H] = k2;
+          for (int j = 0; j < 3; ++j) k[j] = ncb + j >= 3 ? xu[(ncb + j - 3) * kMtM] : xc[(ncb + j) * kMtM];
+          float* cs = a.conv_state + static_cast<int64_t>(bc + sb) * 3 * a.H + ch;
+          cs[0] = k[0];
+          cs[a.H] = k[1];
+          cs[2 * a.H] = k[2];
         }
         named_bar_sync(1, kMtEpiThreads);                  // the staging area is reused by the next chunk
       }

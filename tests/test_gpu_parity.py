@@ -742,7 +742,10 @@ def test_decode_paths_tiny(tiny_layer, shape):
         assert np.array_equal(h2, ref["hist_out"])
         assert_close(c2, ref["conv_out"], f"decode state {shape} path {path}")
         outs.append(out)
-    assert np.abs(outs[0] - outs[1]).max() < 1e-4
+    # steps of up to 8 tokens multiply the two orders' exact codes and scale after the
+    # products, the split-K path the fp16-rounded sum of the orders: equal within the
+    # tolerance, not bit for bit
+    assert_close(outs[0], outs[1], f"decode {shape}: channel-split against split-K")
 
 
 @pytest.mark.parametrize("shape", [(8, 1), (4, 3), (16, 1)])
