@@ -997,6 +997,45 @@ def timed_each(ctx, stream, fn, n, flush=None):
     return ctx["max_over_ranks"](sum(a.elapsed_time(b) for a, b in ev) / n)
 
 
+def graph_time(ctx, stream, fns, reps=20, n=5):
+    """Device time (ms) of one pass of fns (each fn(st) enqueues its work on stream
+    st), from a CUDA graph of reps passes back to back, replayed n times between two
+    events on `stream`; max over ranks."""
+    torch = ctx["torch"]
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for f in fns:
+            f(side)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        cur = torch.cuda.current_stream()
+        for _ in range(reps):
+            for f in fns:
+                f(cur)
+    g.replay()
+    ctx["barrier"]()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ctx["barrier"]()
+    del g
+    return ctx["max_over_ranks"](e0.elapsed_time(e1) / (n * reps))
+
+
+def graph_delta(ctx, stream, base, extra, reps=20):
+    """Device time (ms) that the calls `extra` add to a pass of `base` (for example
+    an L2 flush, so that they start from a cold L2), as the difference of two
+    graph timings: no host launch latency and no events between the kernels."""
+    return graph_time(ctx, stream, base + extra, reps) - graph_time(ctx, stream, base, reps)
+
+
 def l2_flush_buffer(torch):
     """256 MB, twice the B200's 126 MB L2."""
     return torch.zeros(64 << 20, dtype=torch.int32, device="cuda")
@@ -1052,7 +1091,14 @@ def decode_bench(ctx, layer, stream):
 
     flush = l2_flush_buffer(torch)
     n_cold = 200
-    ms_cold = timed_each(ctx, stream, eager, n_cold, flush)
+    fl = lambda st: flush.add_(1)  # noqa: E731
+    ms_cold = graph_delta(ctx, stream, [fl], [lambda st: eager(0, st)])
+    # the same after the flush as one eager call between two events: adds the host's
+    # submission and the events' own cost, which the same two events around a
+    # one-element torch kernel show
+    ms_cold_eager = timed_each(ctx, stream, eager, n_cold, flush)
+    tiny = torch.zeros(1, device="cuda")
+    ms_tiny_eager = timed_each(ctx, stream, lambda i: tiny.add_(1), n_cold, flush)
 
     def prep(i):
         ple.ple_decode_prepare(h, tk, B, q, hs, stream)
@@ -1060,47 +1106,16 @@ def decode_bench(ctx, layer, stream):
     def rest(i):
         ple.ple_decode_step_prepared(h, hd, out, ple.PLE_OUT_BF16, hs, cs, None, stream)
 
-    # the hidden-dependent half after its prepare, both cold: flush, prepare, flush, step
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_cold)]
-    torch.cuda.synchronize()
-    for i in range(n_cold):
-        flush.add_(1)
-        ev[i][0].record(stream)
-        prep(i)
-        ev[i][1].record(stream)
-        flush.add_(1)
-        ev[i][2].record(stream)
-        rest(i)
-        ev[i][3].record(stream)
-    torch.cuda.synchronize()
-    prep_cold = sum(e[0].elapsed_time(e[1]) for e in ev) / n_cold
-    rest_cold = sum(e[2].elapsed_time(e[3]) for e in ev) / n_cold
+    pr = lambda st: ple.ple_decode_prepare(h, tk, B, q, hs, st)  # noqa: E731
+    rs = lambda st: ple.ple_decode_step_prepared(h, hd, out, ple.PLE_OUT_BF16, hs, cs, None, st)  # noqa: E731
+    # each half from a cold L2: flush, prepare, flush, step (the step's rows evicted too)
+    prep_cold = graph_delta(ctx, stream, [fl], [pr])
+    rest_cold = graph_delta(ctx, stream, [fl, pr, fl], [rs])
     # the hidden-dependent half right after its prepare, from a cold L2: flush, prepare, step
     # (the prepare also pulls W_proj into L2, as it would ahead of the hidden states)
-    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_cold)]
-    torch.cuda.synchronize()
-    for i in range(n_cold):
-        flush.add_(1)
-        prep(i)
-        ev2[i][0].record(stream)
-        rest(i)
-        ev2[i][1].record(stream)
-    torch.cuda.synchronize()
-    rest_after_prep = sum(e[0].elapsed_time(e[1]) for e in ev2) / n_cold
-    for i in range(5):
-        prep(i)
-        rest(i)
-    warm = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_cold)]
-    torch.cuda.synchronize()
-    for i in range(n_cold):
-        warm[i][0].record(stream)
-        prep(i)
-        warm[i][1].record(stream)
-        rest(i)
-        warm[i][2].record(stream)
-    torch.cuda.synchronize()
-    prep_warm = sum(e[0].elapsed_time(e[1]) for e in warm) / n_cold
-    rest_warm = sum(e[1].elapsed_time(e[2]) for e in warm) / n_cold
+    rest_after_prep = graph_delta(ctx, stream, [fl, pr], [rs])
+    prep_warm = graph_time(ctx, stream, [pr])
+    rest_warm = graph_delta(ctx, stream, [pr], [rs])
     del flush
     torch.cuda.empty_cache()
     status = ple.ple_get_error(h)
@@ -1116,6 +1131,7 @@ def decode_bench(ctx, layer, stream):
             "value": B * q * world * n / (ms_eager / 1e3), "unit": "tokens/s", "us_per_step": us(ms_eager) / n,
             "graph_us_per_step": us(graphs[1]), "graph10_us_per_step": us(graphs[10]),
             "cold_us_per_step": us(ms_cold),
+            "cold_eager_us_per_step": us(ms_cold_eager), "cold_eager_tiny_torch_kernel_us": us(ms_tiny_eager),
             "cold_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
                               "achieved_gbs": step_bytes / (ms_cold / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                               "frac": step_bytes / (ms_cold / 1e3) / 1e9 / peaks["hbm_gbs"]},
@@ -1128,8 +1144,11 @@ def decode_bench(ctx, layer, stream):
             "device_status": int(status),
             "note": "warm: one batch reused, steps back to back (W_proj and rows stay in L2, each step's W_proj "
                     "copies overlap the previous step under programmatic dependent launch); graph: one or ten "
-                    "captured steps per replay (no overlap across replays); cold: 256 MB written between steps, "
-                    "outside the events"}
+                    "captured steps per replay (no overlap across replays); cold: 256 MB written before every "
+                    "step, the step's time the difference between graphs of 20 x (write, step) and 20 x (write) "
+                    "(the same for the prepared halves, warm ones as graphs of 20 x (prepare, step) minus 20 x "
+                    "(prepare)); cold_eager: one eager call after the write between two events, with the host's "
+                    "submission inside, beside the same around a one-element torch kernel"}
 
 
 def mtp_bench(ctx, layer, stream):
@@ -1171,7 +1190,10 @@ def mtp_bench(ctx, layer, stream):
     hist.copy_(hist0)
     conv.copy_(conv0)
     flush = l2_flush_buffer(torch)
-    ms_cold = timed_each(ctx, stream, step, n, flush)
+    ms_cold_eager = timed_each(ctx, stream, step, n, flush)
+    ms_cold = graph_delta(ctx, stream, [lambda st: flush.add_(1)],
+                          [lambda st: ple.ple_decode_step(h, steps[0][0], B, q, steps[0][1], out, ple.PLE_OUT_BF16,
+                                                          hist, conv, steps[0][2], st)])
     del flush
     torch.cuda.empty_cache()
     status = ple.ple_get_error(h)
@@ -1180,7 +1202,11 @@ def mtp_bench(ctx, layer, stream):
     return {"workload": "MTP decode: 64 sequences x 3 tokens/step, 100 steps, 30% shared prefix",
             "value": B * q * world * n / (ms / 1e3), "unit": "tokens/s (processed)",
             "committed_tokens_per_s": committed * world / (ms / 1e3), "us_per_step": 1e3 * ms / n,
-            "cold_us_per_step": 1e3 * ms_cold, "device_status": int(status)}
+            "cold_us_per_step": 1e3 * ms_cold, "cold_eager_us_per_step": 1e3 * ms_cold_eager,
+            "device_status": int(status),
+            "note": "cold: 256 MB written before every step, the step's time the difference between graphs of 20 x "
+                    "(write, step) and 20 x (write); cold_eager: the 100 steps each after the write, one eager call "
+                    "between two events"}
 
 
 def long_bench(ctx, layer, stream):

@@ -49,6 +49,7 @@ struct ple_handle {
     int32_t* ids = nullptr;
     ple::TokMeta* meta = nullptr;
     int32_t* hist_new = nullptr;
+    float* row_scales = nullptr;   // decode steps of up to 8 tokens: [T][2] the two rows' scales
   } scratch[2];
   __half*& e = scratch[0].e;
   int32_t*& ids = scratch[0].ids;
@@ -78,6 +79,7 @@ struct ple_handle {
     int32_t B = 0, q = 0;
     const int32_t* tokens = nullptr;
     const int32_t* hist = nullptr;
+    bool small = false;    // the channel-split kernel takes the step (chosen when prepared)
   } prepared_decode;
   bool profiling = false;
   struct Rec { int stage; cudaEvent_t a, b; };
@@ -200,6 +202,7 @@ void free_all(ple_handle* h) {
     cudaFree(sc.ids);
     cudaFree(sc.meta);
     cudaFree(sc.hist_new);
+    cudaFree(sc.row_scales);
   }
   cudaFree(h->partial);
   cudaFree(h->conv0);
@@ -356,10 +359,16 @@ ple_status run_projection(ple_handle* h, const ple_handle::Scratch& sc, int32_t 
   return run_stage(h, PLE_STAGE_COMBINE, stream, [&] { return ple::launch_combine_forward(ca, stream); });
 }
 
-// The tokens-only half of a decode step: rows into h->e, metadata into h->meta,
-// and the gates when hidden is given.
+// Whether the channel-split kernel takes a decode step of B x q tokens.
+bool decode_small(const ple_handle* h, int32_t B, int32_t q) {
+  return h->forward_path != 2 && h->decode_proj && ple::decode_proj_supported(B, q);
+}
+
+// The tokens-only half of a decode step: rows into h->e (for a step the
+// channel-split kernel takes on exact codes, the codes and row scales),
+// metadata into h->meta, and the gates when hidden is given.
 ple_status run_decode_embed(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const int32_t* hist,
-                            const void* hidden, cudaStream_t stream) {
+                            const void* hidden, bool small, cudaStream_t stream) {
   const ple_config& c = h->cfg;
   ple::DecodeEmbedArgs a{};
   a.tokens = tokens;
@@ -380,7 +389,8 @@ ple_status run_decode_embed(ple_handle* h, const int32_t* tokens, int32_t B, int
   a.hidden = static_cast<const __nv_bfloat16*>(hidden);
   a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
   a.e = h->e;
-  a.ids = h->ids;
+  a.row_scales = h->scratch[0].row_scales;
+  a.codes2 = small && ple::decode_two_order(B * q, c.table_format) ? 1 : 0;
   a.meta = h->meta;
   a.w16 = h->w16;
   a.w16_bytes = static_cast<int64_t>(c.hidden) * c.row_dim * 2;
@@ -400,10 +410,9 @@ ple::DecodeProjArgs decode_proj_args(const ple_handle* h, const int32_t* tokens,
 // the kernels after it cannot compute them (split-K, or out aliasing hidden).
 ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const void* hidden, void* out,
                            ple_out_dtype dtype, int32_t* hist, float* conv_state, const int32_t* n_commit,
-                           bool gate_ready, cudaStream_t stream) {
+                           bool gate_ready, bool small, cudaStream_t stream) {
   const ple_config& c = h->cfg;
   const int32_t T = B * q;
-  const bool small = h->forward_path != 2 && h->decode_proj && ple::decode_proj_supported(B, q);
   if (!gate_ready && (!small || out == hidden)) {
     ple::PrepareArgs ga{};
     ga.T = T;
@@ -450,7 +459,7 @@ ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int3
                           false, stream);
   ple::DecodeProjArgs a = decode_proj_args(h, tokens, B, q, hidden, out, dtype, hist, conv_state, n_commit);
   a.e = h->e;
-  a.ids = h->ids;
+  a.row_scales = h->scratch[0].row_scales;
   a.meta = h->meta;
   a.gate_ready = gate_ready ? 1 : 0;
   return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_decode_proj(a, h->decode_plan, stream); });
@@ -585,7 +594,8 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
     ok = cudaMalloc(&sc.e, static_cast<size_t>(e_rows) * c.row_dim * 2) == cudaSuccess &&
          cudaMalloc(&sc.ids, static_cast<size_t>(c.max_tokens) * ids_per_token(c) * 4) == cudaSuccess &&
          cudaMalloc(&sc.meta, static_cast<size_t>(c.max_tokens) * sizeof(ple::TokMeta)) == cudaSuccess &&
-         cudaMalloc(&sc.hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess;
+         cudaMalloc(&sc.hist_new, static_cast<size_t>(c.max_seqs) * 2 * 4) == cudaSuccess &&
+         cudaMalloc(&sc.row_scales, 16 * 2 * 4) == cudaSuccess;
   }
   h->decode_proj = ple::decode_proj_plan(c.hidden, c.row_dim, h->num_sms, &h->decode_plan);
   h->mtp = ok && c.max_tokens > 16 && ple::mtp_proj_plan(c.hidden, c.row_dim, h->num_sms, &h->mtp_plan);
@@ -794,7 +804,8 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
   if (!aligned(tokens, 4)) return PLE_ERR_ALIGN;
   h->prepared.valid = false;
   h->prepared_decode.valid = false;
-  if (h->forward_path != 2 && h->decode_proj && ple::decode_proj_supported(B, q) && out != hidden) {
+  const bool small = decode_small(h, B, q);
+  if (small && out != hidden) {
     // the whole step in one kernel: each CTA hashes the tokens and gathers the
     // K range of the rows it multiplies, and computes the gates
     ple::DecodeProjArgs a = decode_proj_args(h, tokens, B, q, hidden, out, out_dtype, hist, conv_state, n_commit);
@@ -803,9 +814,9 @@ ple_status ple_decode_step(ple_handle* h, const int32_t* tokens, int32_t B, int3
     a.gate_ready = 0;
     return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_decode_proj(a, h->decode_plan, stream); });
   }
-  const ple_status st = run_decode_embed(h, tokens, B, q, hist, hidden, stream);
+  const ple_status st = run_decode_embed(h, tokens, B, q, hist, hidden, small, stream);
   if (st != PLE_OK) return st;
-  return run_decode_rest(h, tokens, B, q, hidden, out, out_dtype, hist, conv_state, n_commit, true, stream);
+  return run_decode_rest(h, tokens, B, q, hidden, out, out_dtype, hist, conv_state, n_commit, true, small, stream);
 }
 
 ple_status ple_decode_prepare(ple_handle* h, const int32_t* tokens, int32_t B, int32_t q, const int32_t* hist,
@@ -817,9 +828,10 @@ ple_status ple_decode_prepare(ple_handle* h, const int32_t* tokens, int32_t B, i
   if (!aligned(tokens, 4) || !aligned(hist, 4)) return PLE_ERR_ALIGN;
   h->prepared.valid = false;
   h->prepared_decode.valid = false;
-  const ple_status st = run_decode_embed(h, tokens, B, q, hist, nullptr, stream);
+  const bool small = decode_small(h, B, q);
+  const ple_status st = run_decode_embed(h, tokens, B, q, hist, nullptr, small, stream);
   if (st != PLE_OK) return st;
-  h->prepared_decode = {true, B, q, tokens, hist};
+  h->prepared_decode = {true, B, q, tokens, hist, small};
   return PLE_OK;
 }
 
@@ -833,7 +845,7 @@ ple_status ple_decode_step_prepared(ple_handle* h, const void* hidden, void* out
   if (chk != PLE_OK) return chk;
   h->prepared_decode.valid = false;     // the state advances: the rows belong to this step only
   return run_decode_rest(h, pd.tokens, pd.B, pd.q, hidden, out, out_dtype, hist, conv_state, n_commit, false,
-                         stream);
+                         pd.small, stream);
 }
 
 ple_status ple_get_error(ple_handle* h) {

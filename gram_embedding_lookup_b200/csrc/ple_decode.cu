@@ -63,13 +63,44 @@ __device__ __forceinline__ uint64_t mod_barrett(uint64_t x, uint64_t m, uint64_t
   return r;
 }
 
+constexpr int kTwoOrderMaxTok = 8;     // two-order steps: order 0 of token t in row t, order 1 in row t + 8
+
+// 16 codes of one row as exact fp16 values: E4M3 codes as they are; NVFP4
+// codes times their block scale (an E2M1 value times an E4M3 value has at most
+// 6 significant bits and lies in the fp16 range, so the product is exact).
+template <bool NV>
+__device__ __forceinline__ void codes_to_f16(const RowChunk<NV>& x, uint4& o0, uint4& o1) {
+  uint32_t h[8];
+  if constexpr (NV) {
+    const __half2 bs = __float2half2_rn(e4m3x2_cvt(x.b & 0xFFu).x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t w = k < 4 ? x.c.x : x.c.y;
+      const __half2 v = __hmul2(e2m1x2_cvt(w >> (8 * (k & 3))), bs);
+      h[k] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+  } else {
+    const uint32_t w[4] = {x.c.x, x.c.y, x.c.z, x.c.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu), __NV_E4M3);
+      h[k] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+  }
+  o0 = make_uint4(h[0], h[1], h[2], h[3]);
+  o1 = make_uint4(h[4], h[5], h[6], h[7]);
+}
+
 // ------------------------------------------------------------------ embed: rows, metadata, gate
 // FMT: 0 = E4M3 rows (two orders), 1 = NVFP4 rows, 2 = the multi-head E4M3 layout.
 // Thread j of the block takes 16-code chunks j, j + blockDim, ... of the
 // token's row (of all 16 head rows side by side for FMT 2); warp 0 also
 // computes the gate.
+constexpr int kEmbedThreads = 256;    // most threads of a decode_embed_kernel block
+
 template <int FMT>
-__global__ void __launch_bounds__(512) decode_embed_kernel(const DecodeEmbedArgs a) {
+__global__ void __launch_bounds__(kEmbedThreads) decode_embed_kernel(const DecodeEmbedArgs a) {
   constexpr bool NV = FMT == 1;
   pdl_launch_dependents();             // the projection's prologue (its W_proj copies) may start now
   if (a.w16 != nullptr && threadIdx.x < 32) {
@@ -140,16 +171,31 @@ __global__ void __launch_bounds__(512) decode_embed_kernel(const DecodeEmbedArgs
   } else {
     const int64_t r0 = static_cast<int64_t>(mod_barrett(k2 ^ (k2 >> 32), a.rows0, a.magic0));
     const int64_t r1 = a.rows0 + static_cast<int64_t>(mod_barrett(k3 ^ (k3 >> 32), a.rows1, a.magic1));
-    if (threadIdx.x == 0 && a.ids != nullptr)
-      reinterpret_cast<int2*>(a.ids)[t] = make_int2(static_cast<int32_t>(r0), static_cast<int32_t>(r1 - a.rows0));
     const float s0 = __ldg(a.scales + r0), s1 = __ldg(a.scales + r1);
-    for (int j = threadIdx.x; j < nch; j += blockDim.x) {
-      const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.D, j);
-      const RowChunk<NV> y = load_chunk<NV>(a.table, a.blocks, r1, a.D, j);
-      uint4 o0, o1;
-      deq_chunk<NV>(x, y, s0, s1, o0, o1);
-      erow[2 * j] = o0;
-      erow[2 * j + 1] = o1;
+    if (a.codes2) {
+      // the two rows as exact fp16 codes (rows t and t + 8 of e), the scales apart
+      uint4* crow1 = reinterpret_cast<uint4*>(a.e + static_cast<int64_t>(t + kTwoOrderMaxTok) * a.D);
+      for (int j = threadIdx.x; j < nch; j += blockDim.x) {
+        const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.D, j);
+        const RowChunk<NV> y = load_chunk<NV>(a.table, a.blocks, r1, a.D, j);
+        uint4 o0, o1;
+        codes_to_f16<NV>(x, o0, o1);
+        erow[2 * j] = o0;
+        erow[2 * j + 1] = o1;
+        codes_to_f16<NV>(y, o0, o1);
+        crow1[2 * j] = o0;
+        crow1[2 * j + 1] = o1;
+      }
+      if (threadIdx.x == 0) reinterpret_cast<float2*>(a.row_scales)[t] = make_float2(s0, s1);
+    } else {
+      for (int j = threadIdx.x; j < nch; j += blockDim.x) {
+        const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.D, j);
+        const RowChunk<NV> y = load_chunk<NV>(a.table, a.blocks, r1, a.D, j);
+        uint4 o0, o1;
+        deq_chunk<NV>(x, y, s0, s1, o0, o1);
+        erow[2 * j] = o0;
+        erow[2 * j + 1] = o1;
+      }
     }
   }
   if (threadIdx.x < 32) {
@@ -172,7 +218,6 @@ constexpr int kPjMaxTok = 16;          // the mma's M: tokens
 constexpr int kPjGroup = 8;            // the mma's N: channels per group
 constexpr int kPjMaxGroups = 3;        // groups per CTA (24 channels)
 constexpr int kPjMaxChan = kPjGroup * kPjMaxGroups;
-constexpr int kTwoOrderMaxTok = 8;     // the two orders of up to 8 tokens fill the mma's 16 rows
 constexpr int kSmemLimit = 227 * 1024;
 
 struct __align__(16) ProjSmem {
@@ -187,6 +232,7 @@ struct __align__(16) ProjSmem {
   int64_t rid[kPjMaxTok][2];                                // fused steps: global rows of the two orders
   float sc[kPjMaxTok][2];                                   // two-order steps: the rows' scales
   int32_t rid16[kPjMaxTok][kHeads];                         // fused steps, multi-head layout
+  uint64_t wbar;                                            // W_proj rows landed
 };
 
 // K-steps (16 values of K) of warp w: [ks_begin(w), ks_begin(w + 1)).
@@ -218,33 +264,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 16 codes of one row as exact fp16 values: E4M3 codes as they are; NVFP4
-// codes times their block scale (an E2M1 value times an E4M3 value has at most
-// 6 significant bits and lies in the fp16 range, so the product is exact).
-template <bool NV>
-__device__ __forceinline__ void codes_to_f16(const RowChunk<NV>& x, uint4& o0, uint4& o1) {
-  uint32_t h[8];
-  if constexpr (NV) {
-    const __half2 bs = __float2half2_rn(e4m3x2_cvt(x.b & 0xFFu).x);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t w = k < 4 ? x.c.x : x.c.y;
-      const __half2 v = __hmul2(e2m1x2_cvt(w >> (8 * (k & 3))), bs);
-      h[k] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-  } else {
-    const uint32_t w[4] = {x.c.x, x.c.y, x.c.z, x.c.w};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
-          static_cast<__nv_fp8x2_storage_t>((w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu), __NV_E4M3);
-      h[k] = *reinterpret_cast<const uint32_t*>(&r);
-    }
-  }
-  o0 = make_uint4(h[0], h[1], h[2], h[3]);
-  o1 = make_uint4(h[4], h[5], h[6], h[7]);
-}
-
 // How the kernel gets the step's rows:
 //   kRowsE      from e (fp16 e_t, decode_embed_kernel);
 //   kRowsHash   it hashes the tokens and gathers and dequantises e_t itself;
@@ -252,18 +271,19 @@ __device__ __forceinline__ void codes_to_f16(const RowChunk<NV>& x, uint4& o0, u
 //               fp16 A rows (token t's order-0 row in A row t, order-1 row in A
 //               row t + 8, T <= 8), the row scales applied after the products:
 //               v_t = s0 * (codes0 . W) + s1 * (codes1 . W);
-//   kRowsIds2   the same with the row IDs decode_embed_kernel wrote.
+//   kRowsCodes2 the same with the codes and row scales decode_embed_kernel wrote.
 // The two-order forms leave no rounding of e_t to fp16 and cost one
 // conversion per code pair instead of a fused multiply-add and a rounding per
 // element; a step gives the same bits through ple_decode_step and
 // ple_decode_prepare + ple_decode_step_prepared.
-constexpr int kRowsE = 0, kRowsHash = 1, kRowsHash2 = 2, kRowsIds2 = 3;
+constexpr int kRowsE = 0, kRowsHash = 1, kRowsHash2 = 2, kRowsCodes2 = 3;
 
 // FMT = 0, 1, 2: E4M3, NVFP4 or multi-head table (unused with kRowsE).
 template <int FMT, int MODE>
 __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const DecodeProjArgs a) {
   constexpr bool FUSED = MODE == kRowsHash || MODE == kRowsHash2;   // the kernel reads the history itself
-  constexpr bool TWO = MODE == kRowsHash2 || MODE == kRowsIds2;
+  constexpr bool TWO = MODE == kRowsHash2 || MODE == kRowsCodes2;
+  constexpr bool COPIED = MODE == kRowsE || MODE == kRowsCodes2;      // rows from decode_embed_kernel
   static_assert(!TWO || FMT != 2, "the multi-head rows carry a scale per head: no two-order form");
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -281,27 +301,25 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
   const int KS = a.D / 16;
   const int kb = ks_begin(warp, KS), ke = ks_begin(warp + 1, KS);
 
-  // ---- 1. this warp's K range of the CTA's W_proj rows (constant since
-  //         ple_create), 16-byte cp.async (lane l copies chunks l and l + 32 of the
-  //         range of every row), before the wait, so that under programmatic
-  //         dependent launch they run under the kernel before. Before the wait
-  //         also the conv taps of this lane's channel and, when
-  //         the gates are computed here, w_gate. Each warp reads back only the
-  //         W_proj and e it copied.
+  // ---- 1. the CTA's W_proj rows (constant since ple_create) by bulk copies,
+  //         lane r of the last warp copying row r, counted in bytes on wbar:
+  //         issued before the wait, so that under programmatic dependent launch
+  //         they run under the kernel before, and without holding any warp, so
+  //         that the hashing starts at once. Before the wait also the conv taps
+  //         of this lane's channel and, when the gates are computed here, w_gate.
   const int kchunks = (ke - kb) * 2;                         // 16-byte chunks of one row in this warp's K range
   const bool second = lane + 32 < kchunks;
-  auto copy_w = [&] {
-    const __half* src = a.w16 + static_cast<int64_t>(c0) * a.D + kb * 16 + lane * 8;
-    uint32_t dst = smem_u32(ws + kb * 16 + lane * 8);
-    if (lane < kchunks) {
-      for (int r = 0; r < nch; ++r, src += a.D, dst += ldr * 2) {
-        cp_async_16(dst, src);
-        if (second) cp_async_16(dst + 512, src + 256);
-      }
+  const uint32_t wbar = smem_u32(&sm->wbar);
+  if (warp == kPjWarps - 1) {
+    if (lane == 0) {
+      mbar_init(wbar, 1);
+      fence_barrier_init();
+      mbar_arrive_expect_tx(wbar, static_cast<uint32_t>(nch) * a.D * 2u);
     }
-    cp_async_commit();
-  };
-  copy_w();
+    __syncwarp();
+    for (int r = lane; r < nch; r += 32)
+      bulk_load(smem_u32(ws + r * ldr), a.w16 + static_cast<int64_t>(c0 + r) * a.D, a.D * 2u, wbar);
+  }
   // items: (sequence b, channel c), warp w takes sequences w, w + 8, ..., lane c
   float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane < nch) cw = __ldg(reinterpret_cast<const float4*>(a.conv_w) + c0 + lane);
@@ -318,18 +336,22 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
   pdl_launch_dependents();
   pdl_wait();                                                // tokens, e, meta, hidden and the state are ready
 
-  // ---- 2. everything the step reads, in one round trip: e (this warp's K range)
-  //         or the row IDs; residual, state, gates, tokens, history and n_commit
-  //         into shared memory by cp.async
-  if constexpr (MODE == kRowsE) {
+  // ---- 2. everything the step reads, in one round trip: the rows or codes
+  //         decode_embed_kernel wrote (this warp's K range) and the codes' row
+  //         scales; residual, state, gates, tokens, history and n_commit into
+  //         shared memory by cp.async
+  if constexpr (COPIED) {
+    // this warp's K range of the rows (two-order: rows t and t + 8 of token t)
     if (lane < kchunks) {
-      const __half* src = a.e + kb * 16 + lane * 8;
-      uint32_t dst = smem_u32(es + kb * 16 + lane * 8);
-      for (int r = 0; r < T; ++r, src += a.D, dst += ldr * 2) {
+      for (int r = 0; r < (TWO ? kPjMaxTok : T); ++r) {
+        if (TWO && (r & 7) >= T) continue;
+        const __half* src = a.e + static_cast<int64_t>(r) * a.D + kb * 16 + lane * 8;
+        const uint32_t dst = smem_u32(es + r * ldr + kb * 16 + lane * 8);
         cp_async_16(dst, src);
         if (second) cp_async_16(dst + 512, src + 256);
       }
     }
+    if (TWO && tid < 2 * T) cp_async_4(smem_u32(&sm->sc[tid >> 1][tid & 1]), a.row_scales + tid);
   }
   {
     // hidden at this CTA's channels: ng 16-byte pieces per token
@@ -362,18 +384,26 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
       if (j < H8) hv[r] = ld_stream_v4(reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(warp) * a.H) + j);
     }
   }
+  // gates: warp w takes tokens w, w + 8, ... (its first token's hidden row is in
+  // flight already); computed while the row IDs are found, before any row is read
+  auto gates = [&] {
+    if (!a.gate_ready) {
+      for (int t = warp; t < T; t += kPjWarps) {
+        const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
+        if (t != warp) {
+#pragma unroll
+          for (int r = 0; r < kEmbedH4; ++r) {
+            const int j = lane + 32 * r;
+            if (j < H8) hv[r] = ld_stream_v4(hrow + j);
+          }
+        }
+        const float g = gate_warp_pre(hv, wv, hrow, wg, H8, lane);
+        if (lane == 0) sm->g[t] = g;
+      }
+    }
+  };
   int32_t ticket = -1;
   float s_two[2] = {0.f, 0.f};                               // two-order forms: this thread's token's row scales
-  if constexpr (MODE == kRowsIds2) {
-    if (tid < T) {
-      const int2 id = reinterpret_cast<const int2*>(a.ids)[tid];
-      sm->rid[tid][0] = id.x;
-      sm->rid[tid][1] = a.rows0 + id.y;
-      s_two[0] = __ldg(a.scales + id.x);
-      s_two[1] = __ldg(a.scales + a.rows0 + id.y);
-    }
-    __syncthreads();                                         // row IDs ready
-  }
   if constexpr (FUSED) {
     // row IDs: thread t hashes token t (for the multi-head layout, thread (t, head))
     constexpr int kIdsPerTok = FMT == 2 ? kHeads : 1;
@@ -408,34 +438,32 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
         }
       }
     }
+    gates();                                                 // under the hash's loads
     __syncthreads();                                         // row IDs ready: this CTA has read the history
     // count this CTA in; the last CTA to arrive writes the new history at the end,
     // when no CTA of the grid can still read the old one (the ticket is used only then)
     if (tid == 0) ticket = atomicAdd(a.step_count, 1);
   }
-  if constexpr (TWO) {
+  if constexpr (MODE == kRowsHash2) {
     // this warp's K range (chunks of 16 codes, lane l takes chunk kb + l) of A
-    // rows r = 0..15: token r & 7, order r >> 3; two batches of 8 rows, each
-    // batch's loads in flight before any is used
+    // rows r = 0..15: token r & 7, order r >> 3; all 16 rows' loads in flight
+    // before any is used (from a cold L2 the gather is one HBM round trip)
     const int nck = ke - kb;
+    RowChunk<FMT == 1> x[kPjMaxTok];
 #pragma unroll
-    for (int r0 = 0; r0 < kPjMaxTok; r0 += 8) {
-      RowChunk<FMT == 1> x[8];
+    for (int rr = 0; rr < kPjMaxTok; ++rr) {
+      const int t = rr & 7;
+      if (t < T && lane < nck) x[rr] = load_chunk<FMT == 1>(a.table, a.blocks, sm->rid[t][rr >> 3], a.D, kb + lane);
+    }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = r0 + i, t = rr & 7;
-        if (t < T && lane < nck) x[i] = load_chunk<FMT == 1>(a.table, a.blocks, sm->rid[t][rr >> 3], a.D, kb + lane);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = r0 + i, t = rr & 7;
-        if (t < T && lane < nck) {
-          uint4 o0, o1;
-          codes_to_f16<FMT == 1>(x[i], o0, o1);
-          uint4* dst = reinterpret_cast<uint4*>(es + rr * ldr + (kb + lane) * 16);
-          dst[0] = o0;
-          dst[1] = o1;
-        }
+    for (int rr = 0; rr < kPjMaxTok; ++rr) {
+      const int t = rr & 7;
+      if (t < T && lane < nck) {
+        uint4 o0, o1;
+        codes_to_f16<FMT == 1>(x[rr], o0, o1);
+        uint4* dst = reinterpret_cast<uint4*>(es + rr * ldr + (kb + lane) * 16);
+        dst[0] = o0;
+        dst[1] = o1;
       }
     }
     if (tid < T) {
@@ -486,30 +514,22 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
       }
     }
   }
-  if (!a.gate_ready) {
-    for (int t = warp; t < T; t += kPjWarps) {
-      const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + static_cast<int64_t>(t) * a.H);
-      if (t != warp) {
-#pragma unroll
-        for (int r = 0; r < kEmbedH4; ++r) {
-          const int j = lane + 32 * r;
-          if (j < H8) hv[r] = ld_stream_v4(hrow + j);
-        }
-      }
-      const float g = gate_warp_pre(hv, wv, hrow, wg, H8, lane);
-      if (lane == 0) sm->g[t] = g;
-    }
-  }
+  if constexpr (COPIED) gates();
   cp_async_wait_all();
   __syncthreads();                                           // every copy and every e row has landed
   if (a.gate_ready && tid < T) sm->g[tid] = sm->meta[tid].g;
+
+  // W_proj has landed (bounded: past the limit the status records a timeout and
+  // the products are skipped)
+  const bool w_ok = mbar_wait(wbar, 0);
+  if (!w_ok && tid == 0) set_status(a.status, PLE_ERR_TIMEOUT);
 
   // ---- 3. products over this warp's K range: tokens (A, rows of e) x channels
   //         (B, rows of W_proj), one accumulator per 8-channel group
   float acc[kPjMaxGroups][4];
 #pragma unroll
   for (int g = 0; g < kPjMaxGroups; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
-  {
+  if (w_ok) {
     // ldmatrix.x4 for A: matrix m = lane / 8 covers token rows (m & 1) * 8 + 0..7 and
     // K offset (m >> 1) * 8; rows past T repeat the last token (their sums are unused)
     const int am = lane >> 3;
@@ -609,6 +629,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
     }
     if (FUSED) *a.step_count = 0;                            // ready for the next step
   }
+  if (!w_ok) mbar_wait(wbar, 0);                             // copies in flight land before the CTA leaves
 }
 
 template <typename Kernel, typename Args>
@@ -641,7 +662,7 @@ cudaError_t launch_decode_embed(const DecodeEmbedArgs& a, cudaStream_t stream) {
   if (r != cudaSuccess) return r;
   const int T = a.B * a.q;
   const int nch = a.D / 16;
-  const int threads = std::min(512, std::max(32, (nch + 31) / 32 * 32));
+  const int threads = std::min(kEmbedThreads, std::max(32, (nch + 31) / 32 * 32));
   const dim3 grid(a.w16 != nullptr ? std::max(T, a.prefetch_blocks) : T), block(threads);
   if (a.format == PLE_TABLE_E4M3_HEADS) return launch_pdl(decode_embed_kernel<2>, grid, block, 0, a, stream);
   if (a.format == PLE_TABLE_NVFP4) return launch_pdl(decode_embed_kernel<1>, grid, block, 0, a, stream);
@@ -662,6 +683,10 @@ bool decode_proj_plan(int32_t H, int32_t D, int32_t num_sms, DecodeProjPlan* pla
 
 bool decode_proj_supported(int32_t B, int32_t q) { return static_cast<int64_t>(B) * q <= kPjMaxTok; }
 
+bool decode_two_order(int32_t T, int32_t format) {
+  return T <= kTwoOrderMaxTok && (format == PLE_TABLE_E4M3 || format == PLE_TABLE_NVFP4);
+}
+
 cudaError_t launch_decode_proj(const DecodeProjArgs& a, const DecodeProjPlan& plan, cudaStream_t stream) {
   static PerDeviceOnce configured;
   const cudaError_t e = configured.run([] {
@@ -677,22 +702,20 @@ cudaError_t launch_decode_proj(const DecodeProjArgs& a, const DecodeProjPlan& pl
     set(decode_proj_kernel<2, kRowsHash>);
     set(decode_proj_kernel<0, kRowsHash2>);
     set(decode_proj_kernel<1, kRowsHash2>);
-    set(decode_proj_kernel<0, kRowsIds2>);
-    set(decode_proj_kernel<1, kRowsIds2>);
+    set(decode_proj_kernel<0, kRowsCodes2>);
     return x;
   });
   if (e != cudaSuccess) return e;
   DecodeProjArgs b = a;
   b.max_groups = plan.max_groups;
   const int T = a.B * a.q;
-  const bool two = a.format != PLE_TABLE_E4M3_HEADS && T <= kTwoOrderMaxTok;
+  const bool two = decode_two_order(T, a.format);
   const size_t smem = proj_smem_bytes(plan.max_groups, a.D, two ? kPjMaxTok : T);
   const dim3 grid(plan.grid), block(kPjThreads);
   const bool nv = a.format == PLE_TABLE_NVFP4;
-  if (a.e != nullptr) {                                      // rows prepared by decode_embed_kernel
+  if (a.e != nullptr) {                                      // rows or codes from decode_embed_kernel
     if (!two) return launch_pdl(decode_proj_kernel<0, kRowsE>, grid, block, smem, b, stream);
-    if (nv) return launch_pdl(decode_proj_kernel<1, kRowsIds2>, grid, block, smem, b, stream);
-    return launch_pdl(decode_proj_kernel<0, kRowsIds2>, grid, block, smem, b, stream);
+    return launch_pdl(decode_proj_kernel<0, kRowsCodes2>, grid, block, smem, b, stream);
   }
   if (two) {
     if (nv) return launch_pdl(decode_proj_kernel<1, kRowsHash2>, grid, block, smem, b, stream);

@@ -204,8 +204,9 @@ struct DecodeEmbedArgs {
   int32_t D, H;
   const __nv_bfloat16* hidden;   // [T][H], or null: the gate is computed later
   const __nv_bfloat16* w_gate;
-  __half* e;               // [T][D]
-  int32_t* ids;            // [T][2] row IDs (two-order table formats; null: not written)
+  __half* e;               // [T][D]; with codes2, [16][D]: token t's two rows as exact fp16 codes in rows t and t + 8
+  float* row_scales;       // with codes2: [T][2], the two rows' scales
+  int32_t codes2;          // 1: e takes the codes and row_scales the scales (decode_two_order steps)
   TokMeta* meta;           // [T]
   const __half* w16;       // fp16 W_proj, prefetched into L2 for the kernel after this one (null: none)
   int64_t w16_bytes;
@@ -214,6 +215,9 @@ struct DecodeEmbedArgs {
 };
 cudaError_t launch_decode_embed(const DecodeEmbedArgs& a, cudaStream_t stream);
 uint64_t barrett_magic(int64_t m);
+// Steps of up to 8 tokens of a two-order table (E4M3 or NVFP4) run the
+// channel-split kernel on exact codes with the row scales after the products.
+bool decode_two_order(int32_t T, int32_t format);
 
 // decode_proj_kernel, for steps of B * q <= 16 tokens: the projection, gate,
 // conv against the carried state, residual and state commit, one CTA per SM.
@@ -221,10 +225,10 @@ uint64_t barrett_magic(int64_t m);
 // partial sums cross CTAs and no CTA waits for another. With e null the
 // kernel also computes the row IDs and gathers, in each warp, the K range of
 // every token's rows that the warp multiplies (the whole step in one kernel);
-// otherwise it reads the rows (or, for steps of up to 8 tokens, the row IDs)
-// decode_embed_kernel wrote. Up to 8 tokens of a two-order table run as 16
-// mma rows of exact codes (order 0 and order 1 of each token) with the row
-// scales applied after the products.
+// otherwise it reads what decode_embed_kernel wrote: the rows, or for
+// decode_two_order steps the codes and row scales. Up to 8 tokens of a
+// two-order table run as 16 mma rows of exact codes (order 0 and order 1 of
+// each token) with the row scales applied after the products.
 struct DecodeProjArgs {
   const int32_t* tokens;   // [B][q] (the rows of a fused step, and the new token history)
   int32_t B, q;
@@ -232,8 +236,9 @@ struct DecodeProjArgs {
   float* conv_state;       // [B][3][H] in/out
   const int32_t* n_commit; // [B] or null
   const __half* w16;       // fp16 W_proj [H][D] (K-major)
-  const __half* e;         // [T][D] from decode_embed_kernel, or null: the kernel gathers the rows itself
-  const int32_t* ids;      // [T][2] from decode_embed_kernel (with e; read for steps of up to 8 tokens)
+  const __half* e;         // from decode_embed_kernel ([T][D] rows, or [16][D] codes), or null: the kernel
+                           // gathers the rows itself
+  const float* row_scales; // [T][2] from decode_embed_kernel (with e, decode_two_order steps)
   const TokMeta* meta;     // [T]
   int32_t gate_ready;      // 1: meta[t].g holds the gate; 0: each CTA computes it from hidden
   // the table, for a step whose rows the kernel gathers itself (e null)

@@ -299,71 +299,95 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         const TokMeta* Mm = reinterpret_cast<const TokMeta*>(Ms);
         const float* Cf = reinterpret_cast<const float*>(Cs);
         // Each thread owns its channel's row of every staged array, so the three
-        // passes below need no barrier between them. 1. The gated sums u, every
-        // token independent: the splits' sums are added in split order, four
-        // tokens' loads in flight at once; u overwrites split 0's slot.
+        // passes below need no barrier between them. With one epilogue warp per
+        // scheduler, each pass keeps a batch of tokens' loads in flight before any
+        // of them is used. 1. The gated sums u: 16 tokens at a time, the splits'
+        // sums added in split order; u overwrites split 0's slot.
+        // The loads of a batch are unconditional (a token index past the chunk
+        // reads the chunk's last token again), so that no branch splits them.
         float* Uf = reinterpret_cast<float*>(P);
-        for (int tq = 0; tq < nt; tq += 4) {
-          float part[4][kMtpMaxSplits];
+        for (int tq = 0; tq < nt; tq += 16) {
+          int off[16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float* pt = Pf + (tq + j) * kMtM + row;
+          for (int j = 0; j < 16; ++j) off[j] = min(tq + j, nt - 1) * kMtM + row;
+          float v[16];
 #pragma unroll
-            for (int sp = 0; sp < kMtpMaxSplits; ++sp)
-              part[j][sp] = (tq + j < nt && sp < a.k_splits) ? pt[sp * nt * kMtM] : 0.f;
+          for (int j = 0; j < 16; ++j) v[j] = 0.f;
+#pragma unroll 2
+          for (int sp = 0; sp < a.k_splits; ++sp) {
+            const float* ps = Pf + sp * nt * kMtM;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += ps[off[j]];
           }
+          float g[16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (tq + j < nt) {
-              float v = 0.f;
+          for (int j = 0; j < 16; ++j) g[j] = Mm[min(tq + j, nt - 1)].g;
 #pragma unroll
-              for (int sp = 0; sp < kMtpMaxSplits; ++sp)
-                if (sp < a.k_splits) v += part[j][sp];
-              Uf[(tq + j) * kMtM + row] = Mm[tq + j].g * v;
-            }
-          }
+          for (int j = 0; j < 16; ++j)
+            if (tq + j < nt) Uf[off[j]] = g[j] * v[j];
         }
-        // 2. the outputs, every token independent: the conv reads the sequence's
+        // 2. the outputs, 8 tokens at a time: the conv reads the sequence's
         //    extended stream (three carried entries, then its tokens' u), token i
         //    taps entries i, i + 1, i + 2 and its own u
         {
-          int sb = 0, i = 0;
-#pragma unroll 4
-          for (int tc = 0; tc < nt; ++tc) {
-            const float* xc = Cf + sb * 3 * kMtM + row;
-            const float* xu = Uf + (tc - i) * kMtM + row;
-            const float e0 = i >= 3 ? xu[(i - 3) * kMtM] : xc[i * kMtM];
-            const float e1 = i >= 2 ? xu[(i - 2) * kMtM] : xc[(i + 1) * kMtM];
-            const float e2 = i >= 1 ? xu[(i - 1) * kMtM] : xc[(i + 2) * kMtM];
-            const float u = xu[i * kMtM];
-            const float y = cw.x * e0 + cw.y * e1 + cw.z * e2 + cw.w * u;
-            const int64_t idx = static_cast<int64_t>(t0 + tc) * a.H + ch;
-            const float o = __bfloat162float(Hb[tc * kMtM + row]) + y;
-            if (a.out_f32) reinterpret_cast<float*>(a.out)[idx] = o;
-            else reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(o);
-            if (++i == a.q) {
-              i = 0;
-              ++sb;
+          int sb = 0, i = 0;                               // sequence and position of token tq
+          for (int tq = 0; tq < nt; tq += 8) {
+            float e0[8], e1[8], e2[8], u[8], hv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              // past the chunk's end: the last token's entries again (unused)
+              const int tc = min(tq + j, nt - 1);
+              const int ic = tq + j < nt ? i : a.q - 1, sc = tq + j < nt ? sb : ns - 1;
+              const float* xc = Cf + sc * 3 * kMtM + row;
+              const float* xu = Uf + (tc - ic) * kMtM + row;
+              e0[j] = *(ic >= 3 ? xu + (ic - 3) * kMtM : xc + ic * kMtM);
+              e1[j] = *(ic >= 2 ? xu + (ic - 2) * kMtM : xc + (ic + 1) * kMtM);
+              e2[j] = *(ic >= 1 ? xu + (ic - 1) * kMtM : xc + (ic + 2) * kMtM);
+              u[j] = xu[ic * kMtM];
+              hv[j] = __bfloat162float(Hb[tc * kMtM + row]);
+              if (++i == a.q) {
+                i = 0;
+                ++sb;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (tq + j < nt) {
+                const float y = cw.x * e0[j] + cw.y * e1[j] + cw.z * e2[j] + cw.w * u[j];
+                const int64_t idx = static_cast<int64_t>(t0 + tq + j) * a.H + ch;
+                const float o = hv[j] + y;
+                if (a.out_f32) reinterpret_cast<float*>(a.out)[idx] = o;
+                else reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(o);
+              }
             }
           }
         }
-        // 3. the carried state: the three entries of the extended stream that end
-        //    at the sequence's last committed token
-        for (int sb = 0; sb < ns; ++sb) {
-          int32_t ncb = a.n_commit ? reinterpret_cast<const int32_t*>(Ns)[sb] : a.q;
-          if (ncb < 1 || ncb > a.q) {
-            if (et == 0 && m == 0) set_status(a.status, PLE_ERR_RANGE);
-            ncb = max(1, min(ncb, a.q));
-          }
-          const float* xc = Cf + sb * 3 * kMtM + row;
-          const float* xu = Uf + sb * a.q * kMtM + row;
-          float k[3];
+        // 3. the carried state, 4 sequences at a time: the three entries of the
+        //    extended stream that end at the sequence's last committed token
+        for (int sq = 0; sq < ns; sq += 4) {
+          float k[4][3];
 #pragma unroll
-          for (int j = 0; j < 3; ++j) k[j] = ncb + j >= 3 ? xu[(ncb + j - 3) * kMtM] : xc[(ncb + j) * kMtM];
-          float* cs = a.conv_state + static_cast<int64_t>(bc + sb) * 3 * a.H + ch;
-          cs[0] = k[0];
-          cs[a.H] = k[1];
-          cs[2 * a.H] = k[2];
+          for (int j = 0; j < 4; ++j) {
+            const int sb = min(sq + j, ns - 1);
+            int32_t ncb = a.n_commit ? reinterpret_cast<const int32_t*>(Ns)[sb] : a.q;
+            if (ncb < 1 || ncb > a.q) {
+              if (et == 0 && m == 0) set_status(a.status, PLE_ERR_RANGE);
+              ncb = max(1, min(ncb, a.q));
+            }
+            const float* xc = Cf + sb * 3 * kMtM + row;
+            const float* xu = Uf + sb * a.q * kMtM + row;
+#pragma unroll
+            for (int r = 0; r < 3; ++r) k[j][r] = *(ncb + r >= 3 ? xu + (ncb + r - 3) * kMtM : xc + (ncb + r) * kMtM);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (sq + j < ns) {
+              float* cs = a.conv_state + static_cast<int64_t>(bc + sq + j) * 3 * a.H + ch;
+              cs[0] = k[j][0];
+              cs[a.H] = k[j][1];
+              cs[2 * a.H] = k[j][2];
+            }
+          }
         }
         named_bar_sync(1, kMtEpiThreads);                  // the staging area is reused by the next chunk
       }

@@ -239,8 +239,13 @@ ple_status ple_decode_step(ple_handle* handle, const int32_t* tokens, int32_t B,
  * the SSD-stream model card ("Qwen3.8 Flash-Next NVFP4 - SSD Stream", section
  * "技术细节") fetches the rows before the model reaches the block that uses
  * them. ple_decode_prepare takes the tokens [B][q] and the token history
- * hist [B][2] that ple_decode_step would take, and leaves the step's
- * dequantised rows and per-token metadata in the handle's scratch.
+ * hist [B][2] that ple_decode_step would take, and leaves the step's rows
+ * and per-token metadata in the handle's scratch: for a step of up to 8
+ * tokens of an E4M3 or NVFP4 table, each token's two rows as exact fp16 codes
+ * with their two row scales (the step then reads them in one round trip and
+ * applies the scales after the products, as ple_decode_step does); otherwise
+ * the dequantised rows. The form is chosen here, with the path selection of
+ * ple_set_forward_path in force at this call.
  * ple_decode_step_prepared then takes the rest of ple_decode_step's arguments
  * and runs the gate, the projection, the conv, the residual and the state
  * update. Together they give ple_decode_step's result bit for bit.

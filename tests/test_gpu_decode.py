@@ -138,6 +138,32 @@ def test_decode_step_bits_repeat(full_layer, shape):  # noqa: F811
         assert np.array_equal(again[2], first[2])
 
 
+@pytest.mark.parametrize("shape", [(4, 1), (2, 3), (12, 1)])
+def test_decode_prepared_route_fixed_at_prepare(mid_layer, shape):
+    """ple_decode_prepare chooses the form of the rows it leaves (exact codes and
+    row scales for steps of up to 8 tokens, else dequantised rows) with the path in
+    force then: a path change before ple_decode_step_prepared leaves the step as
+    it was prepared, equal bit for bit to ple_decode_step under the first path."""
+    from ple_inputs.device import bf16_tensor
+    L = mid_layer
+    B, q = shape
+    toks, hid, hist, conv, nc = _inputs(L.w, B, q, 11 + B)
+    ref = _run(L, toks, hid, hist, conv, nc, prepared=False)
+    tk, hs = _i32(toks), _i32(hist)
+    cs = torch.from_numpy(np.ascontiguousarray(conv)).cuda()
+    out = torch.empty(B * q, L.w.hidden, dtype=torch.float32, device="cuda")
+    ple.ple_decode_prepare(L.handle, tk, B, q, hs)
+    ple.ple_set_forward_path(L.handle, 2)
+    try:
+        ple.ple_decode_step_prepared(L.handle, bf16_tensor(hid), out, 1, hs, cs, _i32(nc))
+    finally:
+        ple.ple_set_forward_path(L.handle, 0)
+    torch.cuda.synchronize()
+    assert ple.ple_get_error(L.handle) == 0
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), ref[0])
+    assert np.array_equal(hs.cpu().numpy(), ref[1]) and np.array_equal(cs.cpu().numpy(), ref[2])
+
+
 def test_decode_prepared_errors(tiny_layer):
     L = tiny_layer
     w = L.w
