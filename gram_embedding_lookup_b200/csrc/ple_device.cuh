@@ -349,6 +349,21 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// The same barrier, returning whether pred held for any of the threads: a
+// decision every thread of the group then takes alike.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------------ E4M3 dequantisation
 // e = fp16(a * s0 + b * s1) for 16 codes of two table rows (a, b): each code is
 // decoded exactly (E4M3 -> fp16 -> fp32 conversions; NaN codes stay NaN), the
@@ -585,6 +600,21 @@ __device__ __forceinline__ float gate_warp_row(const uint4* hrow, const uint4* w
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
                : "memory");
+}
+
+// ------------------------------------------------------------------ bulk copies shared -> global
+// One contiguous copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) in the calling thread's current bulk group.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+
+// Orders this thread's global accesses in the async proxy (bulk copies) with
+// its generic ones, both ways.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ bulk copies global -> shared

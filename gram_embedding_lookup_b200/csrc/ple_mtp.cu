@@ -24,9 +24,9 @@
 // grid never exceeds the SM count (one CTA per SM by its shared memory); a CTA
 // that still waits after about a second records PLE_ERR_TIMEOUT and leaves.
 //
-// Warp roles (192 threads): warp 0 issues the TMA loads, warp 1 owns TMEM and
-// issues tcgen05.mma, warps 2-5 (one TMEM lane quarter each) run the
-// epilogue.
+// Warp roles (320 threads): warp 0 issues the TMA loads, warp 1 owns TMEM and
+// issues tcgen05.mma, warps 2-9 run the epilogue (two per TMEM lane quarter,
+// each taking every other 32-token column block).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
@@ -44,11 +44,11 @@ namespace {
 constexpr int kMtM = 128;                 // channels per CTA (TMEM lanes)
 constexpr int kMtBK = 64;                 // K per stage: one 128-byte swizzled row of fp16
 constexpr int kMtUmmaK = 16;
-constexpr int kMtThreads = 192;
+constexpr int kMtThreads = 320;
 constexpr int kMtTmaWarp = 0;
 constexpr int kMtMmaWarp = 1;
 constexpr int kMtEpiWarp0 = 2;
-constexpr int kMtEpiThreads = 128;
+constexpr int kMtEpiThreads = 256;
 constexpr int kMtStages = 5;              // most stages; fewer when 256 tokens do not leave room
 constexpr uint32_t kMtAStage = kMtM * kMtBK * 2;   // 16 KB
 constexpr uint32_t kMtTmemCols = 256;
@@ -195,12 +195,17 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       if (ok) mma_commit(smem_u32(&bars->tfull));
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-5)
-    const int et = threadIdx.x - 32 * kMtEpiWarp0;          // 0..127
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;                     // channel inside the tile
-    const int ch = m * kMtM + row;
-    const float4 cw = __ldg(reinterpret_cast<const float4*>(a.conv_w) + ch);
+    // ------------------------------------------------------------ epilogue (warps 2-9)
+    const int et = threadIdx.x - 32 * kMtEpiWarp0;          // 0..255
+    const int quarter = warp & 3, half = (warp - kMtEpiWarp0) >> 2;
+    const int row = quarter * 32 + lane;                     // TMEM lane: channel inside the tile
+    // in the split sums: lane c4 of each warp takes channels 4 c4 .. 4 c4 + 3 of
+    // the tile, warp ph (0..7) every 8th token or sequence from ph
+    const int c4 = et & 31, ph = et >> 5;
+    const float4 cw0 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + m * kMtM + 4 * c4);
+    const float4 cw1 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + m * kMtM + 4 * c4 + 1);
+    const float4 cw2 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + m * kMtM + 4 * c4 + 2);
+    const float4 cw3 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + m * kMtM + 4 * c4 + 3);
     pdl_launch_dependents();
     pdl_wait();                                              // gates, hidden and the state are ready
     // the new token history, while the products run (the embed kernel, the only
@@ -218,23 +223,73 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     float* slab = a.partial + static_cast<int64_t>(m) * a.k_splits * a.n_pad * kMtM;
     bool ok = wait_bar(smem_u32(&bars->tfull), 0, abort_flag, a.status);
     if (ok) {
+      // this split's sums [T][128] into shared memory (the operand stages are
+      // free: every MMA has completed), then to the slab in one bulk copy
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-      float* mine = slab + static_cast<int64_t>(ks) * a.n_pad * kMtM + row;
-      for (int c = 0; c * 32 < T; ++c) {
+      float* St = reinterpret_cast<float*>(smem);
+      for (int c = half; c * 32 < T; c += 2) {
         float v[32];
         tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(c * 32), v);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (c * 32 + j < T) __stcg(mine + static_cast<int64_t>(c * 32 + j) * kMtM, v[j]);
+          if (c * 32 + j < T) St[(c * 32 + j) * kMtM + row] = v[j];
       }
+      fence_proxy_async_smem();                              // the bulk copy reads these writes
     }
     tc_fence_before();
+    ok = !named_bar_or(1, kMtEpiThreads, !ok);              // one decision for the whole epilogue
+    // This CTA's share of the sequences, all 128 channels of the tile, runs in
+    // chunks of whole sequences. Everything a chunk needs goes into shared memory
+    // at once: the splits' sums by bulk copies (from the start of the staging
+    // area), hidden at the tile's channels, the gates, the carried state and
+    // n_commit by cp.async (the side arrays, at the end of the area), so a chunk
+    // costs one round trip to L2. The first chunk's side arrays need no split
+    // sums: they are loaded now, under the meet, when they clear this split's
+    // sums on their way out.
+    const int b0 = ks * a.B / a.k_splits, b1 = (ks + 1) * a.B / a.k_splits;
+    const uint32_t region = static_cast<uint32_t>(S) * (kMtAStage + b_stage);
+    const uint32_t per_seq = static_cast<uint32_t>(a.q) * (a.k_splits * 512u + 256u + 16u) + 3u * 512u + 32u;
+    const int max_seqs = max(1, static_cast<int>(region / per_seq));
+    auto side_bytes = [&](int ns) -> uint32_t {
+      return (static_cast<uint32_t>(ns) * (a.q * 272u + 3u * 512u + 4u) + 15u) & ~15u;
+    };
+    // threads [first, first + n) of the epilogue issue the side loads
+    auto load_side = [&](int bc, int ns, int first, int n) {
+      const int nt = ns * a.q, t0 = bc * a.q;
+      const int lt = et - first;
+      if (lt < 0) return;
+      uint8_t* Hs = smem + region - side_bytes(ns);               // [nt][128] bf16
+      uint8_t* Ms = Hs + static_cast<size_t>(nt) * 256;          // [nt] TokMeta
+      uint8_t* Cs = Ms + static_cast<size_t>(nt) * 16;           // [ns][3][128] f32
+      uint8_t* Ns = Cs + static_cast<size_t>(ns) * 3 * 512;      // [ns] n_commit
+      for (int x = lt; x < nt * 16; x += n) {
+        const int tk = x >> 4, c16 = x & 15;
+        cp_async_16(smem_u32(Hs + tk * 256 + c16 * 16), a.hidden + static_cast<int64_t>(t0 + tk) * a.H + m * kMtM + c16 * 8);
+      }
+      for (int x = lt; x < nt; x += n) cp_async_16(smem_u32(Ms + x * 16), a.meta + t0 + x);
+      for (int x = lt; x < ns * 3 * 32; x += n) {
+        const int r3 = x >> 5, c32 = x & 31;
+        cp_async_16(smem_u32(Cs + r3 * 512 + c32 * 16),
+                    a.conv_state + (static_cast<int64_t>(bc) * 3 + r3) * a.H + m * kMtM + c32 * 4);
+      }
+      if (a.n_commit != nullptr)
+        for (int x = lt; x < ns; x += n) cp_async_4(smem_u32(Ns + x * 4), a.n_commit + bc + x);
+      cp_async_commit();
+    };
+    const bool side_early = ok && b0 < b1 &&
+                            region - side_bytes(min(max_seqs, b1 - b0)) >= static_cast<uint32_t>(T) * 512u;
+    if (side_early) load_side(b0, min(max_seqs, b1 - b0), 32, kMtEpiThreads - 32);   // not warp 2: it counts in
     // ---- the tile's splits meet: count in, wait (bounded) for the others
-    __threadfence();
-    named_bar_sync(1, kMtEpiThreads);
     __shared__ int32_t go;
     if (et == 0) {
+      if (ok) {
+        bulk_store(slab + static_cast<int64_t>(ks) * a.n_pad * kMtM, smem_u32(smem), static_cast<uint32_t>(T) * 512u);
+        bulk_commit_group();
+        bulk_wait_group<0>();
+        fence_proxy_async_global();                          // the copy's writes before the count
+        __threadfence();
+      }
       int32_t arrived = ok ? atomicAdd(a.tile_count + m, 1) + 1 : 0;
       const long long start = clock64();
       while (ok && arrived < a.k_splits) {
@@ -249,145 +304,121 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     }
     named_bar_sync(1, kMtEpiThreads);
     if (go) {
-      // ---- this CTA's share of the sequences, all 128 channels of the tile, in chunks
-      //      of whole sequences. Everything a chunk needs goes into shared memory at
-      //      once (the operand stages are free: every MMA has completed): the
-      //      splits' sums by bulk copies, hidden at the tile's channels, the gates
-      //      and the carried state by 16-byte cp.async, so a chunk costs one round
-      //      trip to L2. Then each thread runs its channel.
-      const int b0 = ks * a.B / a.k_splits, b1 = (ks + 1) * a.B / a.k_splits;
-      const uint32_t region = static_cast<uint32_t>(S) * (kMtAStage + b_stage);
-      const uint32_t per_seq = static_cast<uint32_t>(a.q) * (a.k_splits * 512u + 256u + 16u) + 3u * 512u + 4u;
-      const int max_seqs = max(1, static_cast<int>(region / per_seq));
       const uint32_t staged_bar = smem_u32(&bars->staged);
       uint32_t chunk_parity = 0;
       for (int bc = b0; bc < b1 && go; bc += max_seqs) {
         const int ns = min(max_seqs, b1 - bc);
         const int nt = ns * a.q, t0 = bc * a.q;
         uint8_t* P = smem;                                           // [k_splits][nt][128] f32
-        uint8_t* Hs = P + static_cast<size_t>(a.k_splits) * nt * 512;   // [nt][128] bf16
-        uint8_t* Ms = Hs + static_cast<size_t>(nt) * 256;              // [nt] TokMeta
-        uint8_t* Cs = Ms + static_cast<size_t>(nt) * 16;               // [ns][3][128] f32
-        uint8_t* Ns = Cs + static_cast<size_t>(ns) * 3 * 512;          // [ns] n_commit
-        if (et == 0) {
-          mbar_arrive_expect_tx(staged_bar, static_cast<uint32_t>(a.k_splits) * nt * 512u);
-          for (int sp = 0; sp < a.k_splits; ++sp)
-            bulk_load(smem_u32(P + static_cast<size_t>(sp) * nt * 512),
-                      slab + (static_cast<int64_t>(sp) * a.n_pad + t0) * kMtM, static_cast<uint32_t>(nt) * 512u,
+        uint8_t* Hs = smem + region - side_bytes(ns);                // the side arrays, as load_side puts them
+        uint8_t* Ms = Hs + static_cast<size_t>(nt) * 256;
+        uint8_t* Cs = Ms + static_cast<size_t>(nt) * 16;
+        uint8_t* Ns = Cs + static_cast<size_t>(ns) * 3 * 512;
+        if (et < 32) {                                     // lane sp of warp 2 copies split sp
+          if (et == 0) mbar_arrive_expect_tx(staged_bar, static_cast<uint32_t>(a.k_splits) * nt * 512u);
+          __syncwarp();
+          if (et < a.k_splits) {
+            fence_proxy_async_global();                    // after the acquire: the others' sums
+            bulk_load(smem_u32(P + static_cast<size_t>(et) * nt * 512),
+                      slab + (static_cast<int64_t>(et) * a.n_pad + t0) * kMtM, static_cast<uint32_t>(nt) * 512u,
                       staged_bar);
+          }
         }
-        for (int x = et; x < nt * 16; x += kMtEpiThreads) {
-          const int tk = x >> 4, c16 = x & 15;
-          cp_async_16(smem_u32(Hs + tk * 256 + c16 * 16),
-                      a.hidden + static_cast<int64_t>(t0 + tk) * a.H + m * kMtM + c16 * 8);
-        }
-        for (int x = et; x < nt; x += kMtEpiThreads) cp_async_16(smem_u32(Ms + x * 16), a.meta + t0 + x);
-        for (int x = et; x < ns * 3 * 32; x += kMtEpiThreads) {
-          const int r3 = x >> 5, c32 = x & 31;
-          cp_async_16(smem_u32(Cs + r3 * 512 + c32 * 16),
-                      a.conv_state + (static_cast<int64_t>(bc) * 3 + r3) * a.H + m * kMtM + c32 * 4);
-        }
-        if (a.n_commit != nullptr)
-          for (int x = et; x < ns; x += kMtEpiThreads) cp_async_4(smem_u32(Ns + x * 4), a.n_commit + bc + x);
-        cp_async_commit();
+        if (!(side_early && bc == b0)) load_side(bc, ns, 0, kMtEpiThreads);
         cp_async_wait_all();
         named_bar_sync(1, kMtEpiThreads);
-        if (!wait_bar(staged_bar, chunk_parity, abort_flag, a.status)) break;
+        const bool landed = wait_bar(staged_bar, chunk_parity, abort_flag, a.status);
+        if (named_bar_or(1, kMtEpiThreads, !landed)) break;  // every thread leaves, or none
         chunk_parity ^= 1;
-        const float* Pf = reinterpret_cast<const float*>(P);
-        const __nv_bfloat16* Hb = reinterpret_cast<const __nv_bfloat16*>(Hs);
+        const float4* P4 = reinterpret_cast<const float4*>(P);      // [k_splits][nt][32] float4
+        const uint2* H4 = reinterpret_cast<const uint2*>(Hs);       // [nt][32]: 4 bf16
         const TokMeta* Mm = reinterpret_cast<const TokMeta*>(Ms);
-        const float* Cf = reinterpret_cast<const float*>(Cs);
-        // Each thread owns its channel's row of every staged array, so the three
-        // passes below need no barrier between them. With one epilogue warp per
-        // scheduler, each pass keeps a batch of tokens' loads in flight before any
-        // of them is used. 1. The gated sums u: 16 tokens at a time, the splits'
-        // sums added in split order; u overwrites split 0's slot.
-        // The loads of a batch are unconditional (a token index past the chunk
-        // reads the chunk's last token again), so that no branch splits them.
-        float* Uf = reinterpret_cast<float*>(P);
-        for (int tq = 0; tq < nt; tq += 16) {
-          int off[16];
+        const float4* C4 = reinterpret_cast<const float4*>(Cs);     // [ns][3][32]
+        float4* U4 = reinterpret_cast<float4*>(P);                  // u into split 0's slots
+        // With 128-bit accesses each thread runs 4 channels, and a batch of 4 of
+        // its tokens keeps that many loads in flight; loads are unconditional (an
+        // index past the chunk reads its last token again).
+        // 1. the gated sums u: the splits' sums added in split order
+        for (int tq = ph; tq < nt; tq += 4 * 8) {
+          int tk[4];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) off[j] = min(tq + j, nt - 1) * kMtM + row;
-          float v[16];
+          for (int j = 0; j < 4; ++j) tk[j] = min(tq + 8 * j, nt - 1);
+          float4 v[4];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0.f;
+          for (int j = 0; j < 4; ++j) v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 2
           for (int sp = 0; sp < a.k_splits; ++sp) {
-            const float* ps = Pf + sp * nt * kMtM;
+            const float4* ps = P4 + sp * nt * 32 + c4;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += ps[off[j]];
-          }
-          float g[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) g[j] = Mm[min(tq + j, nt - 1)].g;
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (tq + j < nt) Uf[off[j]] = g[j] * v[j];
-        }
-        // 2. the outputs, 8 tokens at a time: the conv reads the sequence's
-        //    extended stream (three carried entries, then its tokens' u), token i
-        //    taps entries i, i + 1, i + 2 and its own u
-        {
-          int sb = 0, i = 0;                               // sequence and position of token tq
-          for (int tq = 0; tq < nt; tq += 8) {
-            float e0[8], e1[8], e2[8], u[8], hv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              // past the chunk's end: the last token's entries again (unused)
-              const int tc = min(tq + j, nt - 1);
-              const int ic = tq + j < nt ? i : a.q - 1, sc = tq + j < nt ? sb : ns - 1;
-              const float* xc = Cf + sc * 3 * kMtM + row;
-              const float* xu = Uf + (tc - ic) * kMtM + row;
-              e0[j] = *(ic >= 3 ? xu + (ic - 3) * kMtM : xc + ic * kMtM);
-              e1[j] = *(ic >= 2 ? xu + (ic - 2) * kMtM : xc + (ic + 1) * kMtM);
-              e2[j] = *(ic >= 1 ? xu + (ic - 1) * kMtM : xc + (ic + 2) * kMtM);
-              u[j] = xu[ic * kMtM];
-              hv[j] = __bfloat162float(Hb[tc * kMtM + row]);
-              if (++i == a.q) {
-                i = 0;
-                ++sb;
-              }
+            for (int j = 0; j < 4; ++j) {
+              const float4 x = ps[tk[j] * 32];
+              v[j].x += x.x;
+              v[j].y += x.y;
+              v[j].z += x.z;
+              v[j].w += x.w;
             }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (tq + j < nt) {
-                const float y = cw.x * e0[j] + cw.y * e1[j] + cw.z * e2[j] + cw.w * u[j];
-                const int64_t idx = static_cast<int64_t>(t0 + tq + j) * a.H + ch;
-                const float o = hv[j] + y;
-                if (a.out_f32) reinterpret_cast<float*>(a.out)[idx] = o;
-                else reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(o);
-              }
-            }
-          }
-        }
-        // 3. the carried state, 4 sequences at a time: the three entries of the
-        //    extended stream that end at the sequence's last committed token
-        for (int sq = 0; sq < ns; sq += 4) {
-          float k[4][3];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int sb = min(sq + j, ns - 1);
-            int32_t ncb = a.n_commit ? reinterpret_cast<const int32_t*>(Ns)[sb] : a.q;
-            if (ncb < 1 || ncb > a.q) {
-              if (et == 0 && m == 0) set_status(a.status, PLE_ERR_RANGE);
-              ncb = max(1, min(ncb, a.q));
-            }
-            const float* xc = Cf + sb * 3 * kMtM + row;
-            const float* xu = Uf + sb * a.q * kMtM + row;
-#pragma unroll
-            for (int r = 0; r < 3; ++r) k[j][r] = *(ncb + r >= 3 ? xu + (ncb + r - 3) * kMtM : xc + (ncb + r) * kMtM);
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            if (sq + j < ns) {
-              float* cs = a.conv_state + static_cast<int64_t>(bc + sq + j) * 3 * a.H + ch;
-              cs[0] = k[j][0];
-              cs[a.H] = k[j][1];
-              cs[2 * a.H] = k[j][2];
+            const float g = Mm[tk[j]].g;
+            if (tq + 8 * j < nt) U4[tk[j] * 32 + c4] = make_float4(g * v[j].x, g * v[j].y, g * v[j].z, g * v[j].w);
+          }
+        }
+        named_bar_sync(1, kMtEpiThreads);                  // every u of the chunk is in place
+        // 2. the outputs: the conv reads the sequence's extended stream (three
+        //    carried entries, then its tokens' u); token i taps entries i, i + 1,
+        //    i + 2 and its own u
+        auto ext = [&](int sb, int e) -> float4 {          // entry e of sequence sb's stream
+          return e < 3 ? C4[(sb * 3 + e) * 32 + c4] : U4[(sb * a.q + e - 3) * 32 + c4];
+        };
+        for (int tq = ph; tq < nt; tq += 4 * 8) {
+          float4 x0[4], x1[4], x2[4], xu[4];
+          uint2 hv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int tc = min(tq + 8 * j, nt - 1);
+            const int sb = tc / a.q, i = tc - sb * a.q;
+            x0[j] = ext(sb, i);
+            x1[j] = ext(sb, i + 1);
+            x2[j] = ext(sb, i + 2);
+            xu[j] = ext(sb, i + 3);
+            hv[j] = H4[tc * 32 + c4];
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (tq + 8 * j < nt) {
+              const float2 h01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hv[j].x));
+              const float2 h23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hv[j].y));
+              const float o0 = h01.x + (cw0.x * x0[j].x + cw0.y * x1[j].x + cw0.z * x2[j].x + cw0.w * xu[j].x);
+              const float o1 = h01.y + (cw1.x * x0[j].y + cw1.y * x1[j].y + cw1.z * x2[j].y + cw1.w * xu[j].y);
+              const float o2 = h23.x + (cw2.x * x0[j].z + cw2.y * x1[j].z + cw2.z * x2[j].z + cw2.w * xu[j].z);
+              const float o3 = h23.y + (cw3.x * x0[j].w + cw3.y * x1[j].w + cw3.z * x2[j].w + cw3.w * xu[j].w);
+              const int64_t idx = static_cast<int64_t>(t0 + tq + 8 * j) * a.H + m * kMtM + 4 * c4;
+              if (a.out_f32) {
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + idx) = make_float4(o0, o1, o2, o3);
+              } else {
+                const __nv_bfloat162 b01 = __floats2bfloat162_rn(o0, o1), b23 = __floats2bfloat162_rn(o2, o3);
+                uint2 w;
+                w.x = *reinterpret_cast<const uint32_t*>(&b01);
+                w.y = *reinterpret_cast<const uint32_t*>(&b23);
+                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + idx) = w;
+              }
             }
           }
+        }
+        // 3. the carried state: the three entries of the extended stream that end
+        //    at the sequence's last committed token
+        for (int sq = ph; sq < ns; sq += 8) {
+          int32_t ncb = a.n_commit ? reinterpret_cast<const int32_t*>(Ns)[sq] : a.q;
+          if (ncb < 1 || ncb > a.q) {
+            if (c4 == 0 && m == 0) set_status(a.status, PLE_ERR_RANGE);
+            ncb = max(1, min(ncb, a.q));
+          }
+          const float4 k0 = ext(sq, ncb), k1 = ext(sq, ncb + 1), k2 = ext(sq, ncb + 2);
+          float4* cs = reinterpret_cast<float4*>(a.conv_state + static_cast<int64_t>(bc + sq) * 3 * a.H + m * kMtM) + c4;
+          cs[0] = k0;
+          cs[a.H / 4] = k1;
+          cs[2 * (a.H / 4)] = k2;
         }
         named_bar_sync(1, kMtEpiThreads);                  // the staging area is reused by the next chunk
       }
@@ -437,6 +468,10 @@ cudaError_t launch_mtp_proj(const CUtensorMap& tmap_w, const CUtensorMap& tmap_e
   if (e != cudaSuccess) return e;
   MtpProjArgs b = a;
   b.stages = mtp_stages(a.n_pad);
+  // the split's sums [T][128] f32 pass through the operand stages on their way out
+  if (static_cast<size_t>(a.B) * a.q * 512u >
+      static_cast<size_t>(b.stages) * (kMtAStage + static_cast<size_t>(a.n_pad) * kMtBK * 2))
+    return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(a.m_tiles * a.k_splits);
   cfg.blockDim = dim3(kMtThreads);
