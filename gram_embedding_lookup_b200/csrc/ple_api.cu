@@ -189,7 +189,7 @@ ple::TableRef table_ref(const ple_handle* h) {
 cudaError_t launch_embed_for(ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream) {
   int kernels = 1;
   const cudaError_t r = heads_layout(h)
-                            ? ple::launch_embed_heads(pa, table_ref(h), h->cfg.row_dim, e, stream, &kernels)
+                            ? ple::launch_embed_heads(pa, table_ref(h), h->cfg.row_dim, e, h->num_sms, stream, &kernels)
                             : ple::launch_embed(pa, table_ref(h), h->cfg.row_dim, e, h->num_sms, stream, &kernels);
   h->launches += kernels - 1;           // the stage counts one launch; large batches take two kernels
   return r;

@@ -88,7 +88,7 @@ cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D,
 // 16 head rows (ids [T][16]), the gate and metadata when a.meta is set, and
 // e[t] (the 16 dequantised rows side by side) when e is set; extra blocks do
 // the offsets check and the state work. a.rows0 is the rows per head sub-table.
-cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
+cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
                                cudaStream_t stream, int* kernels = nullptr);
 
 // Gather stage of the multi-head layout: ids [T][16] -> e [T][D].

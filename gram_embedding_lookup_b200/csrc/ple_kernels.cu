@@ -669,6 +669,231 @@ __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
   }
 }
 
+// ------------------------------------------------------------------ embed as a bulk-copy pipeline
+// The gather and gate blocks of embed_split_kernel as one persistent kernel
+// (2 CTAs per SM), after ids_meta_kernel, for the two-order layouts (E4M3,
+// NVFP4) when the rows and hidden rows start on 16-byte boundaries. (The
+// multi-head layout's 16 rows of 160 bytes per token keep the producer warp
+// busier than the split kernel's loads: it stays on embed_split_kernel.) Per CTA a ring of token stages, each the
+// token's rows (codes and, for NVFP4, block scales), its hidden row and a
+// header with the row scales:
+//   warp 0, producer: row IDs and scales of 32 tokens at a time (the next 32
+//     IDs in flight meanwhile); per token, when its stage is free, the bytes
+//     to expect, the bulk copies (cp.async.bulk) of the rows (NVFP4: codes and
+//     block scales apart) and the hidden row, the header, then its arrival on
+//     the stage's full barrier;
+//   warps 1-5, consumers: warp w takes the CTA's tokens w, w + 5, ..., each
+//     whole: the rows dequantised into e (a lane per 16-code chunk, 16-byte
+//     stores), then the gate from the staged hidden row in the order every
+//     gate path takes its sums. Warp w owns stages 2w and 2w + 1, so it meets
+//     each stage's phases in order.
+// The copy engine keeps about 200 KB per SM in flight, where a thread per
+// chunk holds 32 bytes. CTA c takes tokens T - 1 - c, T - 1 - c - grid, ...:
+// the first tokens' rows are the last written, still in L2 when the
+// projection starts on them. Every wait is bounded and taken alike by a whole
+// warp; past the limit the status records a timeout, an abort flag releases
+// the other waits, and the producer waits (bounded) for the copies it issued
+// before the CTA leaves.
+constexpr int kBkConsWarps = 5;
+constexpr int kBkStagesPerWarp = 2;
+constexpr int kBkStages = kBkConsWarps * kBkStagesPerWarp;
+constexpr int kBkThreads = 32 * (1 + kBkConsWarps);
+constexpr int kBkCtasPerSm = 2;
+constexpr uint32_t kBkHeader = 16;          // the two fp32 row scales (and padding)
+
+// Token k of a CTA: consumer warp k % 5, stage 2 (k % 5) + (k / 5) % 2, the
+// (k / 10)-th use of that stage.
+__host__ __device__ __forceinline__ int bk_stage(int k) {
+  return (k % kBkConsWarps) * kBkStagesPerWarp + (k / kBkConsWarps) % kBkStagesPerWarp;
+}
+
+template <int FMT>
+__host__ __device__ __forceinline__ uint32_t bk_codes_bytes(int32_t D) {
+  return FMT == 1 ? 2u * static_cast<uint32_t>(D / 2 + D / 16) : 2u * D;
+}
+
+template <int FMT>
+__host__ __device__ __forceinline__ uint32_t bk_stage_bytes(int32_t D, int32_t H, bool gate) {
+  return ((bk_codes_bytes<FMT>(D) + 15u) & ~15u) + (gate ? 2u * H : 0u) + kBkHeader;
+}
+
+__device__ __forceinline__ bool bk_wait(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag, int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long start = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - start > kWaitLimitCycles) {
+      set_status(status, PLE_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kBkThreads, kBkCtasPerSm)
+    embed_bulk_kernel(const PrepareArgs a, const TableRef tab, int32_t D, __half* __restrict__ e, int32_t gate) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t full[kBkStages], empty[kBkStages];
+  __shared__ int32_t abort_word;
+  volatile int32_t* abort_flag = &abort_word;
+  static_assert(FMT == 0 || FMT == 1, "two-order layouts only");
+  constexpr int kRowsN = 2;                                  // rows (and scales) per token
+  constexpr uint32_t kStageUses = kBkStages;                 // tokens between two uses of a stage
+  const uint32_t hid_off = (bk_codes_bytes<FMT>(D) + 15u) & ~15u;
+  const uint32_t hdr_off = hid_off + (gate ? 2u * a.H : 0u);
+  const uint32_t SB = hdr_off + kBkHeader;
+  const uint32_t tx = bk_codes_bytes<FMT>(D) + (gate ? 2u * a.H : 0u);   // bytes a token's copies bring
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x, G = gridDim.x;
+  const int nk = c < a.T ? (a.T - 1 - c) / G + 1 : 0;       // this CTA's tokens
+  auto tok = [&](int k) { return a.T - 1 - (c + k * G); };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kBkStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    abort_word = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    pdl_wait();                                              // the row IDs
+    // lane l: the two row IDs of token k0 + l
+    int32_t cur[kRowsN], nxt[kRowsN];
+    auto load_ids = [&](int k0, int32_t (&v)[kRowsN]) {
+      const int k = k0 + lane;
+      if (k < nk) {
+        const int2 x = reinterpret_cast<const int2*>(a.ids)[tok(k)];
+        v[0] = x.x;
+        v[1] = x.y;
+      } else {
+#pragma unroll
+        for (int r = 0; r < kRowsN; ++r) v[r] = 0;
+      }
+    };
+    auto global_row = [&](int r, int32_t id) -> int64_t {   // row r of a token: its global row
+      return r == 0 ? static_cast<int64_t>(id) : a.rows0 + id;
+    };
+    load_ids(0, cur);
+    int issued = 0;
+    bool stop = false;                                       // warp-uniform
+    for (int k0 = 0; k0 < nk && !stop; k0 += 32) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      if (k0 + 32 < nk) load_ids(k0 + 32, nxt);
+      float sc[kRowsN];                                       // lane l: the row scales of token k0 + l
+#pragma unroll
+      for (int r = 0; r < kRowsN; ++r) sc[r] = k0 + lane < nk ? __ldg(tab.scales + global_row(r, cur[r])) : 0.f;
+      for (int j = 0; j < 32 && k0 + j < nk; ++j) {
+        const int k = k0 + j, s = bk_stage(k);
+        if (k >= kBkStages &&
+            !__all_sync(0xffffffffu, bk_wait(smem_u32(&empty[s]), (k / kStageUses - 1) & 1, abort_flag, a.status))) {
+          stop = true;
+          break;
+        }
+        const int t = tok(k);
+        uint8_t* st = smem + static_cast<size_t>(s) * SB;
+        const uint32_t fb = smem_u32(&full[s]);
+        if (lane == 0) mbar_expect_tx(fb, tx);
+        __syncwarp();
+        // lane r < kRowsN copies row r of token k
+        int32_t id = 0;
+#pragma unroll
+        for (int r = 0; r < kRowsN; ++r) {
+          const int32_t v = __shfl_sync(0xffffffffu, cur[r], j);
+          if (lane == r) id = v;
+        }
+        if (lane < kRowsN) {
+          const int64_t row = global_row(lane, id);
+          if constexpr (FMT == 1) {
+            const uint32_t o = lane * static_cast<uint32_t>(D / 2 + D / 16);
+            bulk_load(smem_u32(st + o), tab.codes + row * (D / 2), static_cast<uint32_t>(D / 2), fb);
+            bulk_load(smem_u32(st + o + D / 2), tab.blocks + row * (D / 16), static_cast<uint32_t>(D / 16), fb);
+          } else {
+            bulk_load(smem_u32(st + lane * D), tab.codes + row * D, static_cast<uint32_t>(D), fb);
+          }
+        }
+        if (gate && lane == 31)
+          bulk_load(smem_u32(st + hid_off), a.hidden + static_cast<int64_t>(t) * a.H, 2u * a.H, fb);
+        // the header: lane r < kRowsN writes row r's scale
+        float* hdr = reinterpret_cast<float*>(st + hdr_off);
+#pragma unroll
+        for (int r = 0; r < kRowsN; ++r) {
+          const float v = __shfl_sync(0xffffffffu, sc[r], j);
+          if (lane == r) hdr[r] = v;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(fb);
+        issued = k + 1;
+      }
+#pragma unroll
+      for (int r = 0; r < kRowsN; ++r) cur[r] = nxt[r];
+    }
+    // copies in flight land before the CTA's shared memory is released
+    for (int k = max(0, issued - kBkStages); k < issued; ++k) {
+      const long long start = clock64();
+      while (!mbar_try_wait(smem_u32(&full[bk_stage(k)]), (k / kStageUses) & 1) && clock64() - start < kWaitLimitCycles) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int w = warp - 1;
+    const int units = D / 16;
+    const int H8 = a.H / 8;
+    const uint4* wg = reinterpret_cast<const uint4*>(a.w_gate);
+    uint4 wv[kEmbedH4];
+    if (gate) {
+#pragma unroll
+      for (int r = 0; r < kEmbedH4; ++r) {
+        const int j = lane + 32 * r;
+        if (j < H8) wv[r] = __ldg(wg + j);
+      }
+    }
+    for (int k = w; k < nk; k += kBkConsWarps) {
+      const int s = bk_stage(k);
+      if (!__all_sync(0xffffffffu, bk_wait(smem_u32(&full[s]), (k / kStageUses) & 1, abort_flag, a.status))) break;
+      const uint8_t* st = smem + static_cast<size_t>(s) * SB;
+      const float* hdr = reinterpret_cast<const float*>(st + hdr_off);   // the two row scales
+      const int t = tok(k);
+      // the rows -> e: lane l takes chunks l, l + 32, ...
+      uint4* dst = reinterpret_cast<uint4*>(e + static_cast<int64_t>(t) * D);
+#pragma unroll 5
+      for (int j = lane; j < units; j += 32) {
+        uint4 o0, o1;
+        if constexpr (FMT == 1) {
+          const uint32_t rb = static_cast<uint32_t>(D / 2 + D / 16);
+          const uint2 ca = *reinterpret_cast<const uint2*>(st + j * 8);
+          const uint2 cb = *reinterpret_cast<const uint2*>(st + rb + j * 8);
+          deq16_nv(ca, cb, st[D / 2 + j], st[rb + D / 2 + j], hdr[0], hdr[1], o0, o1);
+        } else {
+          deq16(*reinterpret_cast<const uint4*>(st + j * 16), *reinterpret_cast<const uint4*>(st + D + j * 16),
+                hdr[0], hdr[1], o0, o1);
+        }
+        dst[2 * j] = o0;
+        dst[2 * j + 1] = o1;
+      }
+      if (gate) {
+        const uint4* hv = reinterpret_cast<const uint4*>(st + hid_off);
+        float acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < kEmbedH4; ++r) {
+          const int j = lane + 32 * r;
+          if (j < H8) gate_dot8(acc, hv[j], wv[r]);
+        }
+        for (int j = lane + 32 * kEmbedH4; j < H8; j += 32) gate_dot8(acc, hv[j], __ldg(wg + j));
+        const float g = gate_finish(acc);
+        if (lane == 0) a.meta[t].g = g;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ bounded-wait self-test
 // One warp waits, through the same bounded wait the library's kernels use, on
 // an mbarrier that expects one arrival nobody makes. The wait runs out after
@@ -827,9 +1052,24 @@ cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t stream) {
 
 // The embed of a batch of kSplitMinTokens or more as two launches (all table
 // formats): the IDs kernel, then the gate and gather blocks as its dependent.
+// Whether embed_bulk_kernel<FMT> (FMT 0 or 1) takes the rows and gates of a
+// batch: every bulk copy starts on a 16-byte boundary and is a multiple of 16
+// bytes, and kBkCtasPerSm CTAs with kBkStages stages fit an SM's shared memory.
+constexpr size_t kBkSmemPerCta = 112 * 1024;
+
+template <int FMT>
+bool embed_bulk_ok(const PrepareArgs& a, const TableRef& table, int32_t D, const __half* e, bool gate) {
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (e == nullptr || !al16(e) || !al16(table.codes)) return false;
+  if (FMT == 0 ? D % 16 != 0 : D % 256 != 0) return false;   // NVFP4: D / 16 block-scale bytes per row
+  if (FMT == 1 && !al16(table.blocks)) return false;
+  if (gate && (a.H % 8 != 0 || !al16(a.hidden) || !al16(a.w_gate))) return false;
+  return static_cast<size_t>(kBkStages) * bk_stage_bytes<FMT>(D, a.H, gate) <= kBkSmemPerCta;
+}
+
 template <int FMT>
 cudaError_t launch_embed_split(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
-                               cudaStream_t stream, int* kernels) {
+                               int32_t num_sms, cudaStream_t stream, int* kernels) {
   const PrepareArgs am = with_magic(a);
   const int token_blocks = (a.T + kIdsThreads - 1) / kIdsThreads;
   int sblocks = 1;
@@ -840,8 +1080,32 @@ cudaError_t launch_embed_split(const PrepareArgs& a, const TableRef& table, int3
   ids_meta_kernel<FMT><<<token_blocks + sblocks, kIdsThreads, 0, stream>>>(am, token_blocks);
   cudaError_t r = cudaGetLastError();
   if (r != cudaSuccess) return r;
+  const bool gate = a.hidden != nullptr && a.meta != nullptr;
+  if constexpr (FMT != 2) {
+  if (embed_bulk_ok<FMT>(a, table, D, e, gate)) {
+    static PerDeviceOnce configured;
+    r = configured.run([] {
+      cudaError_t x = cudaFuncSetAttribute(embed_bulk_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kBkSmemPerCta));
+      return x == cudaSuccess ? prefer_max_shared(embed_bulk_kernel<FMT>) : x;
+    });
+    if (r != cudaSuccess) return r;
+    if (kernels != nullptr) *kernels = 2;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(kBkCtasPerSm) * num_sms, a.T)));
+    cfg.blockDim = dim3(kBkThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(kBkStages) * bk_stage_bytes<FMT>(D, a.H, gate);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, embed_bulk_kernel<FMT>, am, table, D, e, gate ? 1 : 0);
+  }
+  }
   const int64_t units = static_cast<int64_t>(a.T) * (D / (16 * kSplitChunksPerThread<FMT>));
-  const int64_t n_gate = a.hidden != nullptr && a.meta != nullptr ? (a.T + kSplitGateTokens - 1) / kSplitGateTokens : 0;
+  const int64_t n_gate = gate ? (a.T + kSplitGateTokens - 1) / kSplitGateTokens : 0;
   const int64_t n_gather = e != nullptr ? (units + kSplitThreads - 1) / kSplitThreads : 0;
   if (n_gate + n_gather == 0) return cudaSuccess;
   if (kernels != nullptr) *kernels = 2;
@@ -864,8 +1128,8 @@ cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D,
   const cudaError_t cfg_err = configure_chain_kernels();
   if (cfg_err != cudaSuccess) return cfg_err;
   if (a.T >= kSplitMinTokens) {
-    if (table.nvfp4) return launch_embed_split<1>(a, table, D, e, stream, kernels);
-    return launch_embed_split<0>(a, table, D, e, stream, kernels);
+    if (table.nvfp4) return launch_embed_split<1>(a, table, D, e, num_sms, stream, kernels);
+    return launch_embed_split<0>(a, table, D, e, num_sms, stream, kernels);
   }
   const bool state = a.conv_in != nullptr || a.hist_new != nullptr;
   // small batches spread over the SMs: a few tokens per CTA, no warp taking two in turn
@@ -877,12 +1141,12 @@ cudaError_t launch_embed(const PrepareArgs& a, const TableRef& table, int32_t D,
   return cudaGetLastError();
 }
 
-cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e,
+cudaError_t launch_embed_heads(const PrepareArgs& a, const TableRef& table, int32_t D, __half* e, int32_t num_sms,
                                cudaStream_t stream, int* kernels) {
   if (kernels != nullptr) *kernels = 1;
   const cudaError_t cfg_err = configure_chain_kernels();
   if (cfg_err != cudaSuccess) return cfg_err;
-  if (a.T >= kSplitMinTokens && a.ids != nullptr) return launch_embed_split<2>(a, table, D, e, stream, kernels);
+  if (a.T >= kSplitMinTokens && a.ids != nullptr) return launch_embed_split<2>(a, table, D, e, num_sms, stream, kernels);
   const int token_blocks = (a.T + 7) / 8;
   int sblocks = 1;
   if (a.conv_in != nullptr) {
