@@ -459,7 +459,7 @@ def main():
         embed_bytes, embed_name = T * (2 * H + 8 + 16 + 4), "embed_kernel without rows (ids + gate)"
     else:                   # h, rows, scales in; e, ids, meta out; tokens
         embed_bytes, embed_name = T * (2 * H + 2 * D + 8 + 2 * D + 8 + 16 + 4), (
-            "ids_meta_kernel + embed_split_kernel (row IDs; gate; row gather/dequant)")
+            "ids_meta_kernel + embed_bulk_kernel (row IDs; bulk-copied rows dequantised; gate)")
     embed = {"kernel": embed_name, "bound": "hbm",
              "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
              "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"], "launch_ms": e_s * 1e3,
