@@ -66,7 +66,8 @@ struct ple_handle {
   float* mtp_partial = nullptr;  // its split sums
   int32_t* mtp_counts = nullptr; // its per-tile counters [2][m_tiles], zero between launches
   EncodeTiledFn encode = nullptr;
-  CUtensorMap tmap_w{};
+  CUtensorMap tmap_w{};          // fp16 W_proj, boxes of 64 K x 128 channels
+  CUtensorMap tmap_w_kb2{};      // the same as 3-D boxes of two K-blocks (the SM-pair projection)
   int32_t forward_path = 0;
   struct Prepared {        // the batch ple_prepare left in a scratch set (ids, e, meta, hist_new)
     bool valid = false;
@@ -165,6 +166,20 @@ bool encode_2d(ple_handle* h, CUtensorMap* map, CUtensorMapDataType dt, const vo
   const CUresult r = h->encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                                CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A K-major fp16 operand [outer][K] as a 3-D tensor {64 elements, outer, K / 64}
+// (a row's K-blocks 128 bytes apart), boxes of {64, box_outer, 2}: two K-blocks
+// per copy, each landing as its own 128-byte-swizzled tile.
+bool encode_kb2(ple_handle* h, CUtensorMap* map, const void* base, uint64_t K, uint64_t outer, uint32_t box_outer) {
+  const cuuint64_t dims[3] = {64, outer, K / 64};
+  const cuuint64_t strides[2] = {K * 2, 128};
+  const cuuint32_t box[3] = {64, box_outer, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = h->encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -272,8 +287,10 @@ ple_status run_projection(ple_handle* h, const ple_handle::Scratch& sc, int32_t 
   if (gather && !(pl.fused && pl.ctas == 2)) return PLE_ERR_UNSUPPORTED;
   ple_status st = PLE_OK;
   CUtensorMap tmap_e{}, tmap_h{}, tmap_o{}, tmap_o_head{};
-  if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, sc.e, c.row_dim, T, static_cast<uint64_t>(c.row_dim) * 2,
-                 kTileK, pl.n_tok / pl.ctas, CU_TENSOR_MAP_SWIZZLE_128B))
+  const bool kb2 = pl.ctas == 2 && !gather;     // the SM-pair projection takes two K-blocks per copy
+  if (kb2 ? !encode_kb2(h, &tmap_e, sc.e, c.row_dim, T, pl.n_tok / pl.ctas)
+          : !encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, sc.e, c.row_dim, T,
+                       static_cast<uint64_t>(c.row_dim) * 2, kTileK, pl.n_tok / pl.ctas, CU_TENSOR_MAP_SWIZZLE_128B))
     return PLE_ERR_CUDA;
   if (!encode_2d(h, &tmap_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, c.hidden, T,
                  static_cast<uint64_t>(c.hidden) * 2, kTileM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -319,7 +336,8 @@ ple_status run_projection(ple_handle* h, const ple_handle::Scratch& sc, int32_t 
   const int total = gp.m_tiles * gp.n_tiles * gp.k_splits;
   const int grid = pl.ctas == 2 ? 2 * std::min(total, h->num_sms / 2) : std::min(total, h->num_sms);
   st = run_stage(h, PLE_STAGE_GEMM, stream, [&] {
-    return ple::launch_gemm(h->tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, gp, grid, pl.ctas, gather, stream);
+    return ple::launch_gemm(kb2 ? h->tmap_w_kb2 : h->tmap_w, tmap_e, tmap_h, tmap_o, tmap_o_head, gp, grid, pl.ctas,
+                            gather, stream);
   });
   if (st != PLE_OK || pl.fused) return st;
 
@@ -633,6 +651,7 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   if (cudaMemsetAsync(h->status, 0, 4, stream) != cudaSuccess ||
       !encode_2d(h, &h->tmap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->w16, c.row_dim, c.hidden,
                  static_cast<uint64_t>(c.row_dim) * 2, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_kb2(h, &h->tmap_w_kb2, h->w16, c.row_dim, c.hidden, kTileM) ||
       cudaStreamSynchronize(stream) != cudaSuccess) {
     free_all(h);
     delete h;

@@ -96,11 +96,16 @@ constexpr uint32_t H_CHUNK = EPI_CHUNK * BM * 2;   // 8 KB (bf16 h, 32 tokens x 
 
 template <int CTAS, bool GATHER = false>
 struct Cfg {
-  static constexpr int STAGES = GATHER ? 4 : (CTAS == 2 ? 5 : 4);
-  static constexpr int HBUFS = GATHER ? 4 : (CTAS == 2 ? 7 : 3);   // ring of h / output chunks
+  // K-blocks per stage: the SM-pair form fetches two K-blocks of each operand
+  // per TMA copy (a 3-D box of 32 KB), which the copy engine delivers at about
+  // 72 B/clk per SM against about 41 B/clk for two 16 KB boxes (measured)
+  static constexpr int KBS = (!GATHER && CTAS == 2) ? 2 : 1;
+  static constexpr int STAGES = GATHER ? 4 : (CTAS == 2 ? 3 : 4);
+  static constexpr int HBUFS = GATHER ? 4 : 3;                   // ring of h / output chunks
   static constexpr int LSTAGES = GATHER ? 3 : 0;                  // landing slots of FP8 row segments
   static constexpr uint32_t B_ROWS = BN_MAX / CTAS;              // token rows of e held by one CTA
-  static constexpr uint32_t B_STAGE = B_ROWS * BK * 2;           // 32 KB or 16 KB
+  static constexpr uint32_t A_BYTES = KBS * A_STAGE;             // W_proj bytes of a stage
+  static constexpr uint32_t B_STAGE = KBS * B_ROWS * BK * 2;     // e bytes of a stage
   // landing slot: BK codes of each token's order-0 row, then of its order-1
   // row (64 bytes per token and order); the rows' scales of a tile go into one
   // of two buffers (by tile parity), 8 bytes per token
@@ -108,7 +113,7 @@ struct Cfg {
   static constexpr uint32_t L_SLOT = 2 * L_CODES;
   static constexpr uint32_t S_BUF = B_ROWS * 8;
   static constexpr uint32_t OFF_A = 0;
-  static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
+  static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr uint32_t OFF_L = OFF_B + STAGES * B_STAGE;
   static constexpr uint32_t OFF_S = OFF_L + LSTAGES * L_SLOT;
   static constexpr uint32_t OFF_H = OFF_S + (GATHER ? 2 * S_BUF : 0);
@@ -588,7 +593,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
       for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
       // bytes the even CTA's full barrier receives per stage (both CTAs' loads)
       const uint32_t tx_bytes =
-          GATHER ? CTAS * A_STAGE : CTAS * (A_STAGE + static_cast<uint32_t>(p.n_tok / CTAS) * BK * 2);
+          GATHER ? CTAS * A_STAGE : CTAS * C::KBS * (A_STAGE + static_cast<uint32_t>(p.n_tok / CTAS) * BK * 2);
       bool ok = true;
       bool e_ready = false;
       for (int tile = unit; tile < total_tiles && ok; tile += units) {
@@ -598,11 +603,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
         const int chA = m * BM * CTAS + static_cast<int>(rank) * BM;
         const int tokB = tok0 + static_cast<int>(rank) * (p.n_tok / CTAS);
         const int kb0 = ks * p.num_kb / p.k_splits, kb1 = (ks + 1) * p.num_kb / p.k_splits;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += C::KBS) {
           if (!wait_or_abort(smem_u32(&bars->empty[stage]), phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           const uint32_t fb = smem_u32(&bars->full[stage]);
           if (leader) mbar_arrive_expect_tx(fb, tx_bytes);
-          if constexpr (CTAS == 2) {
+          if constexpr (C::KBS == 2) {
+            // 3-D boxes {64, rows, 2 K-blocks}: a second K-block past the tensor is
+            // zero-filled, one past this tile's K range is loaded and not used
+            const uint32_t fb0 = mapa_shared(fb, 0);
+            tma_load_3d_pair(sA + stage * C::A_BYTES, &tmap_w, 0, chA, kb, fb0);
+            if (!e_ready) { pdl_wait(); e_ready = true; }     // e comes from the previous kernel
+            tma_load_3d_pair(sB + stage * C::B_STAGE, &tmap_e, 0, tokB, kb, fb0);
+          } else if constexpr (CTAS == 2) {
             const uint32_t fb0 = mapa_shared(fb, 0);
             tma_load_2d_pair(sA + stage * A_STAGE, &tmap_w, kb * BK, chA, fb0);
             if constexpr (!GATHER) {
@@ -648,19 +660,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
         if (!wait_or_abort(smem_u32(&bars->tempty[acc]), acc_parity ^ 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tmem_d = tmem_base + static_cast<uint32_t>(acc * BN_MAX);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += C::KBS) {
           // gather-fused: the peer's converter warps arrive with cluster-scope release
           if (!wait_or_abort<GATHER>(smem_u32(&bars->full[stage]), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = sdesc_k_sw128(sA + stage * A_STAGE);
-          const uint64_t bdesc = sdesc_k_sw128(sB + stage * C::B_STAGE);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            // advance 16 fp16 = 32 bytes along K inside the swizzled row: +2 in the >>4 address field
-            if constexpr (CTAS == 2)
-              mma_f16_pair(tmem_d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-            else
-              mma_f16(tmem_d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          for (int hk = 0; hk < C::KBS; ++hk) {
+            if (kb + hk >= kb1) break;                          // the box's second K-block is past this tile's range
+            const uint64_t adesc = sdesc_k_sw128(sA + stage * C::A_BYTES + hk * A_STAGE);
+            // a box lands densely: its second K-block follows the first's n_tok / CTAS rows
+            const uint64_t bdesc = sdesc_k_sw128(sB + stage * C::B_STAGE + hk * static_cast<uint32_t>(p.n_tok / CTAS) * BK * 2);
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              // advance 16 fp16 = 32 bytes along K inside the swizzled row: +2 in the >>4 address field
+              const uint32_t accum = (kb + hk > kb0 || k > 0) ? 1u : 0u;
+              if constexpr (CTAS == 2)
+                mma_f16_pair(tmem_d, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+              else
+                mma_f16(tmem_d, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+            }
           }
           const uint32_t eb = smem_u32(&bars->empty[stage]);
           if constexpr (CTAS == 2) {

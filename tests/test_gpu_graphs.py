@@ -3,11 +3,11 @@ graphs) replays to the same bits as eager launches.
 
 Every call is stream-ordered and does its host work (argument checks, tensor
 maps, launch planning) at capture time; the kernels keep no state between
-launches that a replay could see stale. Four forms are captured: a decode step
+launches that a replay could see stale. The forms captured: a decode step
 (the tokens kernel, then the channel-split projection under programmatic
-dependent launch), an MTP-style decode step on the split-K path, a prefill on
-SM-pair tiles and a small forward on the split-K path (projection then
-combine).
+dependent launch), an MTP-style decode step on the split-K path, prefills on
+SM-pair and single-SM tiles (of 4,096 tokens too, whose embed is two launches)
+and a small forward on the split-K path (projection then combine).
 """
 import numpy as np
 import pytest
@@ -73,8 +73,10 @@ def test_decode_step_graph_replay_matches_eager(mid_layer):  # noqa: F811
     del graph
 
 
-@pytest.mark.parametrize("lengths,path", [([1500, 700, 1], 1), ([40, 3, 5], 2)])
+@pytest.mark.parametrize("lengths,path", [([1500, 700, 1], 1), ([40, 3, 5], 2), ([4000, 90, 6], 1), ([4000, 0, 96], 3)])
 def test_forward_graph_replay_matches_eager(mid_layer, lengths, path):  # noqa: F811
+    """4,096-token batches take the two-launch embed (row IDs, then the bulk-copy
+    pipeline as its programmatic dependent) ahead of the projection."""
     from ple_inputs.device import bf16_tensor
     L = mid_layer
     rng = np.random.default_rng(sum(lengths))
