@@ -446,9 +446,7 @@ ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int3
   if (!small && h->forward_path != 2 && h->mtp && T <= ple::kMtpMaxTokens && q <= ple::kMtpMaxQ) {
     const int n_pad = (T + 15) / 16 * 16;
     CUtensorMap tmap_e{};
-    if (!encode_2d(h, &tmap_e, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h->e, c.row_dim, T,
-                   static_cast<uint64_t>(c.row_dim) * 2, kTileK, n_pad, CU_TENSOR_MAP_SWIZZLE_128B))
-      return PLE_ERR_CUDA;
+    if (!encode_kb2(h, &tmap_e, h->e, c.row_dim, T, n_pad)) return PLE_ERR_CUDA;   // two K-blocks per copy
     ple::MtpProjArgs a{};
     a.tokens = tokens;
     a.B = B;
@@ -470,7 +468,7 @@ ple_status run_decode_rest(ple_handle* h, const int32_t* tokens, int32_t B, int3
     a.tile_count = h->mtp_counts;
     a.tile_done = h->mtp_counts + h->mtp_plan.m_tiles;
     a.status = h->status;
-    return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_mtp_proj(h->tmap_w, tmap_e, a, stream); });
+    return run_stage(h, PLE_STAGE_GEMM, stream, [&] { return ple::launch_mtp_proj(h->tmap_w_kb2, tmap_e, a, stream); });
   }
   if (!small)
     return run_projection(h, h->scratch[0], T, B, q, hidden, out, dtype, nullptr, hist, conv_state, tokens, n_commit,

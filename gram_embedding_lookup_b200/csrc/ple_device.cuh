@@ -269,6 +269,16 @@ __device__ __forceinline__ void cluster_sync() {
 // Tiled load into this CTA's shared memory whose completion is counted on an
 // mbarrier that may live in the peer CTA of the pair (shared::cluster address).
 // One destination CTA.
+// A 3-D box {x, y, z} into this CTA's shared memory, completion on its barrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
 // The same for a 3-D box {x, y, z}: the projection's K-major operands as
 // {64 elements, rows, K-blocks}, two K-blocks per copy.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,

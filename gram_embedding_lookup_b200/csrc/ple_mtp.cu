@@ -9,7 +9,9 @@
 // 1 MB of rows. Per SM the bound is operand traffic, so the grid is 20
 // channel tiles (M = 128, operand A = fp16 W_proj, K-major) x 7 K-splits
 // (operand B = the step's fp16 rows e, N = the step's tokens): 140 CTAs, one
-// per SM, each with 94 KB of W_proj and 140 KB of e. The first stages' W_proj
+// per SM, each with 94 KB of W_proj and 140 KB of e. Each operand arrives two
+// K-blocks per TMA copy (3-D boxes of 32 KB and more, which the copy engine
+// delivers faster per SM than single K-blocks). The first stages' W_proj
 // copies are issued before the programmatic wait, under the embed kernel.
 //
 // The K-split CTAs of a channel tile write their fp32 sums to a scratch slab
@@ -50,7 +52,8 @@ constexpr int kMtMmaWarp = 1;
 constexpr int kMtEpiWarp0 = 2;
 constexpr int kMtEpiThreads = 256;
 constexpr int kMtStages = 5;              // most stages; fewer when 256 tokens do not leave room
-constexpr uint32_t kMtAStage = kMtM * kMtBK * 2;   // 16 KB
+constexpr uint32_t kMtAStage = kMtM * kMtBK * 2;   // 16 KB: W_proj of one K-block
+constexpr int kMtKbs = 2;                 // K-blocks per stage: each operand arrives as one 3-D TMA box of two
 constexpr uint32_t kMtTmemCols = 256;
 constexpr int kMtSmemLimit = 226 * 1024;  // dynamic; the per-block maximum (227 KB) includes the static word
 
@@ -63,10 +66,16 @@ struct MtBars {
   int32_t abort_flag;
 };
 
-// Dynamic shared memory from a 1024-byte aligned base: A stages, B stages
-// (n_pad rows of 128 bytes each), then the barriers.
+// Bytes of one stage: two K-blocks of W_proj (A) and of the step's rows (B,
+// n_pad rows of 128 bytes per K-block).
+size_t mtp_stage_bytes(int n_pad) {
+  return static_cast<size_t>(kMtKbs) * (kMtAStage + static_cast<size_t>(n_pad) * kMtBK * 2);
+}
+
+// Dynamic shared memory from a 1024-byte aligned base: A stages, B stages, then
+// the barriers.
 size_t mtp_smem_bytes(int n_pad, int stages) {
-  return 1024 + static_cast<size_t>(stages) * (kMtAStage + static_cast<size_t>(n_pad) * kMtBK * 2) + sizeof(MtBars);
+  return 1024 + static_cast<size_t>(stages) * mtp_stage_bytes(n_pad) + sizeof(MtBars);
 }
 
 int mtp_stages(int n_pad) {
@@ -104,15 +113,17 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   // generic ones)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int S = a.stages;
-  const uint32_t b_stage = static_cast<uint32_t>(a.n_pad) * kMtBK * 2;
+  const uint32_t b_kb = static_cast<uint32_t>(a.n_pad) * kMtBK * 2;   // B bytes of one K-block
+  const uint32_t a_stage = kMtKbs * kMtAStage, b_stage = kMtKbs * b_kb;
   const uint32_t sA = smem_u32(smem);
-  const uint32_t sB = sA + S * kMtAStage;
-  MtBars* bars = reinterpret_cast<MtBars*>(smem + S * (kMtAStage + b_stage));
+  const uint32_t sB = sA + S * a_stage;
+  MtBars* bars = reinterpret_cast<MtBars*>(smem + S * (a_stage + b_stage));
   volatile int32_t* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.x % a.m_tiles, ks = blockIdx.x / a.m_tiles;
   const int kb0 = ks * a.num_kb / a.k_splits, kb1 = (ks + 1) * a.num_kb / a.k_splits;
   const int nkb = kb1 - kb0;
+  const int nst = (nkb + kMtKbs - 1) / kMtKbs;             // stage loads (the last may hold one K-block)
   const int T = a.B * a.q;
 
   if (threadIdx.x == 0) {
@@ -139,27 +150,29 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_e);
-      const uint32_t tx = kMtAStage + b_stage;
-      const int pre = min(nkb, S);
+      // 3-D boxes {64, rows, 2 K-blocks}: a second K-block past the tensor is
+      // zero-filled, one past this split's K range is loaded and not used
+      const uint32_t tx = a_stage + b_stage;
+      const int pre = min(nst, S);
       // W_proj of the first stages does not depend on the previous kernel
       for (int i = 0; i < pre; ++i) {
         const uint32_t fb = smem_u32(&bars->full[i]);
         mbar_arrive_expect_tx(fb, tx);
-        tma_load_2d(sA + i * kMtAStage, &tmap_w, (kb0 + i) * kMtBK, m * kMtM, fb);
+        tma_load_3d(sA + i * a_stage, &tmap_w, 0, m * kMtM, kb0 + kMtKbs * i, fb);
       }
       pdl_launch_dependents();
       pdl_wait();                                             // e comes from the embed kernel
       for (int i = 0; i < pre; ++i)
-        tma_load_2d(sB + i * b_stage, &tmap_e, (kb0 + i) * kMtBK, 0, smem_u32(&bars->full[i]));
+        tma_load_3d(sB + i * b_stage, &tmap_e, 0, 0, kb0 + kMtKbs * i, smem_u32(&bars->full[i]));
       int issued = pre;
-      for (int i = pre; i < nkb; ++i) {
+      for (int i = pre; i < nst; ++i) {
         const int stage = i % S;
         const uint32_t round = static_cast<uint32_t>(i / S);
         if (!wait_bar(smem_u32(&bars->empty[stage]), (round - 1) & 1, abort_flag, a.status)) break;
         const uint32_t fb = smem_u32(&bars->full[stage]);
         mbar_arrive_expect_tx(fb, tx);
-        tma_load_2d(sA + stage * kMtAStage, &tmap_w, (kb0 + i) * kMtBK, m * kMtM, fb);
-        tma_load_2d(sB + stage * b_stage, &tmap_e, (kb0 + i) * kMtBK, 0, fb);
+        tma_load_3d(sA + stage * a_stage, &tmap_w, 0, m * kMtM, kb0 + kMtKbs * i, fb);
+        tma_load_3d(sB + stage * b_stage, &tmap_e, 0, 0, kb0 + kMtKbs * i, fb);
         issued = i + 1;
       }
       // copies in flight land before the CTA's shared memory is released
@@ -178,18 +191,22 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kMtM, a.n_pad);
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
+      for (int i = 0; i < nst; ++i) {
         const int stage = i % S;
         if (!wait_bar(smem_u32(&bars->full[stage]), static_cast<uint32_t>(i / S) & 1, abort_flag, a.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t adesc = sdesc_k_sw128(sA + stage * kMtAStage);
-        const uint64_t bdesc = sdesc_k_sw128(sB + stage * b_stage);
 #pragma unroll
-        for (int k = 0; k < kMtBK / kMtUmmaK; ++k)
-          mma_f16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
+        for (int hk = 0; hk < kMtKbs; ++hk) {
+          if (kMtKbs * i + hk >= nkb) break;                  // the box's second K-block is past this split
+          const uint64_t adesc = sdesc_k_sw128(sA + stage * a_stage + hk * kMtAStage);
+          const uint64_t bdesc = sdesc_k_sw128(sB + stage * b_stage + hk * b_kb);
+#pragma unroll
+          for (int k = 0; k < kMtBK / kMtUmmaK; ++k)
+            mma_f16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (i > 0 || hk > 0 || k > 0) ? 1u : 0u);
+        }
         mma_commit(smem_u32(&bars->empty[stage]));
       }
       if (ok) mma_commit(smem_u32(&bars->tfull));
@@ -248,7 +265,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     // sums: they are loaded now, under the meet, when they clear this split's
     // sums on their way out.
     const int b0 = ks * a.B / a.k_splits, b1 = (ks + 1) * a.B / a.k_splits;
-    const uint32_t region = static_cast<uint32_t>(S) * (kMtAStage + b_stage);
+    const uint32_t region = static_cast<uint32_t>(S) * (a_stage + b_stage);
     const uint32_t per_seq = static_cast<uint32_t>(a.q) * (a.k_splits * 512u + 256u + 16u) + 3u * 512u + 32u;
     const int max_seqs = max(1, static_cast<int>(region / per_seq));
     auto side_bytes = [&](int ns) -> uint32_t {
@@ -469,8 +486,7 @@ cudaError_t launch_mtp_proj(const CUtensorMap& tmap_w, const CUtensorMap& tmap_e
   MtpProjArgs b = a;
   b.stages = mtp_stages(a.n_pad);
   // the split's sums [T][128] f32 pass through the operand stages on their way out
-  if (static_cast<size_t>(a.B) * a.q * 512u >
-      static_cast<size_t>(b.stages) * (kMtAStage + static_cast<size_t>(a.n_pad) * kMtBK * 2))
+  if (static_cast<size_t>(a.B) * a.q * 512u > static_cast<size_t>(b.stages) * mtp_stage_bytes(a.n_pad))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(a.m_tiles * a.k_splits);
