@@ -1186,6 +1186,13 @@ def mtp_bench(ctx, layer, stream):
     hist.copy_(hist0)
     conv.copy_(conv0)
     ms = timed(ctx, stream, step, n)
+    # the first 20 steps captured in one CUDA graph, replayed (no host in the loop;
+    # consecutive steps overlap under programmatic dependent launch)
+    hist.copy_(hist0)
+    conv.copy_(conv0)
+    ms_graph = graph_time(ctx, stream, [lambda st, i=i: ple.ple_decode_step(
+        h, steps[i][0], B, q, steps[i][1], out, ple.PLE_OUT_BF16, hist, conv, steps[i][2], st) for i in range(20)], reps=1)
+    ms_graph /= 20
     # the same 100 steps again from the same state, each after an L2 flush
     hist.copy_(hist0)
     conv.copy_(conv0)
@@ -1202,11 +1209,13 @@ def mtp_bench(ctx, layer, stream):
     return {"workload": "MTP decode: 64 sequences x 3 tokens/step, 100 steps, 30% shared prefix",
             "value": B * q * world * n / (ms / 1e3), "unit": "tokens/s (processed)",
             "committed_tokens_per_s": committed * world / (ms / 1e3), "us_per_step": 1e3 * ms / n,
+            "graph20_us_per_step": 1e3 * ms_graph,
             "cold_us_per_step": 1e3 * ms_cold, "cold_eager_us_per_step": 1e3 * ms_cold_eager,
             "device_status": int(status),
-            "note": "cold: 256 MB written before every step, the step's time the difference between graphs of 20 x "
-                    "(write, step) and 20 x (write); cold_eager: the 100 steps each after the write, one eager call "
-                    "between two events"}
+            "note": "us_per_step: 100 eager steps back to back; graph20: 20 consecutive steps in one CUDA graph, "
+                    "replayed; cold: 256 MB written before every step, the step's time the difference between "
+                    "graphs of 20 x (write, step) and 20 x (write); cold_eager: the 100 steps each after the write, "
+                    "one eager call between two events"}
 
 
 def long_bench(ctx, layer, stream):
