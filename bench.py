@@ -501,7 +501,10 @@ def main():
         if "long" in want:
             line["long_context"] = long_bench(ctx, layer, stream)
         if "nvfp4" in want:
-            line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks)
+            # the two layouts of the same NVFP4 contents, the array layout first
+            arrays = nvfp4_bench(ctx, w, sets, stream, peaks, ple.PLE_TABLE_NVFP4)
+            line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks, ple.PLE_TABLE_NVFP4_ROWS)
+            line["nvfp4"]["arrays_layout"] = arrays
         if "heads" in want:
             line["heads"] = heads_bench(ctx, sets, stream, peaks)
         if "prepared" in want:
@@ -881,8 +884,13 @@ def heads_bench(ctx, sets, stream, peaks, steps=300):
 
     for i in range(5):
         step(i)
-    ms = timed(ctx, stream, step, steps)
-    ple.ple_set_profiling(h, True)
+    # each measurement starts from an idle GPU, as the headline's steps do: a
+    # second's pause lets the clock come back from the power cap that the
+    # previous lines' steps drove it into
+    idle_pause(ctx)
+    ms = timed(ctx, stream, step, steps)            # no events between the kernels
+    idle_pause(ctx)
+    ple.ple_set_profiling(h, True)                  # then per-kernel durations
     ple.ple_get_stage_times(h)
     for i in range(min(steps, 100)):
         step(i)
@@ -906,13 +914,17 @@ def heads_bench(ctx, sets, stream, peaks, steps=300):
                                "unit": "GB/s", "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"],
                                "algorithmic_bytes_per_launch": embed_bytes},
             "gathered_row_gbs": T * row_bytes / e_s / 1e9,
+            "measured": "value over 300 steps, then stage_ms_per_launch over 100 steps (CUDA events around "
+                        "each kernel), each from an idle GPU after a 1 s pause",
             "decode_us_per_step": d_ms / n_dec * 1e3, "device_status": int(status)}
 
 
-def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
-    """The NVFP4 table variant (PLE_TABLE_NVFP4): the same prefill batches and the
-    decode workload on a table of packed E2M1 codes with E4M3 block scales per 16
-    elements (28.8 GB at full scale instead of 51.2 GB)."""
+def nvfp4_bench(ctx, w, sets, stream, peaks, fmt, steps=300):
+    """The NVFP4 table variant: the same prefill batches and the decode workload on
+    a table of packed E2M1 codes with E4M3 block scales per 16 elements (28.8 GB at
+    full scale instead of 51.2 GB), in layout `fmt`: PLE_TABLE_NVFP4 (codes and
+    block scales in two arrays) or PLE_TABLE_NVFP4_ROWS (each row's block scales
+    after its codes)."""
     torch, ple, pi = ctx["torch"], ctx["ple"], ctx["pi"]
     from ple_inputs.device import DeviceLayer
     R, D, H = w.rows_per_order, w.row_dim, w.hidden
@@ -920,8 +932,9 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
     free, _ = torch.cuda.mem_get_info()
     if free < need + (4 << 30):
         return {"skipped": f"needs {need / 1e9:.1f} GB free for the NVFP4 table, {free / 1e9:.1f} GB free"}
-    layer = DeviceLayer(w, max_tokens=16384, max_seqs=64, table_format=ple.PLE_TABLE_NVFP4)
+    layer = DeviceLayer(w, max_tokens=16384, max_seqs=64, table_format=fmt)
     h = layer.handle
+    rows = fmt == ple.PLE_TABLE_NVFP4_ROWS
 
     # the decode step first, before the prefill loop heats the GPU into its power cap
     # (the headline decode line also runs on a GPU that has been mostly idle)
@@ -949,7 +962,12 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
 
     for i in range(5):
         step(i)
+    # each measurement starts from an idle GPU, as the headline's steps do: a
+    # second's pause lets the clock come back from the power cap that the
+    # previous lines' steps drove it into
+    idle_pause(ctx)
     ms = timed(ctx, stream, step, steps)            # no events between the kernels
+    idle_pause(ctx)
     ple.ple_set_profiling(h, True)                  # then per-kernel durations
     ple.ple_get_stage_times(h)
     for i in range(min(steps, 100)):
@@ -967,14 +985,26 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, steps=300):
     status = ple.ple_get_error(h)
     layer.close()
     world = ctx["world"]
+    layout = ("rows: each row's 1,280 code bytes, then its 160 block-scale bytes" if rows
+              else "arrays: codes [2][R][1280], block scales [2][R][160]")
     return {"workload": "full-scale prefill (the headline batches) and 8 x 1 decode on the NVFP4 table",
-            "table_bytes": int(need), "value": T * world * steps / (ms / 1e3), "unit": "tokens/s",
+            "layout": layout, "table_bytes": int(need), "value": T * world * steps / (ms / 1e3), "unit": "tokens/s",
             "ms_per_step": ms / steps, "stage_ms_per_launch": {"embed": e_s * 1e3, "gemm": g_ms / max(g_n, 1)},
             "embed_roofline": {"bound": "hbm", "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"],
                                "unit": "GB/s", "frac": embed_bytes / e_s / 1e9 / peaks["hbm_gbs"],
                                "algorithmic_bytes_per_launch": embed_bytes},
             "gathered_row_gbs": T * row_bytes / e_s / 1e9,
+            "measured": "value over 300 steps, then stage_ms_per_launch over 100 steps (CUDA events around "
+                        "each kernel), each from an idle GPU after a 1 s pause",
             "decode_us_per_step": 1e3 * d_ms / n_dec, "device_status": int(status)}
+
+
+def idle_pause(ctx, seconds=1.0):
+    """All ranks idle for `seconds` with no work queued (the GPU's clock recovers
+    from the power cap between two measurements)."""
+    ctx["torch"].cuda.synchronize()
+    time.sleep(seconds)
+    ctx["barrier"]()
 
 
 def timed_each(ctx, stream, fn, n, flush=None):

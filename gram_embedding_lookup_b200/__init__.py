@@ -19,7 +19,7 @@ __all__ = [
     "ple_get_error",
     "ple_status_string", "ple_set_profiling", "ple_get_stage_times", "ple_set_forward_path",
     "ple_launch_count", "ple_wait_selftest", "ple_embed_static", "PLE_STATIC_MAX_TOKENS", "PLE_OUT_BF16", "PLE_OUT_F32",
-    "PLE_TABLE_E4M3", "PLE_TABLE_NVFP4", "PLE_TABLE_E4M3_HEADS", "STATUS",
+    "PLE_TABLE_E4M3", "PLE_TABLE_NVFP4", "PLE_TABLE_E4M3_HEADS", "PLE_TABLE_NVFP4_ROWS", "STATUS",
     "STAGES", "LIB_PATH",
 ]
 
@@ -30,6 +30,7 @@ PLE_OUT_F32 = 1
 PLE_TABLE_E4M3 = 0
 PLE_TABLE_NVFP4 = 1
 PLE_TABLE_E4M3_HEADS = 2   # 16 hash-head sub-tables of row_dim / 16 codes; row IDs [T][16]
+PLE_TABLE_NVFP4_ROWS = 3   # the NVFP4 table with each row's block scales after its codes
 PLE_STATIC_MAX_TOKENS = 16384   # the fixed row-ID array of ple_embed_static
 STATUS = {0: "PLE_OK", 1: "PLE_ERR_INVALID_ARG", 2: "PLE_ERR_SHAPE", 3: "PLE_ERR_ALIGN", 4: "PLE_ERR_RANGE",
           5: "PLE_ERR_OOM", 6: "PLE_ERR_CUDA", 7: "PLE_ERR_TIMEOUT", 8: "PLE_ERR_UNSUPPORTED"}

@@ -196,9 +196,28 @@ int ids_per_token(const ple_config& c) { return c.table_format == PLE_TABLE_E4M3
 // state and e) for the handle's table layout.
 cudaError_t launch_embed_for(ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream);
 
+// The format the kernels see: both NVFP4 layouts are PLE_TABLE_NVFP4 there,
+// told apart by the row strides of TableRef.
+int32_t kernel_format(const ple_config& c) {
+  return c.table_format == PLE_TABLE_NVFP4_ROWS ? static_cast<int32_t>(PLE_TABLE_NVFP4) : c.table_format;
+}
+
 ple::TableRef table_ref(const ple_handle* h) {
-  const bool nv = h->cfg.table_format == PLE_TABLE_NVFP4;
-  return ple::TableRef{h->w.table, nv ? h->w.block_scales : nullptr, h->w.scales, nv ? 1 : 0};
+  const ple_config& c = h->cfg;
+  const int32_t D = c.row_dim;
+  ple::TableRef t{h->w.table, nullptr, h->w.scales, 0, D, 0, 0};
+  if (c.table_format == PLE_TABLE_NVFP4) {
+    t.blocks = h->w.block_scales;
+    t.nvfp4 = 1;
+    t.cs = D / 2;
+    t.bs = D / 16;
+  } else if (c.table_format == PLE_TABLE_NVFP4_ROWS) {
+    t.blocks = h->w.table + D / 2;                      // each row's block scales follow its codes
+    t.nvfp4 = 1;
+    t.cs = t.bs = D / 2 + D / 16;
+    t.nv_rows = 1;
+  }
+  return t;
 }
 
 cudaError_t launch_embed_for(ple_handle* h, const ple::PrepareArgs& pa, __half* e, cudaStream_t stream) {
@@ -398,17 +417,20 @@ ple_status run_decode_embed(ple_handle* h, const int32_t* tokens, int32_t B, int
   a.rows1 = c.rows[1];
   a.magic0 = ple::barrett_magic(c.rows[0]);
   a.magic1 = ple::barrett_magic(c.rows[1]);
-  a.table = h->w.table;
-  a.blocks = c.table_format == PLE_TABLE_NVFP4 ? h->w.block_scales : nullptr;
+  const ple::TableRef tab = table_ref(h);
+  a.table = tab.codes;
+  a.blocks = tab.blocks;
+  a.cs = tab.cs;
+  a.bs = tab.bs;
   a.scales = h->w.scales;
-  a.format = c.table_format;
+  a.format = kernel_format(c);
   a.D = c.row_dim;
   a.H = c.hidden;
   a.hidden = static_cast<const __nv_bfloat16*>(hidden);
   a.w_gate = static_cast<const __nv_bfloat16*>(h->w.w_gate);
   a.e = h->e;
   a.row_scales = h->scratch[0].row_scales;
-  a.codes2 = small && ple::decode_two_order(B * q, c.table_format) ? 1 : 0;
+  a.codes2 = small && ple::decode_two_order(B * q, kernel_format(c)) ? 1 : 0;
   a.meta = h->meta;
   a.w16 = h->w16;
   a.w16_bytes = static_cast<int64_t>(c.hidden) * c.row_dim * 2;
@@ -506,10 +528,13 @@ ple::DecodeProjArgs decode_proj_args(const ple_handle* h, const int32_t* tokens,
   a.rows1 = c.rows[1];
   a.magic0 = ple::barrett_magic(c.rows[0]);
   a.magic1 = ple::barrett_magic(c.rows[1]);
-  a.table = h->w.table;
-  a.blocks = c.table_format == PLE_TABLE_NVFP4 ? h->w.block_scales : nullptr;
+  const ple::TableRef tab = table_ref(h);
+  a.table = tab.codes;
+  a.blocks = tab.blocks;
+  a.cs = tab.cs;
+  a.bs = tab.bs;
   a.scales = h->w.scales;
-  a.format = c.table_format;
+  a.format = kernel_format(c);
   a.step_count = h->status + 1;
   a.status = h->status;
   return a;
@@ -553,7 +578,7 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
   *out = nullptr;
   const ple_config& c = *config;
   if ((c.table_format != PLE_TABLE_E4M3 && c.table_format != PLE_TABLE_NVFP4 &&
-       c.table_format != PLE_TABLE_E4M3_HEADS) ||
+       c.table_format != PLE_TABLE_E4M3_HEADS && c.table_format != PLE_TABLE_NVFP4_ROWS) ||
       c.vocab <= 0 || c.hidden <= 0 || c.row_dim <= 0 || c.max_tokens <= 0 || c.max_seqs <= 0)
     return PLE_ERR_INVALID_ARG;
   if (c.prepare_slots < 0 || c.prepare_slots > 2) return PLE_ERR_INVALID_ARG;
@@ -563,12 +588,15 @@ ple_status ple_create(const ple_config* config, const ple_weights* weights, cuda
     if (c.row_dim % 256 != 0) return PLE_ERR_UNSUPPORTED;
     if (c.rows[1] != c.rows[0]) return PLE_ERR_INVALID_ARG;
   }
+  // rows of row_dim * 9/16 bytes: every row starts on a 16-byte boundary
+  if (c.table_format == PLE_TABLE_NVFP4_ROWS && c.row_dim % 256 != 0) return PLE_ERR_UNSUPPORTED;
   for (int n = 0; n < 2; ++n)
     if (c.rows[n] <= 0 || c.rows[n] >= (int64_t(1) << 31)) return PLE_ERR_INVALID_ARG;
   if (weights->table == nullptr || weights->scales == nullptr || weights->w_proj == nullptr ||
       weights->w_gate == nullptr || weights->conv_w == nullptr)
     return PLE_ERR_INVALID_ARG;
   if (c.table_format == PLE_TABLE_NVFP4 && weights->block_scales == nullptr) return PLE_ERR_INVALID_ARG;
+  if (c.table_format == PLE_TABLE_NVFP4_ROWS && weights->block_scales != nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned(weights->table, 16) || !aligned(weights->w_proj, 16) || !aligned(weights->w_gate, 16) ||
       !aligned(weights->conv_w, 16) || !aligned(weights->scales, 4) ||
       (c.table_format == PLE_TABLE_NVFP4 && !aligned(weights->block_scales, 16)))

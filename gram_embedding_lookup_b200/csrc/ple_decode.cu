@@ -176,8 +176,8 @@ __global__ void __launch_bounds__(kEmbedThreads) decode_embed_kernel(const Decod
       // the two rows as exact fp16 codes (rows t and t + 8 of e), the scales apart
       uint4* crow1 = reinterpret_cast<uint4*>(a.e + static_cast<int64_t>(t + kTwoOrderMaxTok) * a.D);
       for (int j = threadIdx.x; j < nch; j += blockDim.x) {
-        const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.D, j);
-        const RowChunk<NV> y = load_chunk<NV>(a.table, a.blocks, r1, a.D, j);
+        const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.cs, a.bs, j);
+        const RowChunk<NV> y = load_chunk<NV>(a.table, a.blocks, r1, a.cs, a.bs, j);
         uint4 o0, o1;
         codes_to_f16<NV>(x, o0, o1);
         erow[2 * j] = o0;
@@ -189,8 +189,8 @@ __global__ void __launch_bounds__(kEmbedThreads) decode_embed_kernel(const Decod
       if (threadIdx.x == 0) reinterpret_cast<float2*>(a.row_scales)[t] = make_float2(s0, s1);
     } else {
       for (int j = threadIdx.x; j < nch; j += blockDim.x) {
-        const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.D, j);
-        const RowChunk<NV> y = load_chunk<NV>(a.table, a.blocks, r1, a.D, j);
+        const RowChunk<NV> x = load_chunk<NV>(a.table, a.blocks, r0, a.cs, a.bs, j);
+        const RowChunk<NV> y = load_chunk<NV>(a.table, a.blocks, r1, a.cs, a.bs, j);
         uint4 o0, o1;
         deq_chunk<NV>(x, y, s0, s1, o0, o1);
         erow[2 * j] = o0;
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
 #pragma unroll
     for (int rr = 0; rr < kPjMaxTok; ++rr) {
       const int t = rr & 7;
-      if (t < T && lane < nck) x[rr] = load_chunk<FMT == 1>(a.table, a.blocks, sm->rid[t][rr >> 3], a.D, kb + lane);
+      if (t < T && lane < nck) x[rr] = load_chunk<FMT == 1>(a.table, a.blocks, sm->rid[t][rr >> 3], a.cs, a.bs, kb + lane);
     }
 #pragma unroll
     for (int rr = 0; rr < kPjMaxTok; ++rr) {
@@ -492,8 +492,8 @@ __global__ void __launch_bounds__(kPjThreads, 1) decode_proj_kernel(const Decode
             sa[r] = __ldg(a.scales + row);
           } else {
             const int64_t r0 = sm->rid[t][0], r1 = sm->rid[t][1];
-            ra[r] = load_chunk<FMT == 1>(a.table, a.blocks, r0, a.D, j);
-            rb[r] = load_chunk<FMT == 1>(a.table, a.blocks, r1, a.D, j);
+            ra[r] = load_chunk<FMT == 1>(a.table, a.blocks, r0, a.cs, a.bs, j);
+            rb[r] = load_chunk<FMT == 1>(a.table, a.blocks, r1, a.cs, a.bs, j);
             sa[r] = __ldg(a.scales + r0);
             sb[r] = __ldg(a.scales + r1);
           }

@@ -511,18 +511,21 @@ template <bool NV> struct RowChunk;
 template <> struct RowChunk<false> { uint4 c; };
 template <> struct RowChunk<true> { uint2 c; uint32_t b; };
 
-// Chunk j of global row `row` (sub-table offset already added) of a table with
-// row_dim D: codes at row * D (E4M3) or row * D/2 (NVFP4), block scales at row * D/16.
+// Chunk j (16 elements) of global row `row` (sub-table offset already added):
+// codes at row * cs, block scales at row * bs, both strides in bytes. E4M3:
+// cs = D. NVFP4 in separate arrays: cs = D/2, bs = D/16; NVFP4 rows (codes and
+// block scales side by side, blocks = codes + D/2): cs = bs = 9D/16.
 template <bool NV>
 __device__ __forceinline__ RowChunk<NV> load_chunk(const uint8_t* codes, const uint8_t* blocks, int64_t row,
-                                                   int32_t D, int j) {
+                                                   int32_t cs, int32_t bs, int j) {
   RowChunk<NV> r;
   if constexpr (NV) {
-    r.c = ld_stream_v2(codes + row * (D / 2) + 8 * j);
-    r.b = ld_stream_u8(blocks + row * (D / 16) + j);
+    r.c = ld_stream_v2(codes + row * cs + 8 * j);
+    r.b = ld_stream_u8(blocks + row * bs + j);
   } else {
     (void)blocks;
-    r.c = ld_stream_v4(codes + row * D + 16 * j);
+    (void)bs;
+    r.c = ld_stream_v4(codes + row * cs + 16 * j);
   }
   return r;
 }

@@ -51,7 +51,9 @@ struct TableRef {
   const uint8_t* codes;        // E4M3: one byte per element; NVFP4: two E2M1 codes per byte
   const uint8_t* blocks;       // NVFP4: one E4M3 block scale per 16 elements; else null
   const float* scales;         // fp32 per row
-  int32_t nvfp4;               // 1: PLE_TABLE_NVFP4
+  int32_t nvfp4;               // 1: PLE_TABLE_NVFP4 or PLE_TABLE_NVFP4_ROWS
+  int32_t cs, bs;              // bytes from one row's codes (block scales) to the next row's
+  int32_t nv_rows;             // 1: PLE_TABLE_NVFP4_ROWS (blocks = codes + D/2, one piece per row)
 };
 
 // Prepare stage: sequence map, n-gram row IDs, gate, state snapshot.
@@ -200,7 +202,8 @@ struct DecodeEmbedArgs {
   const uint8_t* table;
   const uint8_t* blocks;   // NVFP4 block scales (null otherwise)
   const float* scales;
-  int32_t format;          // ple_table_format
+  int32_t cs, bs;          // row strides in bytes of the codes and the block scales (TableRef)
+  int32_t format;          // ple_table_format (PLE_TABLE_NVFP4 for both NVFP4 layouts)
   int32_t D, H;
   const __nv_bfloat16* hidden;   // [T][H], or null: the gate is computed later
   const __nv_bfloat16* w_gate;
@@ -248,7 +251,8 @@ struct DecodeProjArgs {
   const uint8_t* table;
   const uint8_t* blocks;
   const float* scales;
-  int32_t format;          // ple_table_format
+  int32_t cs, bs;          // row strides in bytes of the codes and the block scales (TableRef)
+  int32_t format;          // ple_table_format (PLE_TABLE_NVFP4 for both NVFP4 layouts)
   int32_t* step_count;     // fused steps: CTAs past their hashing, zero between launches
   const __nv_bfloat16* hidden;
   const __nv_bfloat16* w_gate;

@@ -212,8 +212,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const int2* __restrict__ id
   }
   const int64_t row0 = id.x;
   const int64_t row1 = rows0 + id.y;
-  const RowChunk<NV> a = load_chunk<NV>(t.codes, t.blocks, row0, D, c);
-  const RowChunk<NV> b = load_chunk<NV>(t.codes, t.blocks, row1, D, c);
+  const RowChunk<NV> a = load_chunk<NV>(t.codes, t.blocks, row0, t.cs, t.bs, c);
+  const RowChunk<NV> b = load_chunk<NV>(t.codes, t.blocks, row1, t.cs, t.bs, c);
   const float s0 = __ldg(t.scales + row0);
   const float s1 = __ldg(t.scales + row1);
   uint4 o0, o1;
@@ -490,8 +490,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         for (int r = 0; r < kEmbedD16; ++r) {
           const int j = lane + 32 * r;
           if (with_rows && j < D16) {
-            ca[r] = load_chunk<NV>(tab.codes, tab.blocks, ra, D, j);
-            cb[r] = load_chunk<NV>(tab.codes, tab.blocks, rb, D, j);
+            ca[r] = load_chunk<NV>(tab.codes, tab.blocks, ra, tab.cs, tab.bs, j);
+            cb[r] = load_chunk<NV>(tab.codes, tab.blocks, rb, tab.cs, tab.bs, j);
           }
         }
         const float s0 = with_rows ? __ldg(tab.scales + ra) : 0.f;
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           if (j < D16) emit(j, ca[r], cb[r]);
         }
         for (int j = lane + 32 * kEmbedD16; j < D16; j += 32)
-          emit(j, load_chunk<NV>(tab.codes, tab.blocks, ra, D, j), load_chunk<NV>(tab.codes, tab.blocks, rb, D, j));
+          emit(j, load_chunk<NV>(tab.codes, tab.blocks, ra, tab.cs, tab.bs, j), load_chunk<NV>(tab.codes, tab.blocks, rb, tab.cs, tab.bs, j));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.empty[slot]));
@@ -602,10 +602,12 @@ __global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs
   }
 }
 
-// Gather units of a token: E4M3 and the multi-head layout one 16-code chunk per
-// thread; NVFP4 two chunks (16 bytes of packed codes and 2 block-scale bytes
-// per row), so that each load is as wide as an E4M3 thread's.
-template <int FMT> constexpr int kSplitChunksPerThread = FMT == 1 ? 2 : 1;
+// Gather units of a token: E4M3 one 16-code chunk per thread (16 bytes from
+// each of the two rows); NVFP4 two chunks (16 bytes of packed codes and 2
+// block-scale bytes per row); the multi-head layout two consecutive chunks of
+// the token's head rows (32 bytes), so that every thread keeps about as many
+// bytes in flight as an E4M3 thread.
+template <int FMT> constexpr int kSplitChunksPerThread = FMT == 0 ? 1 : 2;
 
 template <int FMT>
 __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
@@ -628,29 +630,55 @@ __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
   constexpr int CPT = kSplitChunksPerThread<FMT>;
   const int units = D / (16 * CPT);                              // per token
   const int64_t idx = (n_blocks - 1 - b) * kSplitThreads + threadIdx.x;
+  if constexpr (FMT == 2) {
+    // warp w takes the 64 chunks [64w, 64w + 64) of the batch's head rows (16 per
+    // token, side by side), lane l chunks 64w + l and 64w + l + 32: both loads in
+    // flight at once, each load instruction 32 consecutive chunks
+    const int hd = D / kHeads, cph = hd / 16, nck = D / 16;
+    const int64_t total = static_cast<int64_t>(a.T) * nck;
+    const int64_t g0 = (idx >> 5) * 64 + (threadIdx.x & 31);
+    if (g0 >= total) return;
+    uint4 v[2];
+    float sc[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t g = g0 + 32 * k;
+      if (g < total) {
+        const int32_t t = static_cast<int32_t>(g / nck);
+        const int c = static_cast<int>(g - static_cast<int64_t>(t) * nck), hh = c / cph;
+        const int64_t row = static_cast<int64_t>(hh) * a.rows0 + a.ids[static_cast<int64_t>(t) * kHeads + hh];
+        v[k] = ld_stream_v4(tab.codes + row * hd + (c - hh * cph) * 16);
+        sc[k] = __ldg(tab.scales + row);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t g = g0 + 32 * k;
+      if (g < total) {
+        uint4 o0, o1;
+        deq16_one(v[k], sc[k], o0, o1);
+        uint4* dst = reinterpret_cast<uint4*>(e + g * 16);
+        dst[0] = o0;
+        dst[1] = o1;
+      }
+    }
+    return;
+  }
   if (idx >= static_cast<int64_t>(a.T) * units) return;
   const int32_t t = static_cast<int32_t>(idx / units);
   const int c = static_cast<int>(idx - static_cast<int64_t>(t) * units);
   uint4* dst = reinterpret_cast<uint4*>(e + idx * 16 * CPT);
-  if constexpr (FMT == 2) {
-    const int hd = D / kHeads, cph = hd / 16, hh = c / cph;
-    const int64_t row = static_cast<int64_t>(hh) * a.rows0 + a.ids[static_cast<int64_t>(t) * kHeads + hh];
-    const uint4 v = ld_stream_v4(tab.codes + row * hd + (c - hh * cph) * 16);
-    uint4 o0, o1;
-    deq16_one(v, __ldg(tab.scales + row), o0, o1);
-    dst[0] = o0;
-    dst[1] = o1;
-  } else {
+  {
     const int2 id = reinterpret_cast<const int2*>(a.ids)[t];
     const int64_t row0 = id.x, row1 = a.rows0 + id.y;
     const float sa = __ldg(tab.scales + row0);
     const float sb = __ldg(tab.scales + row1);
     if constexpr (FMT == 1) {
       // elements [32c, 32c + 32): 16 bytes of codes and 2 block-scale bytes per row
-      const uint4 xa = ld_stream_v4(tab.codes + row0 * (D / 2) + 16 * c);
-      const uint4 xb = ld_stream_v4(tab.codes + row1 * (D / 2) + 16 * c);
-      const uint32_t ba = ld_stream_u16(tab.blocks + row0 * (D / 16) + 2 * c);
-      const uint32_t bb = ld_stream_u16(tab.blocks + row1 * (D / 16) + 2 * c);
+      const uint4 xa = ld_stream_v4(tab.codes + row0 * tab.cs + 16 * c);
+      const uint4 xb = ld_stream_v4(tab.codes + row1 * tab.cs + 16 * c);
+      const uint32_t ba = ld_stream_u16(tab.blocks + row0 * tab.bs + 2 * c);
+      const uint32_t bb = ld_stream_u16(tab.blocks + row1 * tab.bs + 2 * c);
       uint4 o0, o1, o2, o3;
       deq16_nv(make_uint2(xa.x, xa.y), make_uint2(xb.x, xb.y), ba & 0xFFu, bb & 0xFFu, sa, sb, o0, o1);
       deq16_nv(make_uint2(xa.z, xa.w), make_uint2(xb.z, xb.w), ba >> 8, bb >> 8, sa, sb, o2, o3);
@@ -659,8 +687,8 @@ __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
       dst[2] = o2;
       dst[3] = o3;
     } else {
-      const RowChunk<false> ca = load_chunk<false>(tab.codes, tab.blocks, row0, D, c);
-      const RowChunk<false> cb = load_chunk<false>(tab.codes, tab.blocks, row1, D, c);
+      const RowChunk<false> ca = load_chunk<false>(tab.codes, tab.blocks, row0, tab.cs, tab.bs, c);
+      const RowChunk<false> cb = load_chunk<false>(tab.codes, tab.blocks, row1, tab.cs, tab.bs, c);
       uint4 o0, o1;
       deq_chunk<false>(ca, cb, sa, sb, o0, o1);
       dst[0] = o0;
@@ -810,9 +838,15 @@ __global__ void __launch_bounds__(kBkThreads, kBkCtasPerSm)
         if (lane < kRowsN) {
           const int64_t row = global_row(lane, id);
           if constexpr (FMT == 1) {
+            // the row's D/2 code bytes, then its D/16 block-scale bytes: one copy
+            // when the table keeps them side by side
             const uint32_t o = lane * static_cast<uint32_t>(D / 2 + D / 16);
-            bulk_load(smem_u32(st + o), tab.codes + row * (D / 2), static_cast<uint32_t>(D / 2), fb);
-            bulk_load(smem_u32(st + o + D / 2), tab.blocks + row * (D / 16), static_cast<uint32_t>(D / 16), fb);
+            if (tab.nv_rows) {
+              bulk_load(smem_u32(st + o), tab.codes + row * tab.cs, static_cast<uint32_t>(D / 2 + D / 16), fb);
+            } else {
+              bulk_load(smem_u32(st + o), tab.codes + row * tab.cs, static_cast<uint32_t>(D / 2), fb);
+              bulk_load(smem_u32(st + o + D / 2), tab.blocks + row * tab.bs, static_cast<uint32_t>(D / 16), fb);
+            }
           } else {
             bulk_load(smem_u32(st + lane * D), tab.codes + row * D, static_cast<uint32_t>(D), fb);
           }
@@ -1062,7 +1096,7 @@ bool embed_bulk_ok(const PrepareArgs& a, const TableRef& table, int32_t D, const
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (e == nullptr || !al16(e) || !al16(table.codes)) return false;
   if (FMT == 0 ? D % 16 != 0 : D % 256 != 0) return false;   // NVFP4: D / 16 block-scale bytes per row
-  if (FMT == 1 && !al16(table.blocks)) return false;
+  if (FMT == 1 && (!al16(table.blocks) || table.cs % 16 != 0 || table.bs % 16 != 0)) return false;
   if (gate && (a.H % 8 != 0 || !al16(a.hidden) || !al16(a.w_gate))) return false;
   return static_cast<size_t>(kBkStages) * bk_stage_bytes<FMT>(D, a.H, gate) <= kBkSmemPerCta;
 }

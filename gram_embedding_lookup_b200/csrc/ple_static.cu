@@ -141,7 +141,7 @@ extern "C" ple_status ple_embed_static(const int32_t* tokens, int32_t T, const i
   pa.H = 0;
   pa.status = status;
   if (ple::launch_prepare(pa, stream) != cudaSuccess) return PLE_ERR_CUDA;
-  if (ple::launch_gather(ids, T, ple::TableRef{table, nullptr, scales, 0}, rows0, rows1, row_dim,
+  if (ple::launch_gather(ids, T, ple::TableRef{table, nullptr, scales, 0, row_dim, 0, 0}, rows0, rows1, row_dim,
                         static_cast<__half*>(e_out), false, stream) != cudaSuccess)
     return PLE_ERR_CUDA;
   if (status_out != nullptr &&

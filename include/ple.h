@@ -90,8 +90,19 @@ typedef enum { PLE_OUT_BF16 = 0, PLE_OUT_F32 = 1 } ple_out_dtype;
  *     (k_n the order's key below; head 0 is the two-order row), and e is the
  *     16 dequantised rows side by side in sub-table order. rows[1] must equal
  *     rows[0]; row_dim % 256 == 0. The same 51,200,245,760 bytes hold
- *     16 x 20,000,096 rows of 160. Row IDs are [T][16] for this format. */
-typedef enum { PLE_TABLE_E4M3 = 0, PLE_TABLE_NVFP4 = 1, PLE_TABLE_E4M3_HEADS = 2 } ple_table_format;
+ *     16 x 20,000,096 rows of 160. Row IDs are [T][16] for this format.
+ *   PLE_TABLE_NVFP4_ROWS: the contents of PLE_TABLE_NVFP4 (the same codes,
+ *     block scales and row scales, the same results bit for bit) stored row by
+ *     row: each row's row_dim/2 code bytes followed by its row_dim/16
+ *     block-scale bytes, row_dim*9/16 contiguous bytes per row. A token's row
+ *     is then one piece of memory, which the prefill embed fetches with one
+ *     copy instead of two. block_scales must be NULL; row_dim % 256 == 0. */
+typedef enum {
+  PLE_TABLE_E4M3 = 0,
+  PLE_TABLE_NVFP4 = 1,
+  PLE_TABLE_E4M3_HEADS = 2,
+  PLE_TABLE_NVFP4_ROWS = 3
+} ple_table_format;
 
 /* Sizes fixed at creation. hidden % 128 == 0, row_dim % 64 == 0,
  * 0 < rows[n] < 2^31. max_tokens bounds T of every call (and B*q of a decode
@@ -119,12 +130,16 @@ typedef struct {
                                 byte i of the row; row r of sub-table n at byte offset
                                 (n*rows[0] + r)*row_dim/2.
                                 E4M3_HEADS: sub-table h (0..15), row r at byte offset
-                                (h*rows[0] + r)*(row_dim/16). 16-byte aligned */
+                                (h*rows[0] + r)*(row_dim/16).
+                                NVFP4_ROWS: row r of sub-table n at byte offset
+                                (n*rows[0] + r)*row_dim*9/16: its packed codes as for
+                                NVFP4, then at row_dim/2 its block scales as for
+                                block_scales below. 16-byte aligned */
   const float* scales;       /* fp32 per-row scales; sub-table n, row r at n*rows[0] + r */
   const void* w_proj;        /* bf16 [row_dim][hidden], row-major */
   const void* w_gate;        /* bf16 [hidden] */
   const float* conv_w;       /* fp32 [hidden][4]; tap 3 multiplies the current token */
-  const uint8_t* block_scales; /* NVFP4 only (NULL for E4M3): E4M3 scale of elements
+  const uint8_t* block_scales; /* NVFP4 only (NULL for the other formats): E4M3 scale of elements
                                 [16j, 16j+16) of row r of sub-table n at byte offset
                                 (n*rows[0] + r)*row_dim/16 + j; 16-byte aligned */
 } ple_weights;

@@ -207,6 +207,11 @@ class SynthNvTable:
     def scales(self, order: int, rows) -> np.ndarray:
         return table_scales(self.seed, self.rows_per_order, order, rows)
 
+    def packed_rows(self, order: int, rows) -> np.ndarray:
+        """The given rows as the row-by-row layout stores them: uint8 [len(rows)][9D/16],
+        each row's D/2 code bytes followed by its D/16 block-scale bytes."""
+        return np.concatenate([self.codes(order, rows), self.block_scales(order, rows)], axis=1)
+
     def full(self):
         """The whole table as arrays (small tables only): codes, block scales, scales."""
         r = np.arange(self.rows_per_order)
@@ -434,6 +439,9 @@ def _synth_lib():
         lib.ple_synth_fill_nvfp4.restype = ctypes.c_int
         lib.ple_synth_fill_nvfp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                              ctypes.c_int32, ctypes.c_uint64, ctypes.c_void_p]
+        lib.ple_synth_fill_nvfp4_rows.restype = ctypes.c_int
+        lib.ple_synth_fill_nvfp4_rows.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                                  ctypes.c_uint64, ctypes.c_void_p]
         lib.ple_synth_stream_base.restype = ctypes.c_uint64
         lib.ple_synth_stream_base.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
         _SYNTH_LIB = lib
@@ -448,6 +456,17 @@ def fill_nv_table_device(codes_ptr: int, block_ptr: int, scales_ptr: int, rows_p
                                            ctypes.c_void_p(stream))
     if rc != 0:
         raise RuntimeError(f"ple_synth_fill_nvfp4 failed with CUDA error {rc}")
+
+
+def fill_nv_rows_table_device(rows_ptr: int, scales_ptr: int, rows_per_order: int, row_dim: int, seed: int,
+                              stream: int = 0) -> None:
+    """Fill a device NVFP4 table stored row by row, u8[2][R][9D/16] (each row's D/2 code
+    bytes, then its D/16 block-scale bytes: the contents of fill_nv_table_device), and
+    scales f32[2][R]."""
+    rc = _synth_lib().ple_synth_fill_nvfp4_rows(ctypes.c_void_p(rows_ptr), ctypes.c_void_p(scales_ptr),
+                                                rows_per_order, row_dim, seed, ctypes.c_void_p(stream))
+    if rc != 0:
+        raise RuntimeError(f"ple_synth_fill_nvfp4_rows failed with CUDA error {rc}")
 
 
 def fill_table_device(table_ptr: int, scales_ptr: int, rows_per_order: int, row_dim: int,

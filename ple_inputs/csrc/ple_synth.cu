@@ -80,6 +80,30 @@ __global__ void fill_nv_bytes_kernel(uint32_t* __restrict__ dst, uint64_t n4, ui
   }
 }
 
+// The same bytes stored row by row: word w of row r (row_words = 9D/64 words)
+// is code word w of the row (w < D/8) or block-scale word w - D/8, each drawn
+// from the counter index it has in its own flat array.
+__global__ void fill_nv_rows_kernel(uint32_t* __restrict__ dst, uint64_t rows, int32_t row_dim, uint64_t code_base,
+                                    uint64_t block_base) {
+  const uint64_t cw = static_cast<uint64_t>(row_dim / 8), bw = static_cast<uint64_t>(row_dim / 64);
+  const uint64_t row_words = cw + bw, n4 = rows * row_words;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t c = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < n4; c += stride) {
+    const uint64_t r = c / row_words, k = c - r * row_words;
+    const bool code = k < cw;
+    const uint64_t first = code ? (r * cw + k) * 4 : (r * bw + (k - cw)) * 4;
+    const uint64_t base = code ? code_base : block_base;
+    uint32_t v = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint64_t u = sm64_mix(base + (first + b + 1) * kGamma);
+      const uint32_t byte = code ? static_cast<uint32_t>(u >> 56) : kNvBlockBase + static_cast<uint32_t>(u >> 60);
+      v |= byte << (8 * b);
+    }
+    dst[c] = v;
+  }
+}
+
 }  // namespace
 
 extern "C" uint64_t ple_synth_stream_base(uint64_t seed, uint32_t tag) {
@@ -123,5 +147,24 @@ extern "C" int ple_synth_fill_nvfp4(uint8_t* codes, uint8_t* blocks, float* scal
   fill_nv_bytes_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<uint32_t*>(blocks), block_bytes / 4,
                                                     stream_base(seed, kTagNvBlocks), 1);
   fill_scales_kernel<<<sms * 2, 256, 0, stream>>>(scales, rows, stream_base(seed, kTagScales));
+  return static_cast<int>(cudaGetLastError());
+}
+
+// The NVFP4 table stored row by row (rows u8[2][R][9D/16]: each row's D/2 code
+// bytes, then its D/16 block-scale bytes), with the same contents as
+// ple_synth_fill_nvfp4, and scales f32[2][R]. Returns 0 or a CUDA error code.
+extern "C" int ple_synth_fill_nvfp4_rows(uint8_t* rows, float* scales, int64_t rows_per_order, int32_t row_dim,
+                                         uint64_t seed, cudaStream_t stream) {
+  if (rows == nullptr || scales == nullptr || rows_per_order <= 0 || row_dim <= 0 || (row_dim % 64) != 0 ||
+      (reinterpret_cast<uintptr_t>(rows) % 4) != 0) {
+    return static_cast<int>(cudaErrorInvalidValue);
+  }
+  const uint64_t n = 2ull * static_cast<uint64_t>(rows_per_order);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  fill_nv_rows_kernel<<<sms * 8, 256, 0, stream>>>(reinterpret_cast<uint32_t*>(rows), n, row_dim,
+                                                   stream_base(seed, kTagNvCodes), stream_base(seed, kTagNvBlocks));
+  fill_scales_kernel<<<sms * 2, 256, 0, stream>>>(scales, n, stream_base(seed, kTagScales));
   return static_cast<int>(cudaGetLastError());
 }

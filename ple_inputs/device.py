@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 import gram_embedding_lookup_b200 as ple
-from . import Workload, fill_nv_table_device, fill_table_device
+from . import Workload, fill_nv_rows_table_device, fill_nv_table_device, fill_table_device
 
 
 def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
@@ -29,6 +29,8 @@ class DeviceLayer:
 
     table_format ple.PLE_TABLE_NVFP4 builds the synthetic NVFP4 table instead
     (packed codes in ``table``, E4M3 block scales in ``block_scales``);
+    ple.PLE_TABLE_NVFP4_ROWS the same contents row by row in ``table`` (each
+    row's codes, then its block scales);
     ple.PLE_TABLE_E4M3_HEADS builds the multi-head table (16 sub-tables of
     rows_per_order rows of row_dim / 16 codes)."""
 
@@ -51,6 +53,11 @@ class DeviceLayer:
             self.block_scales = torch.empty(2 * R * D // 16, dtype=torch.uint8, device="cuda")
             fill_nv_table_device(self.table.data_ptr(), self.block_scales.data_ptr(), self.scales.data_ptr(), R, D,
                                  w.table_seed, s.cuda_stream)
+        elif table_format == ple.PLE_TABLE_NVFP4_ROWS:
+            self.table = torch.empty(2 * R * (D // 2 + D // 16), dtype=torch.uint8, device="cuda")
+            self.block_scales = None
+            fill_nv_rows_table_device(self.table.data_ptr(), self.scales.data_ptr(), R, D, w.table_seed,
+                                      s.cuda_stream)
         else:
             self.table = torch.empty(2 * R * D, dtype=torch.uint8, device="cuda")
             self.block_scales = None

@@ -1,9 +1,12 @@
-"""GPU parity of the NVFP4 table variant (PLE_TABLE_NVFP4) against the oracle.
+"""GPU parity of the NVFP4 table variant against the oracle, in both layouts.
 
 Every call goes through the C ABI. The table is the synthetic NVFP4 table of
-``ple_inputs`` (packed E2M1 codes, E4M3 block scales, per-row fp32 scales);
-the oracle reads the same bytes through ``oracle.Nvfp4ArrayTable`` or the
-host generator.
+``ple_inputs`` (packed E2M1 codes, E4M3 block scales, per-row fp32 scales),
+stored either in two arrays (PLE_TABLE_NVFP4) or row by row with each row's
+block scales after its codes (PLE_TABLE_NVFP4_ROWS, which needs row_dim % 256
+== 0: its small workloads are the tiny and mid ones at row_dim 256). The
+oracle reads the same contents through ``oracle.Nvfp4ArrayTable`` or the host
+generator, whatever the layout.
 """
 import numpy as np
 import pytest
@@ -20,37 +23,59 @@ from tests.test_gpu_parity import _sample, dev_bf16, dev_i32, gpu_decode, gpu_fo
 pytestmark = pytest.mark.gpu
 
 
-def _layer(w, max_tokens, max_seqs):
+LAYOUTS = [ple.PLE_TABLE_NVFP4, ple.PLE_TABLE_NVFP4_ROWS]
+LAYOUT_IDS = ["arrays", "rows"]
+
+
+def _wide(w, name):
+    """The workload at row_dim 256 (the row layout's smallest row width)."""
+    return pi.Workload(name, w.vocab, w.rows_per_order, 256, w.hidden, w.table_seed, w.seed, w.extra)
+
+
+def _layer(w, max_tokens, max_seqs, fmt):
     from ple_inputs.device import DeviceLayer
-    L = DeviceLayer(w, max_tokens=max_tokens, max_seqs=max_seqs, table_format=ple.PLE_TABLE_NVFP4)
+    L = DeviceLayer(w, max_tokens=max_tokens, max_seqs=max_seqs, table_format=fmt)
+    L.rows_layout = fmt == ple.PLE_TABLE_NVFP4_ROWS
     return L
 
 
-@pytest.fixture(scope="module")
-def nv_tiny():
+def _code_views(L):
+    """Torch views [2][R][D/2] of the device codes and [2][R][D/16] of the block scales."""
+    R, D = L.w.rows_per_order, L.w.row_dim
+    if L.rows_layout:
+        t = L.table.view(2, R, D // 2 + D // 16)
+        return t[:, :, :D // 2], t[:, :, D // 2:]
+    return L.table.view(2, R, D // 2), L.block_scales.view(2, R, D // 16)
+
+
+@pytest.fixture(scope="module", params=LAYOUTS, ids=LAYOUT_IDS)
+def nv_tiny(request):
     w = pi.workload("tiny")
-    L = _layer(w, 2048, 64)
+    if request.param == ple.PLE_TABLE_NVFP4_ROWS:
+        w = _wide(w, "tiny256")
+    L = _layer(w, 4608, 64, request.param)
     L.host_table = O.Nvfp4ArrayTable(*pi.SynthNvTable(w.table_seed, w.rows_per_order, w.row_dim).full())
     yield L
     L.close()
 
 
-@pytest.fixture(scope="module")
-def nv_mid():
-    L = _layer(MID, 4096, 64)
-    L.host_table = O.Nvfp4ArrayTable(*pi.SynthNvTable(MID.table_seed, MID.rows_per_order, MID.row_dim).full())
+@pytest.fixture(scope="module", params=LAYOUTS, ids=LAYOUT_IDS)
+def nv_mid(request):
+    w = MID if request.param == ple.PLE_TABLE_NVFP4 else _wide(MID, "mid256")
+    L = _layer(w, 4096, 64, request.param)
+    L.host_table = O.Nvfp4ArrayTable(*pi.SynthNvTable(w.table_seed, w.rows_per_order, w.row_dim).full())
     yield L
     L.close()
 
 
-@pytest.fixture(scope="module")
-def nv_full():
+@pytest.fixture(scope="module", params=LAYOUTS, ids=LAYOUT_IDS)
+def nv_full(request):
     w = pi.workload("prefill")
     need = 2 * w.rows_per_order * (w.row_dim // 2 + w.row_dim // 16)
     free, _ = torch.cuda.mem_get_info()
     if free < need + (8 << 30):
         pytest.skip(f"needs {need / 1e9:.0f} GB for the NVFP4 table, {free / 1e9:.0f} GB free")
-    L = _layer(w, 16384, 64)
+    L = _layer(w, 16384, 64, request.param)
     L.host_table = pi.SynthNvTable(w.table_seed, w.rows_per_order, w.row_dim)
     yield L
     release_device_memory(L)
@@ -75,9 +100,17 @@ def _ulp(a16, b16):
 
 def test_nv_device_table_matches_host_generator(nv_tiny):
     w = nv_tiny.w
-    codes, blocks, scales = pi.SynthNvTable(w.table_seed, w.rows_per_order, w.row_dim).full()
-    assert np.array_equal(nv_tiny.table.cpu().numpy(), codes.ravel())
-    assert np.array_equal(nv_tiny.block_scales.cpu().numpy(), blocks.ravel())
+    syn = pi.SynthNvTable(w.table_seed, w.rows_per_order, w.row_dim)
+    codes, blocks, scales = syn.full()
+    if nv_tiny.rows_layout:
+        r = np.arange(w.rows_per_order)
+        packed = np.stack([syn.packed_rows(0, r), syn.packed_rows(1, r)])
+        assert np.array_equal(nv_tiny.table.cpu().numpy(), packed.ravel())
+    else:
+        assert np.array_equal(nv_tiny.table.cpu().numpy(), codes.ravel())
+        assert np.array_equal(nv_tiny.block_scales.cpu().numpy(), blocks.ravel())
+    c, b = _code_views(nv_tiny)
+    assert np.array_equal(c.cpu().numpy(), codes) and np.array_equal(b.cpu().numpy(), blocks)
     assert np.array_equal(nv_tiny.scales.cpu().numpy(), scales.ravel())
 
 
@@ -107,8 +140,7 @@ def test_nv_gather_every_code_and_block_scale(nv_tiny):
         blocks[0, i] = kinds[(i + np.arange(D // 16)) % len(kinds)]
         blocks[1, i] = kinds[(3 * i + 2 * np.arange(D // 16) + 1) % len(kinds)]
     scales = np.stack([np.linspace(0.01, 0.2, n), np.linspace(0.3, 0.02, n)]).astype(np.float32)
-    tab = L.table.view(2, R, D // 2)
-    blk = L.block_scales.view(2, R, D // 16)
+    tab, blk = _code_views(L)
     sc = L.scales.view(2, R)
     saved = (tab[:, :n].clone(), blk[:, :n].clone(), sc[:, :n].clone())
     try:
@@ -122,10 +154,20 @@ def test_nv_gather_every_code_and_block_scale(nv_tiny):
         tab[:, :n], blk[:, :n], sc[:, :n] = saved
         torch.cuda.synchronize()
     with np.errstate(invalid="ignore", over="ignore"):
-        ref = O.embed(O.Nvfp4ArrayTable(codes, blocks, scales), ids).astype(np.float16)
+        exact = O.embed(O.Nvfp4ArrayTable(codes, blocks, scales), ids)
+        # the same table with every sign bit cleared: the sum of the two terms' magnitudes
+        mag = O.embed(O.Nvfp4ArrayTable(codes & 0x77, blocks & 0x7F, np.abs(scales)), ids)
+    ref = exact.astype(np.float16)
     nan = np.isnan(ref)
     assert nan.any() and np.array_equal(np.isnan(got), nan)
-    assert _ulp(got[~nan], ref[~nan]).max() <= 1
+    # e is computed in fp32 and rounded to fp16: within one fp16 ulp, except where
+    # the two orders' terms cancel, there within the fp32 rounding of the terms
+    # (2^-23 of their magnitudes) plus an fp16 ulp
+    ulp = _ulp(got[~nan], ref[~nan])
+    err = np.abs(got[~nan].astype(np.float64) - exact[~nan])
+    lim = 2.0 ** -23 * mag[~nan] + np.abs(np.spacing(ref[~nan]))
+    assert np.all((ulp <= 1) | (err <= lim))
+    assert np.mean(ulp > 1) < 1e-4
 
 
 @pytest.mark.parametrize("path", [0, 1, 2])
@@ -157,6 +199,28 @@ def test_nv_forward_mid_with_state(nv_mid, path):
     assert_close(out, ref["out"], f"nvfp4 mid path {path}")
     assert np.array_equal(st[0], ref["hist_out"])
     assert_close(st[1], ref["conv_out"], "nvfp4 mid state")
+
+
+@pytest.mark.parametrize("lengths", [[4000, 90, 6], [1, 4200, 0, 17]])
+def test_nv_bulk_embed_batches(nv_tiny, lengths):
+    """Batches of 4,096 tokens or more take the bulk-copy embed (every NVFP4 row
+    in one copy in the row layout, two in the array layout): every output
+    against the oracle, with carried state."""
+    w = nv_tiny.w
+    rng = np.random.default_rng(sum(lengths))
+    T, S = sum(lengths), len(lengths)
+    toks = rng.integers(0, w.vocab, T).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    hid = pi.hidden_bf16(rng, T, w.hidden)
+    hist = rng.integers(-1, w.vocab, (S, 2)).astype(np.int32)
+    conv = rng.standard_normal((S, 3, w.hidden)).astype(np.float32)
+    W = nv_tiny.host_weights
+    ref = O.ple_forward(toks, offs, hid, W.w_proj, W.w_gate, W.conv_w, nv_tiny.host_table, w.rows_per_order,
+                        hist=hist, conv_state=conv)
+    out, st = gpu_forward(nv_tiny, toks, offs, hid, 1, state=(hist, conv))
+    assert_close(out, ref["out"], f"nvfp4 bulk embed {lengths}")
+    assert np.array_equal(st[0], ref["hist_out"])
+    assert_close(st[1], ref["conv_out"], "nvfp4 bulk embed state")
 
 
 @pytest.mark.parametrize("shape", [(1, 1), (8, 1), (5, 3), (16, 1), (6, 3)])

@@ -22,21 +22,28 @@ R0, R1 = 3000, 5003
 
 
 class _Layer:
-    """A handle over hand-made sub-tables of R0 and R1 rows (E4M3 or NVFP4)."""
+    """A handle over hand-made sub-tables of R0 and R1 rows (E4M3, NVFP4 in two
+    arrays, or NVFP4 row by row at row_dim 256)."""
 
     def __init__(self, fmt):
         from ple_inputs.device import bf16_tensor
         w = pi.workload("tiny")
+        if fmt == ple.PLE_TABLE_NVFP4_ROWS:
+            w = pi.Workload("tiny256", w.vocab, w.rows_per_order, 256, w.hidden, w.table_seed, w.seed, w.extra)
         self.w = w
         D, H = w.row_dim, w.hidden
         rng = np.random.default_rng(41 + fmt)
         scales = rng.uniform(0.01, 0.1, R0 + R1).astype(np.float32)
-        if fmt == ple.PLE_TABLE_NVFP4:
+        if fmt in (ple.PLE_TABLE_NVFP4, ple.PLE_TABLE_NVFP4_ROWS):
             codes = rng.integers(0, 256, (R0 + R1, D // 2)).astype(np.uint8)
             blocks = rng.integers(0x30, 0x40, (R0 + R1, D // 16)).astype(np.uint8)
             self.host_table = O.Nvfp4ArrayTable([codes[:R0], codes[R0:]], [blocks[:R0], blocks[R0:]],
                                                 [scales[:R0], scales[R0:]])
-            self.block_scales = torch.from_numpy(blocks.ravel()).cuda()
+            if fmt == ple.PLE_TABLE_NVFP4_ROWS:             # each row's block scales after its codes
+                codes = np.concatenate([codes, blocks], axis=1)
+                self.block_scales = None
+            else:
+                self.block_scales = torch.from_numpy(blocks.ravel()).cuda()
         else:
             codes = rng.integers(0, 256, (R0 + R1, D)).astype(np.uint8)
             codes[(codes & 0x7F) == 0x7F] = 0x42                # finite codes only
@@ -61,7 +68,7 @@ class _Layer:
         ple.ple_destroy(self.handle)
 
 
-@pytest.fixture(scope="module", params=[0, 1], ids=["e4m3", "nvfp4"])
+@pytest.fixture(scope="module", params=[0, 1, 3], ids=["e4m3", "nvfp4", "nvfp4_rows"])
 def layer(request):
     L = _Layer(request.param)
     yield L

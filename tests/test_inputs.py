@@ -69,3 +69,15 @@ def test_mtp_session_structure():
     for toks, hid, nc in s["steps"]:
         assert toks.shape == (64, 3) and hid.shape == (192, 2560)
         assert np.all(toks[:19] == toks[0]) and nc.min() >= 1 and nc.max() <= 3
+
+
+def test_nv_packed_rows_layout():
+    """The row layout of the NVFP4 table: row r is its D/2 code bytes, then its D/16
+    block-scale bytes (9D/16 bytes), the same contents as the two-array layout."""
+    t = pi.SynthNvTable(seed=3, rows_per_order=64, row_dim=256)
+    rows = np.array([0, 63, 5, 5])
+    p = t.packed_rows(1, rows)
+    assert p.dtype == np.uint8 and p.shape == (4, 256 // 2 + 256 // 16)
+    assert np.array_equal(p[:, :128], t.codes(1, rows))
+    assert np.array_equal(p[:, 128:], t.block_scales(1, rows))
+    assert not np.array_equal(t.packed_rows(0, rows), p)

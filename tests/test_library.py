@@ -73,7 +73,7 @@ def test_null_arguments_rejected_on_host(libple):
     wts.table = 17
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 3  # misaligned
     wts.table = 16
-    cfg.table_format = 3                          # no such format
+    cfg.table_format = 4                          # no such format
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
     cfg.table_format = ple.PLE_TABLE_E4M3_HEADS   # 16 head rows need row_dim % 256 == 0 ...
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 8
@@ -85,6 +85,10 @@ def test_null_arguments_rejected_on_host(libple):
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
     wts.block_scales = 24                         # ... 16-byte aligned
     assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 3
+    cfg.table_format = ple.PLE_TABLE_NVFP4_ROWS   # rows of row_dim * 9/16 bytes need row_dim % 256 == 0 ...
+    assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 8
+    cfg.row_dim = 256                             # ... and keep the block scales in the rows
+    assert libple.ple_create(ctypes.byref(cfg), ctypes.byref(wts), None, ctypes.byref(out)) == 1
     assert libple.ple_destroy(None) == 1
     assert libple.ple_forward(None, None, 0, None, 1, None, None, 0, None, None) == 1
     assert libple.ple_decode_step(None, None, 1, 1, None, None, 0, None, None, None, None) == 1
