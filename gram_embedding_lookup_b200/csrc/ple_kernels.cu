@@ -602,12 +602,10 @@ __global__ void __launch_bounds__(kIdsThreads) ids_meta_kernel(const PrepareArgs
   }
 }
 
-// Gather units of a token: E4M3 one 16-code chunk per thread (16 bytes from
-// each of the two rows); NVFP4 two chunks (16 bytes of packed codes and 2
-// block-scale bytes per row); the multi-head layout two consecutive chunks of
-// the token's head rows (32 bytes), so that every thread keeps about as many
-// bytes in flight as an E4M3 thread.
-template <int FMT> constexpr int kSplitChunksPerThread = FMT == 0 ? 1 : 2;
+// Gather units of a token: E4M3 and the multi-head layout one 16-code chunk per
+// thread; NVFP4 two chunks (16 bytes of packed codes and 2 block-scale bytes
+// per row), so that each load is as wide as an E4M3 thread's.
+template <int FMT> constexpr int kSplitChunksPerThread = FMT == 1 ? 2 : 1;
 
 template <int FMT>
 __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
@@ -630,45 +628,19 @@ __global__ void __launch_bounds__(kSplitThreads, kSplitBlocksPerSm)
   constexpr int CPT = kSplitChunksPerThread<FMT>;
   const int units = D / (16 * CPT);                              // per token
   const int64_t idx = (n_blocks - 1 - b) * kSplitThreads + threadIdx.x;
-  if constexpr (FMT == 2) {
-    // warp w takes the 64 chunks [64w, 64w + 64) of the batch's head rows (16 per
-    // token, side by side), lane l chunks 64w + l and 64w + l + 32: both loads in
-    // flight at once, each load instruction 32 consecutive chunks
-    const int hd = D / kHeads, cph = hd / 16, nck = D / 16;
-    const int64_t total = static_cast<int64_t>(a.T) * nck;
-    const int64_t g0 = (idx >> 5) * 64 + (threadIdx.x & 31);
-    if (g0 >= total) return;
-    uint4 v[2];
-    float sc[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t g = g0 + 32 * k;
-      if (g < total) {
-        const int32_t t = static_cast<int32_t>(g / nck);
-        const int c = static_cast<int>(g - static_cast<int64_t>(t) * nck), hh = c / cph;
-        const int64_t row = static_cast<int64_t>(hh) * a.rows0 + a.ids[static_cast<int64_t>(t) * kHeads + hh];
-        v[k] = ld_stream_v4(tab.codes + row * hd + (c - hh * cph) * 16);
-        sc[k] = __ldg(tab.scales + row);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t g = g0 + 32 * k;
-      if (g < total) {
-        uint4 o0, o1;
-        deq16_one(v[k], sc[k], o0, o1);
-        uint4* dst = reinterpret_cast<uint4*>(e + g * 16);
-        dst[0] = o0;
-        dst[1] = o1;
-      }
-    }
-    return;
-  }
   if (idx >= static_cast<int64_t>(a.T) * units) return;
   const int32_t t = static_cast<int32_t>(idx / units);
   const int c = static_cast<int>(idx - static_cast<int64_t>(t) * units);
   uint4* dst = reinterpret_cast<uint4*>(e + idx * 16 * CPT);
-  {
+  if constexpr (FMT == 2) {
+    const int hd = D / kHeads, cph = hd / 16, hh = c / cph;
+    const int64_t row = static_cast<int64_t>(hh) * a.rows0 + a.ids[static_cast<int64_t>(t) * kHeads + hh];
+    const uint4 v = ld_stream_v4(tab.codes + row * hd + (c - hh * cph) * 16);
+    uint4 o0, o1;
+    deq16_one(v, __ldg(tab.scales + row), o0, o1);
+    dst[0] = o0;
+    dst[1] = o1;
+  } else {
     const int2 id = reinterpret_cast<const int2*>(a.ids)[t];
     const int64_t row0 = id.x, row1 = a.rows0 + id.y;
     const float sa = __ldg(tab.scales + row0);
