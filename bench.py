@@ -506,7 +506,7 @@ def main():
             line["nvfp4"] = nvfp4_bench(ctx, w, sets, stream, peaks, ple.PLE_TABLE_NVFP4_ROWS)
             line["nvfp4"]["arrays_layout"] = arrays
         if "heads" in want:
-            line["heads"] = heads_bench(ctx, sets, stream, peaks)
+            line["heads"] = heads_bench(ctx, sets, stream, peaks, args.table_rows)
         if "prepared" in want:
             line["prepared"] = prepared_bench(ctx, layer, sets, stream)
         if "pipelined" in want:
@@ -847,13 +847,17 @@ def pipelined_bench(ctx, layer, sets, stream, steps=300):
             "device_status": int(status)}
 
 
-def heads_bench(ctx, sets, stream, peaks, steps=300):
+def heads_bench(ctx, sets, stream, peaks, table_rows=0, steps=300):
     """The multi-head row layout (PLE_TABLE_E4M3_HEADS: 16 lookups of 160-byte rows
     per token, 16 sub-tables of 20,000,096 rows, the same 51.2 GB): the headline
-    prefill batches and the 8 x 1 decode workload (a split-K step on this layout)."""
+    prefill batches and the 8 x 1 decode workload (a split-K step on this layout).
+    With table_rows > 0 (--table-rows) each head sub-table has 2 * table_rows rows,
+    the same bytes as a two-order table of table_rows rows per order."""
     torch, ple, pi = ctx["torch"], ctx["ple"], ctx["pi"]
     from ple_inputs.device import DeviceLayer
     w = pi.workload("heads_full")
+    if table_rows > 0:
+        w = pi.Workload(w.name, w.vocab, 2 * table_rows, w.row_dim, w.hidden, w.table_seed, w.seed, w.extra)
     R, D, H = w.rows_per_order, w.row_dim, w.hidden
     need = R * D + 16 * R * 4
     free, _ = torch.cuda.mem_get_info()
@@ -907,7 +911,7 @@ def heads_bench(ctx, sets, stream, peaks, steps=300):
     layer.close()
     world = ctx["world"]
     return {"workload": "full-scale prefill (the headline batches) and 8 x 1 decode on the multi-head table "
-                        "(16 x 20,000,096 rows x 160 codes)",
+                        f"(16 x {R:,} rows x 160 codes)",
             "table_bytes": int(need), "value": T * world * steps / (ms / 1e3), "unit": "tokens/s",
             "ms_per_step": ms / steps, "stage_ms_per_launch": {"embed": e_s * 1e3, "gemm": g_ms / max(g_n, 1)},
             "embed_roofline": {"bound": "hbm", "achieved": embed_bytes / e_s / 1e9, "peak": peaks["hbm_gbs"],
