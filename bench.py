@@ -909,6 +909,8 @@ def heads_bench(ctx, sets, stream, peaks, table_rows=0, steps=300):
     g_ms, g_n = stage["gemm"]
     status = ple.ple_get_error(h)
     layer.close()
+    del layer                                       # the table back to the device for the next line
+    torch.cuda.empty_cache()
     world = ctx["world"]
     return {"workload": "full-scale prefill (the headline batches) and 8 x 1 decode on the multi-head table "
                         f"(16 x {R:,} rows x 160 codes)",
@@ -988,6 +990,8 @@ def nvfp4_bench(ctx, w, sets, stream, peaks, fmt, steps=300):
 
     status = ple.ple_get_error(h)
     layer.close()
+    del layer                                       # the table back to the device for the next line
+    torch.cuda.empty_cache()
     world = ctx["world"]
     layout = ("rows: each row's 1,280 code bytes, then its 160 block-scale bytes" if rows
               else "arrays: codes [2][R][1280], block scales [2][R][160]")
